@@ -1,0 +1,193 @@
+/*
+ * slikl.h — C ABI of the B200 (sm_100a) sparse Lightning Indexer KL-loss backward.
+ *
+ * The operation is the one defined by aclnnSparseLightningIndexerKLLossGrad (Ascend
+ * CANN operator documentation, section "计算公式"). For each query token t:
+ *
+ *   S_t   = q_t . K_topk(t)^T          K_topk(t) = key rows named by sparse_indices[t]
+ *   I_t   = W_t . ReLU(S_t)            W = w
+ *   y_t   = Softmax(I_t)               over the valid slots; written to softmax_out
+ *   dI_t  = y_t - p_t                  p = attn_softmax_l1norm
+ *   dW_t  = dI_t . ReLU(S_t)^T         -> dw
+ *   dS_t  = dI_t * W_t * 1[S_t > 0]    (chain rule on I_t = W_t . ReLU(S_t))
+ *   dq_t  = dS_t . K_topk(t)           -> dq
+ *   dK_topk(t) = dS_t^T . q_t          scatter-added into the key rows -> dk
+ *
+ * Invalid top-k slots hold -1 and take no part ("无效top-k位置不参与计算"):
+ * softmax_out is exactly 0 there and nothing is added for them. A token with no valid
+ * slot gets softmax_out = 0 and zero dq/dw. Key rows that no valid slot names get dk = +0.
+ *
+ * The call sequence follows the page's two-phase interface (section "函数原型": first
+ * "...GetWorkspaceSize", which validates the parameters and returns the workspace size,
+ * then the asynchronous launch on a stream): slikl_grad_workspace_size(), then slikl_grad().
+ *
+ * Conventions for every entry point
+ *   - Ownership: the caller allocates every tensor and the workspace. The library
+ *     allocates no memory and keeps no state between calls.
+ *   - Pointers named "device" are CUDA device pointers on the current device; tensors are
+ *     dense and contiguous in the layouts stated below.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Launch-phase calls are
+ *     asynchronous: they return after queueing work on `stream`.
+ *   - Return codes mirror the aclnn convention (161001 parameter null pointer, 161002
+ *     parameter invalid, 561103 inner null pointer), plus two codes of this library.
+ */
+#ifndef SLIKL_H
+#define SLIKL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Entry points are the only symbols the shared library exports. */
+#if defined(__GNUC__)
+#define SLIKL_API __attribute__((visibility("default")))
+#else
+#define SLIKL_API
+#endif
+
+typedef int32_t slikl_status;
+
+#define SLIKL_OK                      0
+#define SLIKL_ERR_PARAM_NULLPTR       161001  /* a required pointer argument is NULL          */
+#define SLIKL_ERR_PARAM_INVALID       161002  /* dtype, layout, shape or attribute not supported */
+#define SLIKL_ERR_WORKSPACE_TOO_SMALL 161003  /* workspace_bytes below slikl_grad_workspace_size */
+#define SLIKL_ERR_INNER_NULLPTR       561103  /* the size/flags output pointer is NULL         */
+#define SLIKL_ERR_CUDA                561001  /* a CUDA runtime call or kernel launch failed   */
+
+/* dtype of q, k, dq, dk ("公共约束": the four share one dtype, FLOAT16 or BFLOAT16). */
+#define SLIKL_FP16 0
+#define SLIKL_BF16 1
+
+/* layoutQ / layoutK ("公共约束": BSND or TND; TND needs cuSeqLens of that side). */
+#define SLIKL_BSND 0
+#define SLIKL_TND  1
+
+/*
+ * Problem description (host memory).
+ *
+ *   layout_q = BSND: q [B,S1,N1,D], w/dw [B,S1,N1], sparse_indices, attn_softmax_l1norm and
+ *                    softmax_out [B,S1,1,topk]; requires B > 0 and S1 > 0; T1 is ignored
+ *                    (taken as B*S1).
+ *   layout_q = TND:  q [T1,N1,D], w/dw [T1,N1], the three top-k tensors [T1,1,topk];
+ *                    cu_seqlens_q [B+1] on the device with cu_seqlens_q[0] = 0 and
+ *                    cu_seqlens_q[B] = T1; S1 is ignored.
+ *   layout_k = BSND: k/dk [B,S2,1,D], requires S2 > 0; T2 is ignored (taken as B*S2).
+ *   layout_k = TND:  k/dk [T2,1,D], cu_seqlens_k [B+1] on the device, cu_seqlens_k[B] = T2.
+ *
+ * The key tensor has one head (N2 = 1): the page's formulas carry no key-head index.
+ * Valid indices of a batch-b token are local to batch b's key range: key row =
+ * (BSND) b*S2 + index, (TND) cu_seqlens_k[b] + index, and must lie in [0, len_k(b)).
+ *
+ * Supported set: N1 in [1, 128]; D in {64, 128}; topk in [1, 8192]; B >= 1;
+ * T1*topk < 2^31; T2 < 2^31. deterministic: 0 = dk by fp32 atomic adds (the page's default,
+ * section "确定性计算"), 1 = bitwise reproducible dk by a fixed-order reduction.
+ */
+typedef struct {
+    int32_t dtype;           /* SLIKL_FP16 or SLIKL_BF16 */
+    int32_t layout_q;        /* SLIKL_BSND or SLIKL_TND */
+    int32_t layout_k;        /* SLIKL_BSND or SLIKL_TND */
+    int32_t deterministic;   /* 0 or 1 */
+    int64_t B;               /* batches (TND: number of sequences = len(cu_seqlens) - 1) */
+    int64_t S1, S2;          /* BSND query / key lengths */
+    int64_t T1, T2;          /* TND total query / key rows */
+    int64_t N1, D, topk;     /* query heads, head dim, top-k slots per token */
+} slikl_problem;
+
+/* Tensors of one call. All DEVICE pointers, caller-owned, contiguous; q, k, dq, dk 16-byte
+ * aligned, the others 4-byte aligned (SLIKL_ERR_PARAM_INVALID otherwise). */
+typedef struct {
+    const void *q;                      /* dtype  [B,S1,N1,D] / [T1,N1,D]            */
+    const void *k;                      /* dtype  [B,S2,1,D]  / [T2,1,D]             */
+    const float *w;                     /* fp32   [B,S1,N1]   / [T1,N1]              */
+    const float *attn_softmax_l1norm;   /* fp32   [.., 1, topk] target distribution p  */
+    const int32_t *sparse_indices;      /* int32  [.., 1, topk], -1 = invalid slot     */
+    const int32_t *cu_seqlens_q;        /* int32  [B+1], TND query side only, else NULL */
+    const int32_t *cu_seqlens_k;        /* int32  [B+1], TND key side only, else NULL   */
+    void *dq;                           /* out dtype  same shape as q                  */
+    void *dk;                           /* out dtype  same shape as k                  */
+    float *dw;                          /* out fp32   same shape as w                  */
+    float *softmax_out;                 /* out fp32   same shape as sparse_indices     */
+} slikl_tensors;
+
+/*
+ * Phase 1 (host only, no CUDA call). Validates `problem` and writes the workspace size in
+ * bytes that slikl_grad needs.
+ * Errors: SLIKL_ERR_INNER_NULLPTR if workspace_bytes is NULL; SLIKL_ERR_PARAM_NULLPTR if
+ * problem is NULL; SLIKL_ERR_PARAM_INVALID for any value outside the supported set.
+ */
+SLIKL_API slikl_status slikl_grad_workspace_size(const slikl_problem *problem, size_t *workspace_bytes);
+
+/*
+ * Phase 2. Re-validates, then queues on `stream`: zeroing of the status word and of the
+ * fp32 dk accumulator, the work-split kernel, the fused per-token kernel, and (atomic mode)
+ * the dk cast or (deterministic mode) the key-major sort and fixed-order reduction.
+ * Writes dq, dk, dw and softmax_out in full.
+ * `workspace` (device, >= the phase-1 size, 256-byte aligned) is scratch owned by the
+ * caller for the duration of the call; its first 256 bytes hold the device status word
+ * read by slikl_read_device_status().
+ * Errors: SLIKL_ERR_PARAM_NULLPTR (problem, tensors, a required tensor pointer or
+ * workspace is NULL; cu_seqlens of a TND side is NULL), SLIKL_ERR_PARAM_INVALID,
+ * SLIKL_ERR_WORKSPACE_TOO_SMALL, SLIKL_ERR_CUDA (launch failure or no usable sm_100 device).
+ * Problems that only the device can see (an index outside its batch's key range, malformed
+ * cu_seqlens) never fault: the slot is treated as invalid and a bit is set in the status word.
+ */
+SLIKL_API slikl_status slikl_grad(const slikl_problem *problem, const slikl_tensors *tensors,
+                        void *workspace, size_t workspace_bytes, void *stream);
+
+/* Device status bits (see slikl_read_device_status). */
+#define SLIKL_DEV_INDEX_OUT_OF_RANGE  0x1u  /* some valid-looking index was >= len_k(b) or < -1 */
+#define SLIKL_DEV_BAD_CU_SEQLENS_Q    0x2u  /* cu_seqlens_q not 0..T1 non-decreasing           */
+#define SLIKL_DEV_BAD_CU_SEQLENS_K    0x4u  /* cu_seqlens_k not 0..T2 non-decreasing; the key
+                                               ranges of the batches were emptied            */
+#define SLIKL_DEV_WAIT_TIMEOUT        0x8u  /* an internal bounded wait gave up; outputs invalid */
+
+/*
+ * Copies the status word of the last slikl_grad call that used `workspace` (device) into
+ * *flags (host) after synchronising `stream`. Bits are the SLIKL_DEV_* values above.
+ * Errors: SLIKL_ERR_PARAM_NULLPTR (workspace NULL), SLIKL_ERR_INNER_NULLPTR (flags NULL),
+ * SLIKL_ERR_CUDA.
+ */
+SLIKL_API slikl_status slikl_read_device_status(const void *workspace, void *stream, uint32_t *flags);
+
+/*
+ * Work split ("metadata"), the analogue of DenseLightningIndexerKLLossGradMetadata (article
+ * on that AICPU operator, sections "功能定位" and "Metadata 输出布局"): the merged B*S1 query
+ * rows are split into contiguous ranges, one per worker (CTA) of the fused kernel.
+ * slikl_grad runs the same kernel into its workspace; this entry point exposes it.
+ *
+ * metadata (device, int32, slikl_grad_metadata_size(num_workers) entries) receives:
+ *   [0] totalSize      merged query rows T1
+ *   [1] formerCoreSize ceil(T1 / num_workers)
+ *   [2] remainCoreSize formerCoreSize - 1 (0 if T1 == 0)
+ *   [3] remainCoreNum  workers that take remainCoreSize rows in the row-count split
+ *   [4] usedCoreNum    min(num_workers, T1)
+ *   [5] maxSeqK        longest key range of a batch
+ *   [6] mode           0 = row-count split (the page's), 1 = cost-weighted split
+ *   [7] num_workers
+ *   [8 + 2c], [9 + 2c] first and one-past-last query row of worker c.
+ * Fields 0..5 follow the page's layout; the page's fixed 64-entry size is not kept, since
+ * the ranges of every worker are stored. In mode 1 the ranges balance
+ * cost(t) = 1 + (number of 128-slot tiles of row t holding an index >= 0).
+ * `tensors` needs sparse_indices and, for TND sides, cu_seqlens_q/k; other fields ignored.
+ * `workspace` (device, >= slikl_grad_metadata_workspace_size bytes) is scratch.
+ * Errors: as slikl_grad; SLIKL_ERR_PARAM_INVALID if num_workers is not in [1, 4096] or
+ * mode is not 0/1.
+ */
+SLIKL_API int64_t slikl_grad_metadata_size(int32_t num_workers);
+SLIKL_API slikl_status slikl_grad_metadata_workspace_size(const slikl_problem *problem,
+                                                size_t *workspace_bytes);
+SLIKL_API slikl_status slikl_grad_metadata(const slikl_problem *problem, const slikl_tensors *tensors,
+                                 int32_t num_workers, int32_t mode, int32_t *metadata,
+                                 void *workspace, size_t workspace_bytes, void *stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+SLIKL_API const char *slikl_status_string(slikl_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SLIKL_H */

@@ -1,0 +1,226 @@
+"""Python binding of the sm_100a sparse Lightning Indexer KL-loss backward library.
+
+Argument marshalling only: every step of the operator runs in the CUDA kernels of
+``libslikl.so`` behind the C ABI declared in ``include/slikl.h``. The functions here keep
+the C names (``slikl_grad_workspace_size``, ``slikl_grad``, ...) and take ctypes structs;
+``grad()`` is a convenience wrapper that allocates outputs and the workspace with torch and
+calls through the same ABI. There is no CPU fallback: if the library is missing or no
+sm_100 device is present the calls raise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libslikl.so")
+
+SLIKL_OK = 0
+SLIKL_ERR_PARAM_NULLPTR = 161001
+SLIKL_ERR_PARAM_INVALID = 161002
+SLIKL_ERR_WORKSPACE_TOO_SMALL = 161003
+SLIKL_ERR_INNER_NULLPTR = 561103
+SLIKL_ERR_CUDA = 561001
+
+SLIKL_FP16 = 0
+SLIKL_BF16 = 1
+SLIKL_BSND = 0
+SLIKL_TND = 1
+
+SLIKL_DEV_INDEX_OUT_OF_RANGE = 0x1
+SLIKL_DEV_BAD_CU_SEQLENS_Q = 0x2
+SLIKL_DEV_BAD_CU_SEQLENS_K = 0x4
+SLIKL_DEV_WAIT_TIMEOUT = 0x8
+
+EXPORTED = ("slikl_grad_workspace_size", "slikl_grad", "slikl_read_device_status",
+            "slikl_grad_metadata_size", "slikl_grad_metadata_workspace_size",
+            "slikl_grad_metadata", "slikl_status_string")
+
+
+class slikl_problem(ctypes.Structure):
+    _fields_ = [("dtype", ctypes.c_int32), ("layout_q", ctypes.c_int32),
+                ("layout_k", ctypes.c_int32), ("deterministic", ctypes.c_int32),
+                ("B", ctypes.c_int64), ("S1", ctypes.c_int64), ("S2", ctypes.c_int64),
+                ("T1", ctypes.c_int64), ("T2", ctypes.c_int64), ("N1", ctypes.c_int64),
+                ("D", ctypes.c_int64), ("topk", ctypes.c_int64)]
+
+
+class slikl_tensors(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_void_p) for name in
+                ("q", "k", "w", "attn_softmax_l1norm", "sparse_indices", "cu_seqlens_q",
+                 "cu_seqlens_k", "dq", "dk", "dw", "softmax_out")]
+
+
+class SliklError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {status_string(code)} ({code})")
+
+
+_lib = None
+
+
+def load_library() -> ctypes.CDLL:
+    """Load libslikl.so (built by sparse_lightning_indexer_b200.build). Raises if missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run python -m sparse_lightning_indexer_b200.build")
+        lib = ctypes.CDLL(LIB_PATH)
+        P, VP = ctypes.POINTER, ctypes.c_void_p
+        lib.slikl_grad_workspace_size.argtypes = [P(slikl_problem), P(ctypes.c_size_t)]
+        lib.slikl_grad.argtypes = [P(slikl_problem), P(slikl_tensors), VP, ctypes.c_size_t, VP]
+        lib.slikl_read_device_status.argtypes = [VP, VP, P(ctypes.c_uint32)]
+        lib.slikl_grad_metadata_size.argtypes = [ctypes.c_int32]
+        lib.slikl_grad_metadata_size.restype = ctypes.c_int64
+        lib.slikl_grad_metadata_workspace_size.argtypes = [P(slikl_problem), P(ctypes.c_size_t)]
+        lib.slikl_grad_metadata.argtypes = [P(slikl_problem), P(slikl_tensors), ctypes.c_int32,
+                                            ctypes.c_int32, VP, VP, ctypes.c_size_t, VP]
+        lib.slikl_status_string.argtypes = [ctypes.c_int32]
+        lib.slikl_status_string.restype = ctypes.c_char_p
+        for name in ("slikl_grad_workspace_size", "slikl_grad", "slikl_read_device_status",
+                     "slikl_grad_metadata_workspace_size", "slikl_grad_metadata"):
+            getattr(lib, name).restype = ctypes.c_int32
+        _lib = lib
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return load_library().slikl_status_string(int(code)).decode()
+
+
+# --- C names, marshalling only -------------------------------------------------------
+
+def slikl_grad_workspace_size(problem: slikl_problem) -> int:
+    n = ctypes.c_size_t(0)
+    rc = load_library().slikl_grad_workspace_size(ctypes.byref(problem), ctypes.byref(n))
+    if rc != SLIKL_OK:
+        raise SliklError(rc, "slikl_grad_workspace_size")
+    return int(n.value)
+
+
+def slikl_grad(problem: slikl_problem, tensors: slikl_tensors, workspace: int,
+               workspace_bytes: int, stream: int = 0) -> None:
+    rc = load_library().slikl_grad(ctypes.byref(problem), ctypes.byref(tensors), workspace,
+                                   workspace_bytes, stream)
+    if rc != SLIKL_OK:
+        raise SliklError(rc, "slikl_grad")
+
+
+def slikl_read_device_status(workspace: int, stream: int = 0) -> int:
+    flags = ctypes.c_uint32(0)
+    rc = load_library().slikl_read_device_status(workspace, stream, ctypes.byref(flags))
+    if rc != SLIKL_OK:
+        raise SliklError(rc, "slikl_read_device_status")
+    return int(flags.value)
+
+
+def slikl_grad_metadata_size(num_workers: int) -> int:
+    return int(load_library().slikl_grad_metadata_size(num_workers))
+
+
+def slikl_grad_metadata_workspace_size(problem: slikl_problem) -> int:
+    n = ctypes.c_size_t(0)
+    rc = load_library().slikl_grad_metadata_workspace_size(ctypes.byref(problem), ctypes.byref(n))
+    if rc != SLIKL_OK:
+        raise SliklError(rc, "slikl_grad_metadata_workspace_size")
+    return int(n.value)
+
+
+def slikl_grad_metadata(problem: slikl_problem, tensors: slikl_tensors, num_workers: int,
+                        mode: int, metadata: int, workspace: int, workspace_bytes: int,
+                        stream: int = 0) -> None:
+    rc = load_library().slikl_grad_metadata(ctypes.byref(problem), ctypes.byref(tensors),
+                                            num_workers, mode, metadata, workspace,
+                                            workspace_bytes, stream)
+    if rc != SLIKL_OK:
+        raise SliklError(rc, "slikl_grad_metadata")
+
+
+# --- torch convenience ------------------------------------------------------------------
+
+_DT = {torch.bfloat16: SLIKL_BF16, torch.float16: SLIKL_FP16}
+
+
+def make_problem(q: torch.Tensor, k: torch.Tensor, sparse_indices: torch.Tensor,
+                 layout_q: str = "BSND", layout_k: str = "BSND", deterministic: bool = False,
+                 B: Optional[int] = None) -> slikl_problem:
+    """Problem struct from tensor shapes (BSND q [B,S1,N1,D]; TND q [T1,N1,D])."""
+    pr = slikl_problem()
+    if q.dtype not in _DT or k.dtype != q.dtype:
+        raise ValueError("q and k must share dtype float16 or bfloat16")
+    pr.dtype = _DT[q.dtype]
+    pr.layout_q = SLIKL_BSND if layout_q == "BSND" else SLIKL_TND
+    pr.layout_k = SLIKL_BSND if layout_k == "BSND" else SLIKL_TND
+    pr.deterministic = 1 if deterministic else 0
+    if layout_q == "BSND":
+        pr.B, pr.S1, pr.N1, pr.D = q.shape
+        pr.T1 = pr.B * pr.S1
+    else:
+        pr.T1, pr.N1, pr.D = q.shape
+        if B is None:
+            raise ValueError("TND needs B (len(cu_seqlens) - 1)")
+        pr.B = B
+    if layout_k == "BSND":
+        pr.S2 = k.shape[1]
+        pr.T2 = k.shape[0] * k.shape[1]
+    else:
+        pr.T2 = k.shape[0]
+    pr.topk = sparse_indices.shape[-1]
+    return pr
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError("tensors must be contiguous CUDA tensors")
+    return t.data_ptr()
+
+
+def grad(q, k, w, attn_softmax_l1norm, sparse_indices, layout_q="BSND", layout_k="BSND",
+         cu_seqlens_q=None, cu_seqlens_k=None, deterministic=False, stream=None, out=None,
+         workspace=None):
+    """Run slikl_grad on CUDA tensors. Returns dict(dq, dk, dw, softmax_out, workspace).
+
+    `out` may supply preallocated dq/dk/dw/softmax_out, `workspace` a uint8 CUDA buffer.
+    """
+    B = None
+    if layout_q == "TND":
+        B = cu_seqlens_q.numel() - 1
+    elif layout_k == "TND":
+        B = cu_seqlens_k.numel() - 1
+    pr = make_problem(q, k, sparse_indices, layout_q, layout_k, deterministic, B)
+    nbytes = slikl_grad_workspace_size(pr)
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k),
+                   dw=torch.empty_like(w), softmax_out=torch.empty_like(attn_softmax_l1norm))
+    tn = slikl_tensors()
+    tn.q, tn.k, tn.w = _ptr(q), _ptr(k), _ptr(w)
+    tn.attn_softmax_l1norm = _ptr(attn_softmax_l1norm)
+    tn.sparse_indices = _ptr(sparse_indices)
+    tn.cu_seqlens_q = _ptr(cu_seqlens_q) if layout_q == "TND" else None
+    tn.cu_seqlens_k = _ptr(cu_seqlens_k) if layout_k == "TND" else None
+    tn.dq, tn.dk, tn.dw = _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dw"])
+    tn.softmax_out = _ptr(out["softmax_out"])
+    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+    slikl_grad(pr, tn, workspace.data_ptr(), workspace.numel(), s.cuda_stream)
+    res = dict(out)
+    res["workspace"] = workspace
+    return res
+
+
+def grad_workload(wl, device="cuda", deterministic=False, stream=None):
+    """Move a slikl_inputs.Workload to the device and run grad()."""
+    dev = torch.device(device)
+    t = {n: getattr(wl, n).to(dev) for n in ("q", "k", "w", "p", "idx")}
+    cuq = wl.cu_seqlens_q.to(dev) if wl.cu_seqlens_q is not None else None
+    cuk = wl.cu_seqlens_k.to(dev) if wl.cu_seqlens_k is not None else None
+    return grad(t["q"], t["k"], t["w"], t["p"], t["idx"], wl.layout, wl.layout, cuq, cuk,
+                deterministic=deterministic, stream=stream)

@@ -1,0 +1,235 @@
+// C ABI of the library (declarations and contract in include/slikl.h).
+//
+// Two-phase call, after aclnnSparseLightningIndexerKLLossGrad ("函数原型": a first call that
+// validates the parameters and returns the workspace size, then the launch on a stream).
+// Validation follows the page's constraints ("公共约束" and "规格约束") restricted to what
+// this sm_100a build supports.
+#include <string.h>
+
+#include "slikl_common.cuh"
+
+namespace slikl {
+
+cudaError_t launch_fused_sm100(const Params &P, int workers, cudaStream_t s, bool *handled);
+
+namespace {
+
+struct Derived {
+    int64_t T1, T2;
+};
+
+slikl_status validate(const slikl_problem *pr, Derived *out) {
+    if (!pr) return SLIKL_ERR_PARAM_NULLPTR;
+    if (pr->dtype != SLIKL_FP16 && pr->dtype != SLIKL_BF16) return SLIKL_ERR_PARAM_INVALID;
+    if (pr->layout_q != SLIKL_BSND && pr->layout_q != SLIKL_TND) return SLIKL_ERR_PARAM_INVALID;
+    if (pr->layout_k != SLIKL_BSND && pr->layout_k != SLIKL_TND) return SLIKL_ERR_PARAM_INVALID;
+    if (pr->deterministic != 0 && pr->deterministic != 1) return SLIKL_ERR_PARAM_INVALID;
+    if (pr->B < 1 || pr->B > (int64_t(1) << 30)) return SLIKL_ERR_PARAM_INVALID;
+    if (pr->N1 < 1 || pr->N1 > 128) return SLIKL_ERR_PARAM_INVALID;
+    if (pr->D != 64 && pr->D != 128) return SLIKL_ERR_PARAM_INVALID;
+    if (pr->topk < 1 || pr->topk > 8192) return SLIKL_ERR_PARAM_INVALID;
+    int64_t T1, T2;
+    if (pr->layout_q == SLIKL_BSND) {
+        if (pr->S1 < 1) return SLIKL_ERR_PARAM_INVALID;
+        T1 = pr->B * pr->S1;
+    } else {
+        if (pr->T1 < 0) return SLIKL_ERR_PARAM_INVALID;
+        T1 = pr->T1;
+    }
+    if (pr->layout_k == SLIKL_BSND) {
+        if (pr->S2 < 1) return SLIKL_ERR_PARAM_INVALID;
+        T2 = pr->B * pr->S2;
+    } else {
+        if (pr->T2 < 0) return SLIKL_ERR_PARAM_INVALID;
+        T2 = pr->T2;
+    }
+    if (T1 * pr->topk >= (int64_t(1) << 31) || T2 >= (int64_t(1) << 31) - 2)
+        return SLIKL_ERR_PARAM_INVALID;
+    out->T1 = T1;
+    out->T2 = T2;
+    return SLIKL_OK;
+}
+
+int current_sm_count(bool *ok) {
+    int dev = 0, major = 0, sms = 0;
+    *ok = cudaGetDevice(&dev) == cudaSuccess &&
+          cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) == cudaSuccess &&
+          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+          major == 10;
+    return sms;
+}
+
+Params make_params(const slikl_problem *pr, const Derived &dv, const slikl_tensors *tn,
+                   void *ws) {
+    Params P{};
+    P.dtype = pr->dtype;
+    P.layout_q = pr->layout_q;
+    P.layout_k = pr->layout_k;
+    P.deterministic = pr->deterministic;
+    P.B = pr->B;
+    P.S1 = pr->layout_q == SLIKL_BSND ? pr->S1 : 0;
+    P.S2 = pr->layout_k == SLIKL_BSND ? pr->S2 : 0;
+    P.T1 = dv.T1;
+    P.T2 = dv.T2;
+    P.N1 = (int)pr->N1;
+    P.D = (int)pr->D;
+    P.K = (int)pr->topk;
+    if (tn) {
+        P.q = tn->q; P.k = tn->k; P.w = tn->w; P.p = tn->attn_softmax_l1norm;
+        P.idx = tn->sparse_indices; P.cu_q = tn->cu_seqlens_q; P.cu_k = tn->cu_seqlens_k;
+        P.dq = tn->dq; P.dk = tn->dk; P.dw = tn->dw; P.y = tn->softmax_out;
+    }
+    WsLayout L = make_layout(dv.T1, dv.T2, pr->topk, pr->D, pr->deterministic);
+    char *base = static_cast<char *>(ws);
+    P.status = reinterpret_cast<uint32_t *>(base + L.status);
+    P.meta = reinterpret_cast<int32_t *>(base + L.meta);
+    P.tok_kbase = reinterpret_cast<int32_t *>(base + L.tok_kbase);
+    P.tok_klen = reinterpret_cast<int32_t *>(base + L.tok_klen);
+    P.tok_cost = reinterpret_cast<int32_t *>(base + L.tok_cost);
+    P.cost_prefix = reinterpret_cast<int64_t *>(base + L.cost_prefix);
+    P.dk_acc = reinterpret_cast<float *>(base + L.dk_acc);
+    P.partials = reinterpret_cast<float *>(base + L.partials);
+    P.keys0 = reinterpret_cast<int32_t *>(base + L.keys0);
+    P.vals0 = reinterpret_cast<int32_t *>(base + L.vals0);
+    P.keys1 = reinterpret_cast<int32_t *>(base + L.keys1);
+    P.vals1 = reinterpret_cast<int32_t *>(base + L.vals1);
+    P.hist = reinterpret_cast<int32_t *>(base + L.hist);
+    P.row_ptr = reinterpret_cast<int32_t *>(base + L.row_ptr);
+    return P;
+}
+
+slikl_status check_tensors(const slikl_problem *pr, const slikl_tensors *tn, bool need_all) {
+    if (!tn) return SLIKL_ERR_PARAM_NULLPTR;
+    if (!tn->sparse_indices) return SLIKL_ERR_PARAM_NULLPTR;
+    if (pr->layout_q == SLIKL_TND && !tn->cu_seqlens_q) return SLIKL_ERR_PARAM_NULLPTR;
+    if (pr->layout_k == SLIKL_TND && !tn->cu_seqlens_k) return SLIKL_ERR_PARAM_NULLPTR;
+    if (need_all && (!tn->q || !tn->k || !tn->w || !tn->attn_softmax_l1norm || !tn->dq ||
+                     !tn->dk || !tn->dw || !tn->softmax_out))
+        return SLIKL_ERR_PARAM_NULLPTR;
+    // 16-byte vector loads/stores of q, k, dq, dk rows; 4-byte elements elsewhere
+    auto mis = [](const void *p, uintptr_t a) { return p && (reinterpret_cast<uintptr_t>(p) & (a - 1)); };
+    if (mis(tn->q, 16) || mis(tn->k, 16) || mis(tn->dq, 16) || mis(tn->dk, 16) ||
+        mis(tn->w, 4) || mis(tn->attn_softmax_l1norm, 4) || mis(tn->sparse_indices, 4) ||
+        mis(tn->cu_seqlens_q, 4) || mis(tn->cu_seqlens_k, 4) || mis(tn->dw, 4) ||
+        mis(tn->softmax_out, 4))
+        return SLIKL_ERR_PARAM_INVALID;
+    return SLIKL_OK;
+}
+
+}  // namespace
+}  // namespace slikl
+
+using namespace slikl;
+
+extern "C" {
+
+slikl_status slikl_grad_workspace_size(const slikl_problem *problem, size_t *workspace_bytes) {
+    if (!workspace_bytes) return SLIKL_ERR_INNER_NULLPTR;
+    Derived dv;
+    slikl_status st = validate(problem, &dv);
+    if (st != SLIKL_OK) return st;
+    *workspace_bytes = make_layout(dv.T1, dv.T2, problem->topk, problem->D,
+                                   problem->deterministic).total;
+    return SLIKL_OK;
+}
+
+slikl_status slikl_grad(const slikl_problem *problem, const slikl_tensors *tensors,
+                        void *workspace, size_t workspace_bytes, void *stream) {
+    Derived dv;
+    slikl_status st = validate(problem, &dv);
+    if (st != SLIKL_OK) return st;
+    st = check_tensors(problem, tensors, true);
+    if (st != SLIKL_OK) return st;
+    if (!workspace) return SLIKL_ERR_PARAM_NULLPTR;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255) return SLIKL_ERR_PARAM_INVALID;
+    WsLayout L = make_layout(dv.T1, dv.T2, problem->topk, problem->D, problem->deterministic);
+    if (workspace_bytes < L.total) return SLIKL_ERR_WORKSPACE_TOO_SMALL;
+    bool ok = false;
+    int sms = current_sm_count(&ok);
+    if (!ok) return SLIKL_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    Params P = make_params(problem, dv, tensors, workspace);
+
+    const int workers = sms < kMaxWorkers ? sms : kMaxWorkers;
+    if (cudaMemsetAsync(P.status, 0, 256, s) != cudaSuccess) return SLIKL_ERR_CUDA;
+    if (!P.deterministic && dv.T2 > 0 &&
+        cudaMemsetAsync(P.dk_acc, 0, sizeof(float) * (size_t)dv.T2 * problem->D, s) != cudaSuccess)
+        return SLIKL_ERR_CUDA;
+    if (launch_metadata(P, workers, 1, s) != cudaSuccess) return SLIKL_ERR_CUDA;
+    if (dv.T1 > 0) {
+        bool handled = false;
+        if (launch_fused_sm100(P, workers, s, &handled) != cudaSuccess) return SLIKL_ERR_CUDA;
+        if (!handled && launch_fused_simt(P, workers, s) != cudaSuccess) return SLIKL_ERR_CUDA;
+    }
+    cudaError_t e = P.deterministic ? launch_deterministic_reduce(P, s) : launch_cast(P, s);
+    return e == cudaSuccess ? SLIKL_OK : SLIKL_ERR_CUDA;
+}
+
+slikl_status slikl_read_device_status(const void *workspace, void *stream, uint32_t *flags) {
+    if (!flags) return SLIKL_ERR_INNER_NULLPTR;
+    if (!workspace) return SLIKL_ERR_PARAM_NULLPTR;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t v = 0;
+    if (cudaMemcpyAsync(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return SLIKL_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return SLIKL_ERR_CUDA;
+    *flags = v;
+    return SLIKL_OK;
+}
+
+int64_t slikl_grad_metadata_size(int32_t num_workers) {
+    if (num_workers < 1 || num_workers > kMaxWorkers) return -1;
+    return kMetaHeader + 2 * (int64_t)num_workers;
+}
+
+slikl_status slikl_grad_metadata_workspace_size(const slikl_problem *problem,
+                                                size_t *workspace_bytes) {
+    if (!workspace_bytes) return SLIKL_ERR_INNER_NULLPTR;
+    Derived dv;
+    slikl_status st = validate(problem, &dv);
+    if (st != SLIKL_OK) return st;
+    // the metadata kernels touch the regions up to and including cost_prefix
+    *workspace_bytes = make_layout(dv.T1, dv.T2, problem->topk, problem->D, 1).dk_acc;
+    return SLIKL_OK;
+}
+
+slikl_status slikl_grad_metadata(const slikl_problem *problem, const slikl_tensors *tensors,
+                                 int32_t num_workers, int32_t mode, int32_t *metadata,
+                                 void *workspace, size_t workspace_bytes, void *stream) {
+    Derived dv;
+    slikl_status st = validate(problem, &dv);
+    if (st != SLIKL_OK) return st;
+    st = check_tensors(problem, tensors, false);
+    if (st != SLIKL_OK) return st;
+    if (!metadata || !workspace) return SLIKL_ERR_PARAM_NULLPTR;
+    if (num_workers < 1 || num_workers > kMaxWorkers || (mode != 0 && mode != 1))
+        return SLIKL_ERR_PARAM_INVALID;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255) return SLIKL_ERR_PARAM_INVALID;
+    size_t need = make_layout(dv.T1, dv.T2, problem->topk, problem->D, 1).dk_acc;
+    if (workspace_bytes < need) return SLIKL_ERR_WORKSPACE_TOO_SMALL;
+    bool ok = false;
+    current_sm_count(&ok);
+    if (!ok) return SLIKL_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    Params P = make_params(problem, dv, tensors, workspace);
+    if (cudaMemsetAsync(P.status, 0, 256, s) != cudaSuccess) return SLIKL_ERR_CUDA;
+    if (launch_metadata(P, num_workers, mode, s) != cudaSuccess) return SLIKL_ERR_CUDA;
+    size_t bytes = sizeof(int32_t) * (size_t)(kMetaHeader + 2 * num_workers);
+    if (cudaMemcpyAsync(metadata, P.meta, bytes, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return SLIKL_ERR_CUDA;
+    return SLIKL_OK;
+}
+
+const char *slikl_status_string(slikl_status status) {
+    switch (status) {
+        case SLIKL_OK: return "SLIKL_OK";
+        case SLIKL_ERR_PARAM_NULLPTR: return "SLIKL_ERR_PARAM_NULLPTR: a required pointer is NULL";
+        case SLIKL_ERR_PARAM_INVALID: return "SLIKL_ERR_PARAM_INVALID: parameter outside the supported set";
+        case SLIKL_ERR_WORKSPACE_TOO_SMALL: return "SLIKL_ERR_WORKSPACE_TOO_SMALL: workspace below the phase-1 size";
+        case SLIKL_ERR_INNER_NULLPTR: return "SLIKL_ERR_INNER_NULLPTR: output pointer is NULL";
+        case SLIKL_ERR_CUDA: return "SLIKL_ERR_CUDA: CUDA runtime error or no sm_100 device";
+        default: return "unknown slikl status";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,122 @@
+// Shared definitions of the CUDA library: problem parameters as the kernels see them,
+// the workspace layout, device status bits and small device helpers.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "slikl.h"
+
+namespace slikl {
+
+constexpr int kMaxWorkers = 4096;        // metadata capacity (workers = CTAs of the fused kernel)
+constexpr int kSlotTile = 128;           // top-k slots per tile of the fused kernel
+constexpr int kMetaHeader = 8;
+
+// Everything a kernel needs about one call. Built on the host, passed by value.
+struct Params {
+    int dtype;            // SLIKL_FP16 / SLIKL_BF16
+    int layout_q, layout_k;
+    int deterministic;
+    int64_t B, S1, S2;    // BSND lengths (0 when that side is TND)
+    int64_t T1, T2;       // total query / key rows
+    int N1, D, K;         // heads, head dim, top-k
+    const void *q, *k;
+    const float *w, *p;
+    const int32_t *idx, *cu_q, *cu_k;
+    void *dq, *dk;
+    float *dw, *y;
+    // workspace regions
+    uint32_t *status;     // device status word(s)
+    int32_t *meta;        // [kMetaHeader + 2*workers]
+    int32_t *tok_kbase;   // [T1] first key row of the token's batch
+    int32_t *tok_klen;    // [T1] key count of the token's batch
+    int32_t *tok_cost;    // [T1] work estimate per token
+    int64_t *cost_prefix; // [T1 + 1]
+    float *dk_acc;        // [T2*D] fp32 accumulator (atomic mode)
+    float *partials;      // [T1*K*D] per-slot dK rows (deterministic mode)
+    int32_t *keys0, *vals0, *keys1, *vals1;   // radix-sort buffers [T1*K]
+    int32_t *hist;        // [256 * sort_blocks]
+    int32_t *row_ptr;     // [T2 + 2]
+};
+
+// Byte offsets of the workspace regions; every region starts 256-byte aligned.
+struct WsLayout {
+    size_t status, meta, tok_kbase, tok_klen, tok_cost, cost_prefix;
+    size_t dk_acc, partials, keys0, vals0, keys1, vals1, hist, row_ptr;
+    size_t total;
+};
+
+constexpr int kSortTile = 4096;          // elements per block of one radix-sort pass
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline WsLayout make_layout(int64_t T1, int64_t T2, int64_t K, int64_t D, int det) {
+    WsLayout L{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
+    L.status = take(256);
+    L.meta = take(sizeof(int32_t) * (kMetaHeader + 2 * kMaxWorkers));
+    L.tok_kbase = take(sizeof(int32_t) * (size_t)T1);
+    L.tok_klen = take(sizeof(int32_t) * (size_t)T1);
+    L.tok_cost = take(sizeof(int32_t) * (size_t)T1);
+    L.cost_prefix = take(sizeof(int64_t) * (size_t)(T1 + 1));
+    L.dk_acc = take(det ? 0 : sizeof(float) * (size_t)T2 * (size_t)D);
+    size_t n = (size_t)T1 * (size_t)K;
+    size_t sort_blocks = (n + kSortTile - 1) / kSortTile;
+    L.partials = take(det ? sizeof(float) * n * (size_t)D : 0);
+    L.keys0 = take(det ? sizeof(int32_t) * n : 0);
+    L.vals0 = take(det ? sizeof(int32_t) * n : 0);
+    L.keys1 = take(det ? sizeof(int32_t) * n : 0);
+    L.vals1 = take(det ? sizeof(int32_t) * n : 0);
+    L.hist = take(det ? sizeof(int32_t) * 256 * sort_blocks : 0);
+    L.row_ptr = take(det ? sizeof(int32_t) * (size_t)(T2 + 2) : 0);
+    L.total = off;
+    return L;
+}
+
+// status word layout: status[0] = SLIKL_DEV_* bits; status[1] = 1 when cu_seqlens_k is
+// unusable (every batch's key range is then empty); status[2..] reserved.
+
+__device__ __forceinline__ void set_status(uint32_t *status, uint32_t bit) {
+    atomicOr(status, bit);
+}
+
+__device__ __forceinline__ float load_as_float(const void *base, size_t i, int dtype) {
+    if (dtype == SLIKL_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(base)[i]);
+    return __half2float(reinterpret_cast<const __half *>(base)[i]);
+}
+
+__device__ __forceinline__ void store_from_float(void *base, size_t i, float v, int dtype) {
+    if (dtype == SLIKL_BF16) reinterpret_cast<__nv_bfloat16 *>(base)[i] = __float2bfloat16_rn(v);
+    else reinterpret_cast<__half *>(base)[i] = __float2half_rn(v);
+}
+
+__device__ __forceinline__ void red_add_f32(float *addr, float v) {
+    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
+}
+
+__device__ __forceinline__ void red_add_v4_f32(float *addr, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
+                 "f"(c), "f"(d)
+                 : "memory");
+}
+
+// Key row of slot value v for a token whose batch keys are [kbase, kbase + klen), or -1.
+// Values outside [-1, klen) break the index contract: they are flagged and treated as invalid.
+__device__ __forceinline__ int32_t slot_row(int32_t v, int32_t kbase, int32_t klen,
+                                            uint32_t *status) {
+    if (v >= 0 && v < klen) return kbase + v;
+    if (v != -1) set_status(status, SLIKL_DEV_INDEX_OUT_OF_RANGE);
+    return -1;
+}
+
+// kernels (defined in the .cu files)
+cudaError_t launch_metadata(const Params &P, int workers, int mode, cudaStream_t s);
+cudaError_t launch_fused_simt(const Params &P, int workers, cudaStream_t s);
+cudaError_t launch_cast(const Params &P, cudaStream_t s);
+cudaError_t launch_deterministic_reduce(const Params &P, cudaStream_t s);
+
+}  // namespace slikl

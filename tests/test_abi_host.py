@@ -1,0 +1,146 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry point that
+include/slikl.h declares, and phase 1 validates parameters per the operator's constraints
+(aclnnSparseLightningIndexerKLLossGrad, "公共约束" / "规格约束"; return codes after the aclnn
+convention). No compute call runs here."""
+
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import sparse_lightning_indexer_b200 as sli
+from sparse_lightning_indexer_b200 import build as slibuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    slibuild.build()
+    return sli.load_library()
+
+
+def declared_symbols():
+    with open(os.path.join(ROOT, "include", "slikl.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"SLIKL_API\s+[\w\s\*]+?\b(slikl_\w+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_symbols()
+    assert len(names) >= 7
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(sli.EXPORTED) == names
+
+
+def base_problem(**kw):
+    pr = sli.slikl_problem()
+    pr.dtype, pr.layout_q, pr.layout_k, pr.deterministic = sli.SLIKL_BF16, sli.SLIKL_BSND, sli.SLIKL_BSND, 0
+    pr.B, pr.S1, pr.S2, pr.T1, pr.T2, pr.N1, pr.D, pr.topk = 1, 4096, 4096, 0, 0, 64, 128, 2048
+    for k, v in kw.items():
+        setattr(pr, k, v)
+    return pr
+
+
+def ws_rc(lib, pr):
+    n = ctypes.c_size_t(0)
+    return lib.slikl_grad_workspace_size(ctypes.byref(pr), ctypes.byref(n)), n.value
+
+
+def test_workspace_size_valid(lib):
+    rc, n = ws_rc(lib, base_problem())
+    assert rc == sli.SLIKL_OK
+    # fp32 dk accumulator alone is T2*D*4 bytes
+    assert n >= 4096 * 128 * 4
+    rc, n_det = ws_rc(lib, base_problem(deterministic=1))
+    assert rc == sli.SLIKL_OK
+    assert n_det >= 4096 * 2048 * 128 * 4       # one fp32 dK row per slot
+
+
+@pytest.mark.parametrize("field,value", [
+    ("dtype", 2), ("layout_q", 2), ("layout_k", -1), ("deterministic", 2), ("B", 0),
+    ("N1", 0), ("N1", 129), ("D", 96), ("D", 256), ("topk", 0), ("topk", 8193), ("S1", 0),
+    ("S2", 0),
+])
+def test_workspace_size_rejects(lib, field, value):
+    rc, _ = ws_rc(lib, base_problem(**{field: value}))
+    assert rc == sli.SLIKL_ERR_PARAM_INVALID
+
+
+def test_tnd_sizes(lib):
+    pr = base_problem(layout_q=sli.SLIKL_TND, layout_k=sli.SLIKL_TND, B=8, S1=0, S2=0,
+                      T1=35000, T2=35000, N1=32)
+    assert ws_rc(lib, pr)[0] == sli.SLIKL_OK
+    assert ws_rc(lib, base_problem(layout_q=sli.SLIKL_TND, T1=-1))[0] == sli.SLIKL_ERR_PARAM_INVALID
+    # T1*topk must stay below 2^31
+    big = base_problem(layout_q=sli.SLIKL_TND, T1=2 ** 20, topk=4096)
+    assert ws_rc(lib, big)[0] == sli.SLIKL_ERR_PARAM_INVALID
+
+
+def test_null_pointers(lib):
+    n = ctypes.c_size_t(0)
+    assert lib.slikl_grad_workspace_size(None, ctypes.byref(n)) == sli.SLIKL_ERR_PARAM_NULLPTR
+    pr = base_problem()
+    assert lib.slikl_grad_workspace_size(ctypes.byref(pr), None) == sli.SLIKL_ERR_INNER_NULLPTR
+    tn = sli.slikl_tensors()
+    # every tensor NULL -> 161001 before any CUDA call
+    assert lib.slikl_grad(ctypes.byref(pr), ctypes.byref(tn), None, 0, None) == sli.SLIKL_ERR_PARAM_NULLPTR
+    assert lib.slikl_grad(ctypes.byref(pr), None, None, 0, None) == sli.SLIKL_ERR_PARAM_NULLPTR
+    assert lib.slikl_grad(None, ctypes.byref(tn), None, 0, None) == sli.SLIKL_ERR_PARAM_NULLPTR
+    flags = ctypes.c_uint32(0)
+    assert lib.slikl_read_device_status(None, None, ctypes.byref(flags)) == sli.SLIKL_ERR_PARAM_NULLPTR
+    assert lib.slikl_read_device_status(ctypes.c_void_p(256), None, None) == sli.SLIKL_ERR_INNER_NULLPTR
+
+
+def fake_tensors(tnd_q=False, tnd_k=False):
+    """Non-NULL pointers that are never dereferenced by host validation."""
+    tn = sli.slikl_tensors()
+    for i, (name, _) in enumerate(sli.slikl_tensors._fields_):
+        setattr(tn, name, 0x1000 * (i + 1))
+    if not tnd_q:
+        tn.cu_seqlens_q = None
+    if not tnd_k:
+        tn.cu_seqlens_k = None
+    return tn
+
+
+def test_tnd_requires_cu_seqlens(lib):
+    pr = base_problem(layout_q=sli.SLIKL_TND, T1=100)
+    tn = fake_tensors(tnd_q=False)
+    assert lib.slikl_grad(ctypes.byref(pr), ctypes.byref(tn), ctypes.c_void_p(1 << 20), 1 << 40,
+                          None) == sli.SLIKL_ERR_PARAM_NULLPTR
+
+
+def test_workspace_checks(lib):
+    pr = base_problem()
+    tn = fake_tensors()
+    _, need = ws_rc(lib, pr)
+    # misaligned workspace -> invalid; too small -> 161003 (both before any CUDA call)
+    assert lib.slikl_grad(ctypes.byref(pr), ctypes.byref(tn), ctypes.c_void_p((1 << 20) + 8), need,
+                          None) == sli.SLIKL_ERR_PARAM_INVALID
+    assert lib.slikl_grad(ctypes.byref(pr), ctypes.byref(tn), ctypes.c_void_p(1 << 20), need - 1,
+                          None) == sli.SLIKL_ERR_WORKSPACE_TOO_SMALL
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device error path")
+def test_no_device_is_an_error_not_a_fallback(lib):
+    pr = base_problem()
+    tn = fake_tensors()
+    _, need = ws_rc(lib, pr)
+    assert lib.slikl_grad(ctypes.byref(pr), ctypes.byref(tn), ctypes.c_void_p(1 << 20), need,
+                          None) == sli.SLIKL_ERR_CUDA
+
+
+def test_metadata_size_and_strings(lib):
+    assert lib.slikl_grad_metadata_size(148) == 8 + 2 * 148
+    assert lib.slikl_grad_metadata_size(0) == -1
+    assert lib.slikl_grad_metadata_size(4097) == -1
+    for code in (0, 161001, 161002, 161003, 561103, 561001, 12345):
+        assert len(lib.slikl_status_string(code)) > 0
+    pr = base_problem()
+    n = ctypes.c_size_t(0)
+    assert lib.slikl_grad_metadata_workspace_size(ctypes.byref(pr), ctypes.byref(n)) == 0
+    assert 0 < n.value < 4096 * 128 * 4 + 4096 * 64

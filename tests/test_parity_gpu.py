@@ -1,0 +1,310 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle on the same seeded
+inputs.
+
+Tolerances (floating point): softmax_out rel-L2 <= 1e-5; dw rel-L2 <= 1e-4; dq and dk
+rel-L2 <= 5e-3 and max-abs <= 2e-2 * max|ref|. Bit-exact: softmax_out = 0 at invalid
+slots, dk = 0 on key rows no valid slot names, the work split, and deterministic-mode
+repeats.
+
+Full-size workloads: softmax_out, dw and dq are compared on a sample of tokens (the oracle
+computes any token on its own); dk is compared in full on the same launch shape with every
+token outside the sample masked to -1, which leaves each sampled token's outputs unchanged
+(a pinned invariant of the oracle) and makes the full dk computable by the oracle.
+"""
+
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import slikl_inputs as si
+import sparse_lightning_indexer_b200 as sli
+
+pytestmark = pytest.mark.gpu
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+TOL = {"y": (1e-5, None), "dw": (1e-4, None), "dq": (5e-3, 2e-2), "dk": (5e-3, 2e-2)}
+
+
+def rel_l2(got, ref):
+    n = np.linalg.norm(ref)
+    d = np.linalg.norm(got - ref)
+    return d / n if n > 0 else (0.0 if d == 0 else np.inf)
+
+
+def assert_close(name, got, ref):
+    rtol, mtol = TOL[name]
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (name, got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), name
+    e = rel_l2(got, ref)
+    assert e <= rtol, f"{name}: rel-L2 {e:.3e} > {rtol}"
+    if mtol is not None:
+        m = np.abs(ref).max()
+        a = np.abs(got - ref).max()
+        assert a <= mtol * m, f"{name}: max-abs {a:.3e} > {mtol} * {m:.3e}"
+
+
+def run_gpu(wl, deterministic=False):
+    res = sli.grad_workload(wl, deterministic=deterministic)
+    torch.cuda.synchronize()
+    flags = sli.slikl_read_device_status(res["workspace"].data_ptr())
+    T1, T2, N1, D, K = wl.T1, wl.T2, wl.N1, wl.D, wl.K
+    return dict(y=res["softmax_out"].double().cpu().numpy().reshape(T1, K),
+                dw=res["dw"].double().cpu().numpy().reshape(T1, N1),
+                dq=res["dq"].double().cpu().numpy().reshape(T1, N1, D),
+                dk=res["dk"].double().cpu().numpy().reshape(T2, D),
+                dk_raw=res["dk"].cpu(), flags=flags)
+
+
+def referenced_rows(wl):
+    """Key rows named by some valid slot (index in [0, len_k(b)))."""
+    idx = wl.idx.numpy().reshape(wl.T1, wl.K)
+    qs, ks = oracle.row_starts(wl.layout, wl.layout, wl.B, wl.S1, wl.S2,
+                               None if wl.cu_seqlens_q is None else wl.cu_seqlens_q.numpy(),
+                               None if wl.cu_seqlens_k is None else wl.cu_seqlens_k.numpy())
+    batch = np.searchsorted(qs, np.arange(wl.T1), side="right") - 1
+    rows = idx + ks[batch][:, None]
+    ref = np.zeros(wl.T2, dtype=bool)
+    ref[rows[idx >= 0]] = True
+    return ref
+
+
+def check_exact(wl, got):
+    idx = wl.idx.numpy().reshape(wl.T1, wl.K)
+    assert np.all(got["y"][idx < 0] == 0.0), "softmax_out must be exactly 0 at invalid slots"
+    untouched = ~referenced_rows(wl)
+    raw = got["dk_raw"].reshape(wl.T2, wl.D)
+    assert torch.all(raw[torch.from_numpy(untouched)].view(torch.int16) == 0), \
+        "dk must be exactly +0 on rows no valid slot names"
+
+
+def check_against(wl, got, ref, tokens=None):
+    sel = slice(None) if tokens is None else tokens
+    for name in ("y", "dw", "dq"):
+        assert_close(name, got[name][sel], ref[name][sel])
+    assert_close("dk", got["dk"], ref["dk"])
+
+
+SMALL = [
+    dict(seed=1, layout="BSND", B=2, S1=40, S2=300, N1=16, D=128, K=200),
+    dict(seed=2, layout="TND", B=3, S1=50, S2=400, N1=32, D=128, K=300, dtype=torch.float16,
+         pattern="causal"),
+    dict(seed=3, layout="BSND", B=1, S1=33, S2=7, N1=1, D=64, K=1),
+    dict(seed=4, layout="BSND", B=1, S1=64, S2=64, N1=8, D=64, K=64, pattern="causal",
+         qk_scale=1.0, w_var=1 / 8),
+    dict(seed=5, layout="BSND", B=1, S1=24, S2=3000, N1=64, D=128, K=2048, qk_scale=0.1,
+         w_var=1 / 64),
+    dict(seed=6, layout="TND", B=2, S1=20, S2=600, N1=128, D=128, K=257),
+    dict(seed=7, layout="BSND", B=2, S1=17, S2=500, N1=24, D=128, K=130, dtype=torch.float16),
+    dict(seed=8, layout="BSND", B=2, S1=30, S2=100, N1=16, D=128, K=160, pattern="dup"),
+    dict(seed=9, layout="BSND", B=2, S1=30, S2=700, N1=16, D=64, K=512, invalid_frac=0.3),
+    dict(seed=10, layout="BSND", B=1, S1=9, S2=50, N1=16, D=128, K=64, pattern="none"),
+    dict(seed=11, layout="TND", B=3, lens_q=[0, 5, 3], lens_k=[4, 0, 6], N1=16, D=128, K=8,
+         pattern="uniform"),
+    dict(seed=12, layout="TND", B=4, S1=70, S2=900, N1=48, D=64, K=700, dtype=torch.float16,
+         pattern="causal", invalid_frac=0.1),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: f"s{c['seed']}")
+@pytest.mark.parametrize("det", [False, True], ids=["atomic", "det"])
+def test_small_parity(case, det):
+    wl = si.small(**case)
+    ref = oracle.grad(wl)
+    got = run_gpu(wl, deterministic=det)
+    assert got["flags"] == 0
+    check_exact(wl, got)
+    check_against(wl, got, ref)
+
+
+def test_config0_full_parity():
+    wl = si.config(0)
+    ref = oracle.grad(wl)
+    for det in (False, True):
+        got = run_gpu(wl, deterministic=det)
+        assert got["flags"] == 0
+        check_exact(wl, got)
+        check_against(wl, got, ref)
+
+
+def masked(wl, tokens):
+    """Same workload with every token outside `tokens` made all-invalid."""
+    idx = wl.idx.clone().reshape(wl.T1, wl.K)
+    keep = torch.zeros(wl.T1, dtype=torch.bool)
+    keep[torch.from_numpy(np.asarray(tokens))] = True
+    idx[~keep] = -1
+    out = si.Workload(**{f: getattr(wl, f) for f in wl.__dataclass_fields__})
+    out.idx = idx.reshape(wl.idx.shape).contiguous()
+    return out
+
+
+def sample_tokens(wl, n, seed):
+    rng = np.random.default_rng(seed)
+    pick = rng.choice(wl.T1, size=min(n, wl.T1), replace=False)
+    pick = np.union1d(pick, [0, wl.T1 - 1])           # first and last rows always
+    return np.sort(pick)
+
+
+_CFG_CACHE = {}
+
+
+def cfg(cid):
+    if cid not in _CFG_CACHE:
+        _CFG_CACHE[cid] = si.config(cid)
+    return _CFG_CACHE[cid]
+
+
+@pytest.mark.parametrize("cid", [1, 2, 3, 4])
+def test_full_size_sampled_parity(cid):
+    wl = cfg(cid)
+    toks = sample_tokens(wl, 48, seed=cid)
+    ref = oracle.grad(wl, tokens=toks)
+    got = run_gpu(wl)
+    assert got["flags"] == 0
+    check_exact(wl, got)
+    for name in ("y", "dw", "dq"):
+        assert_close(name, got[name][toks], ref[name][toks])
+    # full dk on the masked problem of the same shape
+    wm = masked(wl, toks)
+    gm = run_gpu(wm)
+    assert gm["flags"] == 0
+    check_exact(wm, gm)
+    assert_close("dk", gm["dk"], ref["dk"])
+    for name in ("y", "dw", "dq"):
+        assert_close(name, gm[name][toks], ref[name][toks])
+
+
+@pytest.mark.parametrize("cid", [1, 3])
+def test_full_size_identities(cid):
+    """Properties that hold at any size, checked on the full GPU outputs:
+    sum_d q_hd dq_hd = w_h dW_h per token and head, and
+    sum_r <k_r, dk_r> = sum_t,h w_th dW_th."""
+    wl = cfg(cid)
+    got = run_gpu(wl)
+    q = wl.q.double().numpy().reshape(wl.T1, wl.N1, wl.D)
+    k = wl.k.double().numpy().reshape(wl.T2, wl.D)
+    w = wl.w.double().numpy().reshape(wl.T1, wl.N1)
+    lhs = (q * got["dq"]).sum(-1)
+    rhs = w * got["dw"]
+    assert rel_l2(lhs, rhs) < 1e-2
+    total = (k * got["dk"]).sum()
+    assert abs(total - rhs.sum()) <= 1e-2 * np.abs(rhs).sum()
+
+
+def test_deterministic_bitwise_repeat_config4():
+    wl = cfg(4)
+    dev = torch.device("cuda")
+    t = {n: getattr(wl, n).to(dev) for n in ("q", "k", "w", "p", "idx")}
+    first = None
+    ws = None
+    for rep in range(10):
+        res = sli.grad(t["q"], t["k"], t["w"], t["p"], t["idx"], deterministic=True,
+                       workspace=ws)
+        ws = res["workspace"]
+        cur = [res[n].clone() for n in ("dq", "dk", "dw", "softmax_out")]
+        if first is None:
+            first = cur
+        else:
+            for a, b in zip(first, cur):
+                assert torch.equal(a.view(torch.uint8) if a.dtype != torch.float32 else a.view(torch.int32),
+                                   b.view(torch.uint8) if b.dtype != torch.float32 else b.view(torch.int32))
+
+
+def test_deterministic_parity_config4():
+    wl = cfg(4)
+    toks = sample_tokens(wl, 48, seed=44)
+    ref = oracle.grad(wl, tokens=toks)
+    wm = masked(wl, toks)
+    gm = run_gpu(wm, deterministic=True)
+    assert gm["flags"] == 0
+    check_exact(wm, gm)
+    assert_close("dk", gm["dk"], ref["dk"])
+    got = run_gpu(wl, deterministic=True)
+    for name in ("y", "dw", "dq"):
+        assert_close(name, got[name][toks], ref[name][toks])
+    check_exact(wl, got)
+
+
+def test_out_of_range_index_flagged_and_ignored():
+    wl = si.small(seed=21, layout="TND", B=2, S1=10, S2=50, N1=16, D=128, K=40)
+    idx = wl.idx.clone().reshape(wl.T1, wl.K)
+    klen0 = int(wl.cu_seqlens_k[1] - wl.cu_seqlens_k[0])
+    idx[0, 3] = klen0            # one past the batch's key range
+    idx[1, 5] = -7               # below -1
+    bad = si.Workload(**{f: getattr(wl, f) for f in wl.__dataclass_fields__})
+    bad.idx = idx.reshape(wl.idx.shape).contiguous()
+    got = run_gpu(bad)
+    assert got["flags"] & sli.SLIKL_DEV_INDEX_OUT_OF_RANGE
+    fixed = idx.clone()
+    fixed[0, 3] = -1
+    fixed[1, 5] = -1
+    good = si.Workload(**{f: getattr(wl, f) for f in wl.__dataclass_fields__})
+    good.idx = fixed.reshape(wl.idx.shape).contiguous()
+    ref = oracle.grad(good)
+    check_against(good, got, ref)
+
+
+def test_bad_cu_seqlens_flagged():
+    wl = si.small(seed=22, layout="TND", B=2, S1=10, S2=50, N1=16, D=128, K=40)
+    bad = si.Workload(**{f: getattr(wl, f) for f in wl.__dataclass_fields__})
+    cuk = wl.cu_seqlens_k.clone()
+    cuk[1] = cuk[2] + 5            # not monotone and beyond T2
+    bad.cu_seqlens_k = cuk
+    got = run_gpu(bad)
+    assert got["flags"] & sli.SLIKL_DEV_BAD_CU_SEQLENS_K
+    assert np.all(got["y"] == 0) and np.all(got["dk"] == 0)
+
+
+def metadata_gpu(wl, workers, mode):
+    dev = torch.device("cuda")
+    idx = wl.idx.to(dev)
+    pr = sli.make_problem(wl.q, wl.k, wl.idx, wl.layout, wl.layout, False,
+                          B=wl.B if wl.layout == "TND" else None)
+    tn = sli.slikl_tensors()
+    tn.sparse_indices = idx.data_ptr()
+    cuq = cuk = None
+    if wl.layout == "TND":
+        cuq, cuk = wl.cu_seqlens_q.to(dev), wl.cu_seqlens_k.to(dev)
+        tn.cu_seqlens_q, tn.cu_seqlens_k = cuq.data_ptr(), cuk.data_ptr()
+    n = sli.slikl_grad_metadata_size(workers)
+    meta = torch.full((n,), -5, dtype=torch.int32, device=dev)
+    wsb = sli.slikl_grad_metadata_workspace_size(pr)
+    ws = torch.empty(max(wsb, 256), dtype=torch.uint8, device=dev)
+    sli.slikl_grad_metadata(pr, tn, workers, mode, meta.data_ptr(), ws.data_ptr(), ws.numel(),
+                            torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    return meta.cpu().numpy().astype(np.int64)
+
+
+@pytest.mark.parametrize("cid", [0, 2, 4])
+@pytest.mark.parametrize("workers", [148, 37])
+def test_metadata_bit_exact(cid, workers):
+    wl = cfg(cid)
+    idx = wl.idx.numpy().reshape(wl.T1, wl.K)
+    cuk = None if wl.cu_seqlens_k is None else wl.cu_seqlens_k.numpy()
+    maxk = wl.S2 if cuk is None else int(np.diff(cuk).max())
+    hdr, ranges_eq = oracle.split_equal(wl.T1, workers, maxk)
+    m0 = metadata_gpu(wl, workers, 0)
+    assert list(m0[:6]) == list(hdr) and m0[6] == 0 and m0[7] == workers
+    assert np.array_equal(m0[8:].reshape(workers, 2), ranges_eq)
+    m1 = metadata_gpu(wl, workers, 1)
+    assert list(m1[:6]) == list(hdr) and m1[6] == 1
+    assert np.array_equal(m1[8:].reshape(workers, 2), oracle.split_weighted(idx, workers))
+
+
+def test_metadata_golden_sample_shapes():
+    with open(os.path.join(GOLDEN, "metadata_sample_shapes.json")) as f:
+        fx = json.load(f)
+    for case in fx["cases"]:
+        cuq = case["cu_seqlens_q"]
+        cuk = case["cu_seqlens_k"]
+        lq, lk = np.diff(cuq), np.diff(cuk)
+        wl = si.small(seed=0, layout="TND", B=len(lq), lens_q=list(lq), lens_k=list(lk), N1=8,
+                      D=128, K=4)
+        m = metadata_gpu(wl, case["cores"], 0)
+        assert list(m[:6]) == case["header"]
