@@ -1,0 +1,365 @@
+"""Benchmark of the sparse Lightning Indexer KL-loss backward on B200.
+
+One step = one slikl_grad call (work split, fused per-token kernel, dK cast) on the
+headline workload: causal BSND, B=1, S1=S2=4096, N1=64, D=128, topk=2048, bf16 q/k,
+inputs already resident in HBM. L2 is flushed (256 MiB write) before every timed step,
+outside the step's events.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--deterministic]
+  python bench.py --impl reference ...    # the fp64 CPU oracle on the host cores
+
+With N > 1 (torchrun, one process per GPU) every rank runs an independent replica of the
+workload (the operator has no cross-GPU exchange): weak scaling, value = all ranks' tokens
+divided by the slowest rank's device time.
+
+Prints ONE JSON line on rank 0.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import slikl_inputs as si  # noqa: E402
+
+METRIC = "query-tokens/s & TFLOP/s, % of B200 roofline (N1=64, D=128, topk=2048)"
+UNIT = "query-tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def workload_stats(wl):
+    """Nominal / valid FLOPs and compulsory bytes of one call (roofline definition:
+    unique gathered key rows, q, w, p, indices, outputs and the fp32 dK workspace)."""
+    T1, T2, N1, D, K = wl.T1, wl.T2, wl.N1, wl.D, wl.K
+    idx = wl.idx.numpy().reshape(T1, K)
+    valid = int((idx >= 0).sum())
+    flop_nom = 6.0 * N1 * K * D * T1
+    flop_valid = 6.0 * N1 * D * valid
+    # unique key rows referenced
+    if wl.layout == "BSND":
+        batch = np.arange(T1) // wl.S1
+        rows = idx + (batch * wl.S2)[:, None]
+    else:
+        cuq = wl.cu_seqlens_q.numpy()
+        cuk = wl.cu_seqlens_k.numpy()
+        batch = np.searchsorted(cuq, np.arange(T1), side="right") - 1
+        rows = idx + cuk[batch][:, None]
+    uniq = np.unique(rows[idx >= 0]).size
+    el = 2  # bf16 / fp16
+    bytes_comp = (uniq * D * el                        # gathered key rows
+                  + T1 * N1 * D * el                   # q
+                  + T1 * N1 * 4 + T1 * K * 4 + T1 * K * 4   # w, p, indices
+                  + T1 * K * 4 + T1 * N1 * 4 + T1 * N1 * D * el  # softmax_out, dw, dq
+                  + T2 * D * el                        # dk
+                  + T2 * D * 4)                        # fp32 dK workspace
+    return dict(valid=valid, flop_nom=flop_nom, flop_valid=flop_valid, bytes=bytes_comp,
+                uniq_rows=int(uniq))
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            self.path = f"/tmp/slikl_clocks_{os.getpid()}.csv"
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = max(mx, float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def raw_event():
+    """A timing cudaEvent_t created through the CUDA runtime (recorded by the C library)."""
+    from cuda.bindings import runtime as cudart
+    err, ev = cudart.cudaEventCreate()
+    if err != cudart.cudaError_t.cudaSuccess:
+        raise RuntimeError(f"cudaEventCreate: {err}")
+    return ev
+
+
+def raw_elapsed_ms(a, b):
+    from cuda.bindings import runtime as cudart
+    err, ms = cudart.cudaEventElapsedTime(a, b)
+    if err != cudart.cudaError_t.cudaSuccess:
+        raise RuntimeError(f"cudaEventElapsedTime: {err}")
+    return ms
+
+
+def oracle_rate(wl, ntok, seed=0):
+    """fp64 oracle on a seeded sample of ntok query tokens; returns (tokens/s, cores, secs)."""
+    import oracle  # CPU baseline leg only
+    oracle.build()
+    rng = np.random.default_rng(seed)
+    toks = np.sort(rng.choice(wl.T1, size=min(ntok, wl.T1), replace=False))
+    t0 = time.perf_counter()
+    oracle.grad(wl, tokens=toks)
+    dt = time.perf_counter() - t0
+    return len(toks) / dt, os.cpu_count(), dt, len(toks)
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = si.config(args.config)
+    ntok = args.ref_tokens
+    for _ in range(args.warmup):
+        oracle_rate(wl, max(ntok // 4, 1), seed=1)
+    total_tok, total_s = 0, 0.0
+    for s in range(args.steps):
+        _, cores, dt, n = oracle_rate(wl, ntok, seed=100 + s)
+        total_tok += n
+        total_s += dt
+    value = total_tok / total_s
+    sample = f"{ntok} seeded query tokens of the workload per step (full per-token outputs and their dk contributions)"
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_s / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": wl.name, "T1": wl.T1},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--deterministic", action="store_true")
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--ref-tokens", type=int, default=96)
+    ap.add_argument("--cpu-baseline-tokens", type=int, default=1024)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+    import sparse_lightning_indexer_b200 as sli
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local),
+                                timeout=__import__("datetime").timedelta(seconds=300))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    wl = si.config(args.config)
+    stats = workload_stats(wl)
+    stream = torch.cuda.Stream(device=dev)
+    # device-resident inputs
+    q, k, w, p, idx = (getattr(wl, n).to(dev) for n in ("q", "k", "w", "p", "idx"))
+    cuq = wl.cu_seqlens_q.to(dev) if wl.cu_seqlens_q is not None else None
+    cuk = wl.cu_seqlens_k.to(dev) if wl.cu_seqlens_k is not None else None
+    B = wl.B if wl.layout == "TND" else None
+    pr = sli.make_problem(q, k, idx, wl.layout, wl.layout, args.deterministic, B)
+    nbytes = sli.slikl_grad_workspace_size(pr)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dw=torch.empty_like(w),
+               softmax_out=torch.empty_like(p))
+
+    def tensors(qq, kk, ww, pp, ii, o):
+        tn = sli.slikl_tensors()
+        tn.q, tn.k, tn.w, tn.attn_softmax_l1norm, tn.sparse_indices = (
+            qq.data_ptr(), kk.data_ptr(), ww.data_ptr(), pp.data_ptr(), ii.data_ptr())
+        tn.cu_seqlens_q = cuq.data_ptr() if cuq is not None else None
+        tn.cu_seqlens_k = cuk.data_ptr() if cuk is not None else None
+        tn.dq, tn.dk, tn.dw, tn.softmax_out = (o["dq"].data_ptr(), o["dk"].data_ptr(),
+                                               o["dw"].data_ptr(), o["softmax_out"].data_ptr())
+        return tn
+
+    tn = tensors(q, k, w, p, idx, out)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    sid = stream.cuda_stream
+
+    def step(evs=None):
+        if evs is None:
+            sli.slikl_grad(pr, tn, ws.data_ptr(), nbytes, sid)
+        else:
+            sli.slikl_grad_with_events(pr, tn, ws.data_ptr(), nbytes, sid, int(evs[0]),
+                                       int(evs[1]))
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            flush.fill_(1)
+            step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        clocks = ClockSampler(vis.split(",")[local] if vis else str(local))
+        clocks.start()
+        time.sleep(0.3)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        kev = [(raw_event(), raw_event()) for _ in range(args.steps)]
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        for i in range(args.steps):
+            flush.fill_(1)
+            ev[i][0].record(stream)
+            step(kev[i])
+            ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        step_ms = [a.elapsed_time(b) for a, b in ev]
+        kern_ms = [raw_elapsed_ms(a, b) for a, b in kev]
+        flags = sli.slikl_read_device_status(ws.data_ptr(), sid)
+
+        # end to end through the public API with pinned host buffers
+        hq, hk, hw, hp, hi = (t.cpu().pin_memory() for t in (q, k, w, p, idx))
+        hout = {n: torch.empty(t.shape, dtype=t.dtype).pin_memory() for n, t in out.items()}
+        q2, k2, w2, p2, i2 = (torch.empty_like(t) for t in (q, k, w, p, idx))
+        tn2 = tensors(q2, k2, w2, p2, i2, out)
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hw, hp, hi))
+        d2h = sum(t.numel() * t.element_size() for t in hout.values())
+        e2e_ms = []
+        for i in range(args.warmup + args.steps):
+            flush.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for dst, src in ((q2, hq), (k2, hk), (w2, hw), (p2, hp), (i2, hi)):
+                dst.copy_(src, non_blocking=True)
+            sli.slikl_grad(pr, tn2, ws.data_ptr(), nbytes, sid)
+            for n, t in out.items():
+                hout[n].copy_(t, non_blocking=True)
+            b.record(stream)
+            b.synchronize()
+            if i >= args.warmup:
+                e2e_ms.append(a.elapsed_time(b))
+        clk = clocks.stop()
+
+    t_total = sum(step_ms) / 1e3
+    t_e2e = sum(e2e_ms) / 1e3
+    if world > 1:
+        tt = torch.tensor([t_total, t_e2e, sum(kern_ms) / 1e3], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_total, t_e2e, t_kern = tt.tolist()
+    else:
+        t_kern = sum(kern_ms) / 1e3
+    tokens = wl.T1 * args.steps * world
+    value = tokens / t_total
+    peaks, peak_src = load_peaks()
+    k_avg = t_kern / args.steps
+    flop = stats["flop_nom"]
+    achieved_tf = flop / k_avg / 1e12
+    peak_tf = peaks["bf16_tflops"]
+    step_avg = t_total / args.steps
+    t_roof = max(flop / (peak_tf * 1e12), stats["bytes"] / (peaks["hbm_gbs"] * 1e9))
+    # our kernels per call: 3 work-split + fused + (cast | sort init, 3 per radix pass,
+    # row pointers, segmented reduce)
+    launches_per_step = 5
+    if args.deterministic:
+        passes = (int(wl.T2).bit_length() + 7) // 8
+        launches_per_step = 3 + 1 + 1 + 3 * passes + 2
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, cores, dt, ntok = oracle_rate(wl, args.cpu_baseline_tokens)
+        cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"{ntok} seeded query tokens of the workload ({dt:.1f} s of fp64 oracle)"}
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * step_avg,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if wl.dtype.__repr__().endswith("bfloat16") else "fp16",
+            "data": "synthetic (seeded, shaped like the operator's workloads)",
+            "config": {"workload": wl.name, "T1": wl.T1, "T2": wl.T2, "N1": wl.N1, "D": wl.D,
+                       "topk": wl.K, "deterministic": bool(args.deterministic),
+                       "l2": "flushed before every timed step (256 MiB write, outside the events)",
+                       "parallelism": f"replicas x{world}"},
+            "tflops_nominal": flop / step_avg / 1e12,
+            "tflops_valid": stats["flop_valid"] / step_avg / 1e12,
+            "roofline_step": {"t_roof_ms": 1e3 * t_roof, "frac": t_roof / step_avg,
+                              "flop_nominal": flop, "compulsory_bytes": stats["bytes"],
+                              "peaks": peak_src},
+            "roofline": {"bound": "tensor", "achieved": achieved_tf, "peak": peak_tf,
+                         "unit": "TFLOP/s", "frac": achieved_tf / peak_tf, "traffic": None,
+                         "kernel": "fused per-token kernel", "peak_source": f"bf16_tflops ({peak_src})"},
+            "fused_kernel_ms": 1e3 * k_avg,
+            "e2e": {"value": tokens / t_e2e, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches_per_step * args.steps,
+            "device_status": flags,
+            "clocks": clk,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -137,6 +137,17 @@ SLIKL_API slikl_status slikl_grad_workspace_size(const slikl_problem *problem, s
 SLIKL_API slikl_status slikl_grad(const slikl_problem *problem, const slikl_tensors *tensors,
                         void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * slikl_grad with a measurement aid: when fused_begin / fused_end are not NULL they are
+ * cudaEvent_t handles (created by the caller) recorded on `stream` immediately before and
+ * after the fused per-token kernel, so its duration can be read with cudaEventElapsedTime.
+ * Everything else, including errors, is as slikl_grad (which is this call with NULL events).
+ */
+SLIKL_API slikl_status slikl_grad_with_events(const slikl_problem *problem,
+                                              const slikl_tensors *tensors, void *workspace,
+                                              size_t workspace_bytes, void *stream,
+                                              void *fused_begin, void *fused_end);
+
 /* Device status bits (see slikl_read_device_status). */
 #define SLIKL_DEV_INDEX_OUT_OF_RANGE  0x1u  /* some valid-looking index was >= len_k(b) or < -1 */
 #define SLIKL_DEV_BAD_CU_SEQLENS_Q    0x2u  /* cu_seqlens_q not 0..T1 non-decreasing           */

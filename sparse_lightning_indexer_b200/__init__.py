@@ -36,7 +36,8 @@ SLIKL_DEV_BAD_CU_SEQLENS_Q = 0x2
 SLIKL_DEV_BAD_CU_SEQLENS_K = 0x4
 SLIKL_DEV_WAIT_TIMEOUT = 0x8
 
-EXPORTED = ("slikl_grad_workspace_size", "slikl_grad", "slikl_read_device_status",
+EXPORTED = ("slikl_grad_workspace_size", "slikl_grad", "slikl_grad_with_events",
+            "slikl_read_device_status",
             "slikl_grad_metadata_size", "slikl_grad_metadata_workspace_size",
             "slikl_grad_metadata", "slikl_status_string")
 
@@ -74,6 +75,8 @@ def load_library() -> ctypes.CDLL:
         P, VP = ctypes.POINTER, ctypes.c_void_p
         lib.slikl_grad_workspace_size.argtypes = [P(slikl_problem), P(ctypes.c_size_t)]
         lib.slikl_grad.argtypes = [P(slikl_problem), P(slikl_tensors), VP, ctypes.c_size_t, VP]
+        lib.slikl_grad_with_events.argtypes = [P(slikl_problem), P(slikl_tensors), VP,
+                                               ctypes.c_size_t, VP, VP, VP]
         lib.slikl_read_device_status.argtypes = [VP, VP, P(ctypes.c_uint32)]
         lib.slikl_grad_metadata_size.argtypes = [ctypes.c_int32]
         lib.slikl_grad_metadata_size.restype = ctypes.c_int64
@@ -82,7 +85,8 @@ def load_library() -> ctypes.CDLL:
                                             ctypes.c_int32, VP, VP, ctypes.c_size_t, VP]
         lib.slikl_status_string.argtypes = [ctypes.c_int32]
         lib.slikl_status_string.restype = ctypes.c_char_p
-        for name in ("slikl_grad_workspace_size", "slikl_grad", "slikl_read_device_status",
+        for name in ("slikl_grad_workspace_size", "slikl_grad", "slikl_grad_with_events",
+                     "slikl_read_device_status",
                      "slikl_grad_metadata_workspace_size", "slikl_grad_metadata"):
             getattr(lib, name).restype = ctypes.c_int32
         _lib = lib
@@ -109,6 +113,16 @@ def slikl_grad(problem: slikl_problem, tensors: slikl_tensors, workspace: int,
                                    workspace_bytes, stream)
     if rc != SLIKL_OK:
         raise SliklError(rc, "slikl_grad")
+
+
+def slikl_grad_with_events(problem: slikl_problem, tensors: slikl_tensors, workspace: int,
+                           workspace_bytes: int, stream: int = 0, fused_begin: int = 0,
+                           fused_end: int = 0) -> None:
+    rc = load_library().slikl_grad_with_events(ctypes.byref(problem), ctypes.byref(tensors),
+                                               workspace, workspace_bytes, stream,
+                                               fused_begin or None, fused_end or None)
+    if rc != SLIKL_OK:
+        raise SliklError(rc, "slikl_grad_with_events")
 
 
 def slikl_read_device_status(workspace: int, stream: int = 0) -> int:

@@ -10,8 +10,6 @@
 
 namespace slikl {
 
-cudaError_t launch_fused_sm100(const Params &P, int workers, cudaStream_t s, bool *handled);
-
 namespace {
 
 struct Derived {
@@ -86,6 +84,7 @@ Params make_params(const slikl_problem *pr, const Derived &dv, const slikl_tenso
     P.tok_kbase = reinterpret_cast<int32_t *>(base + L.tok_kbase);
     P.tok_klen = reinterpret_cast<int32_t *>(base + L.tok_klen);
     P.tok_cost = reinterpret_cast<int32_t *>(base + L.tok_cost);
+    P.tok_tiles = reinterpret_cast<uint64_t *>(base + L.tok_tiles);
     P.cost_prefix = reinterpret_cast<int64_t *>(base + L.cost_prefix);
     P.dk_acc = reinterpret_cast<float *>(base + L.dk_acc);
     P.partials = reinterpret_cast<float *>(base + L.partials);
@@ -135,6 +134,13 @@ slikl_status slikl_grad_workspace_size(const slikl_problem *problem, size_t *wor
 
 slikl_status slikl_grad(const slikl_problem *problem, const slikl_tensors *tensors,
                         void *workspace, size_t workspace_bytes, void *stream) {
+    return slikl_grad_with_events(problem, tensors, workspace, workspace_bytes, stream, nullptr,
+                                  nullptr);
+}
+
+slikl_status slikl_grad_with_events(const slikl_problem *problem, const slikl_tensors *tensors,
+                                    void *workspace, size_t workspace_bytes, void *stream,
+                                    void *fused_begin, void *fused_end) {
     Derived dv;
     slikl_status st = validate(problem, &dv);
     if (st != SLIKL_OK) return st;
@@ -156,11 +162,15 @@ slikl_status slikl_grad(const slikl_problem *problem, const slikl_tensors *tenso
         cudaMemsetAsync(P.dk_acc, 0, sizeof(float) * (size_t)dv.T2 * problem->D, s) != cudaSuccess)
         return SLIKL_ERR_CUDA;
     if (launch_metadata(P, workers, 1, s) != cudaSuccess) return SLIKL_ERR_CUDA;
+    if (fused_begin && cudaEventRecord(static_cast<cudaEvent_t>(fused_begin), s) != cudaSuccess)
+        return SLIKL_ERR_CUDA;
     if (dv.T1 > 0) {
         bool handled = false;
         if (launch_fused_sm100(P, workers, s, &handled) != cudaSuccess) return SLIKL_ERR_CUDA;
         if (!handled && launch_fused_simt(P, workers, s) != cudaSuccess) return SLIKL_ERR_CUDA;
     }
+    if (fused_end && cudaEventRecord(static_cast<cudaEvent_t>(fused_end), s) != cudaSuccess)
+        return SLIKL_ERR_CUDA;
     cudaError_t e = P.deterministic ? launch_deterministic_reduce(P, s) : launch_cast(P, s);
     return e == cudaSuccess ? SLIKL_OK : SLIKL_ERR_CUDA;
 }

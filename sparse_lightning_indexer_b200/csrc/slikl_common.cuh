@@ -34,6 +34,7 @@ struct Params {
     int32_t *tok_kbase;   // [T1] first key row of the token's batch
     int32_t *tok_klen;    // [T1] key count of the token's batch
     int32_t *tok_cost;    // [T1] work estimate per token
+    uint64_t *tok_tiles;  // [T1] bit i set when slot tile i holds an index >= 0
     int64_t *cost_prefix; // [T1 + 1]
     float *dk_acc;        // [T2*D] fp32 accumulator (atomic mode)
     float *partials;      // [T1*K*D] per-slot dK rows (deterministic mode)
@@ -44,7 +45,7 @@ struct Params {
 
 // Byte offsets of the workspace regions; every region starts 256-byte aligned.
 struct WsLayout {
-    size_t status, meta, tok_kbase, tok_klen, tok_cost, cost_prefix;
+    size_t status, meta, tok_kbase, tok_klen, tok_cost, tok_tiles, cost_prefix;
     size_t dk_acc, partials, keys0, vals0, keys1, vals1, hist, row_ptr;
     size_t total;
 };
@@ -62,6 +63,7 @@ inline WsLayout make_layout(int64_t T1, int64_t T2, int64_t K, int64_t D, int de
     L.tok_kbase = take(sizeof(int32_t) * (size_t)T1);
     L.tok_klen = take(sizeof(int32_t) * (size_t)T1);
     L.tok_cost = take(sizeof(int32_t) * (size_t)T1);
+    L.tok_tiles = take(sizeof(uint64_t) * (size_t)T1);
     L.cost_prefix = take(sizeof(int64_t) * (size_t)(T1 + 1));
     L.dk_acc = take(det ? 0 : sizeof(float) * (size_t)T2 * (size_t)D);
     size_t n = (size_t)T1 * (size_t)K;
@@ -116,6 +118,7 @@ __device__ __forceinline__ int32_t slot_row(int32_t v, int32_t kbase, int32_t kl
 // kernels (defined in the .cu files)
 cudaError_t launch_metadata(const Params &P, int workers, int mode, cudaStream_t s);
 cudaError_t launch_fused_simt(const Params &P, int workers, cudaStream_t s);
+cudaError_t launch_fused_sm100(const Params &P, int workers, cudaStream_t s, bool *handled);
 cudaError_t launch_cast(const Params &P, cudaStream_t s);
 cudaError_t launch_deterministic_reduce(const Params &P, cudaStream_t s);
 

@@ -70,15 +70,20 @@ __global__ void meta_tokens(Params P) {
     // cost = 1 + number of 128-slot tiles holding an index >= 0
     const int32_t *row = P.idx + t * (int64_t)P.K;
     int tiles = 0;
-    for (int j0 = 0; j0 < P.K; j0 += kSlotTile) {
+    uint64_t mask = 0;
+    for (int j0 = 0, i = 0; j0 < P.K; j0 += kSlotTile, ++i) {
         bool any = false;
         for (int j = j0 + lane; j < j0 + kSlotTile && j < P.K; j += 32) any |= row[j] >= 0;
-        tiles += __any_sync(0xffffffffu, any) ? 1 : 0;
+        if (__any_sync(0xffffffffu, any)) {
+            tiles += 1;
+            mask |= uint64_t(1) << i;
+        }
     }
     if (lane == 0) {
         P.tok_kbase[t] = kbase;
         P.tok_klen[t] = klen;
         P.tok_cost[t] = 1 + tiles;
+        P.tok_tiles[t] = klen > 0 ? mask : 0;
     }
 }
 
