@@ -23,7 +23,8 @@
  *
  * Conventions for every entry point
  *   - Ownership: the caller allocates every tensor and the workspace. The library
- *     allocates no memory and keeps no state between calls.
+ *     allocates no memory and keeps no state between calls (slikl_grad_noalloc, for
+ *     callers that cannot allocate, uses a fixed device array of the library instead).
  *   - Pointers named "device" are CUDA device pointers on the current device; tensors are
  *     dense and contiguous in the layouts stated below.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream). Launch-phase calls are
@@ -193,6 +194,26 @@ SLIKL_API slikl_status slikl_grad_metadata_workspace_size(const slikl_problem *p
 SLIKL_API slikl_status slikl_grad_metadata(const slikl_problem *problem, const slikl_tensors *tensors,
                                  int32_t num_workers, int32_t mode, int32_t *metadata,
                                  void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * slikl_grad for callers that cannot allocate device memory when they call (code that runs
+ * under an allocator which forbids cudaMalloc, or that has no way to reach its framework's
+ * allocator). Nothing is allocated per call: the scratch that slikl_grad takes as
+ * `workspace` is a fixed array of SLIKL_NOALLOC_SCRATCH_BYTES in the library's device code,
+ * which every GPU that loads the library keeps until the process exits. The operator pages
+ * have no counterpart of this call; it is an addition of this library.
+ *
+ * `problem`, `tensors` and `stream` are as for slikl_grad; the caller still owns every input
+ * and output tensor. The first call on each device looks up the array's device address
+ * (make that first call outside any stream capture). All calls share the array: calls whose
+ * GPU work overlaps (unordered streams) race and give wrong results.
+ * Errors: as slikl_grad; SLIKL_ERR_WORKSPACE_TOO_SMALL if the problem needs more scratch than
+ * SLIKL_NOALLOC_SCRATCH_BYTES (slikl_grad_workspace_size tells how much);
+ * SLIKL_ERR_PARAM_INVALID for deterministic = 1, whose per-slot scratch does not fit.
+ */
+#define SLIKL_NOALLOC_SCRATCH_BYTES (32u << 20)
+SLIKL_API slikl_status slikl_grad_noalloc(const slikl_problem *problem,
+                                          const slikl_tensors *tensors, void *stream);
 
 /* Human-readable name of a status code (static string, never NULL). */
 SLIKL_API const char *slikl_status_string(slikl_status status);

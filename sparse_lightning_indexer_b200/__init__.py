@@ -39,7 +39,9 @@ SLIKL_DEV_WAIT_TIMEOUT = 0x8
 EXPORTED = ("slikl_grad_workspace_size", "slikl_grad", "slikl_grad_with_events",
             "slikl_read_device_status",
             "slikl_grad_metadata_size", "slikl_grad_metadata_workspace_size",
-            "slikl_grad_metadata", "slikl_status_string")
+            "slikl_grad_metadata", "slikl_status_string", "slikl_grad_noalloc")
+
+SLIKL_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class slikl_problem(ctypes.Structure):
@@ -83,6 +85,8 @@ def load_library() -> ctypes.CDLL:
         lib.slikl_grad_metadata_workspace_size.argtypes = [P(slikl_problem), P(ctypes.c_size_t)]
         lib.slikl_grad_metadata.argtypes = [P(slikl_problem), P(slikl_tensors), ctypes.c_int32,
                                             ctypes.c_int32, VP, VP, ctypes.c_size_t, VP]
+        lib.slikl_grad_noalloc.argtypes = [P(slikl_problem), P(slikl_tensors), VP]
+        lib.slikl_grad_noalloc.restype = ctypes.c_int32
         lib.slikl_status_string.argtypes = [ctypes.c_int32]
         lib.slikl_status_string.restype = ctypes.c_char_p
         for name in ("slikl_grad_workspace_size", "slikl_grad", "slikl_grad_with_events",
@@ -131,6 +135,14 @@ def slikl_read_device_status(workspace: int, stream: int = 0) -> int:
     if rc != SLIKL_OK:
         raise SliklError(rc, "slikl_read_device_status")
     return int(flags.value)
+
+
+def slikl_grad_noalloc(problem: slikl_problem, tensors: slikl_tensors, stream: int = 0) -> None:
+    """slikl_grad with the library's fixed device scratch array instead of a caller workspace
+    (for callers that cannot allocate device memory when they call)."""
+    rc = load_library().slikl_grad_noalloc(ctypes.byref(problem), ctypes.byref(tensors), stream)
+    if rc != SLIKL_OK:
+        raise SliklError(rc, "slikl_grad_noalloc")
 
 
 def slikl_grad_metadata_size(num_workers: int) -> int:
