@@ -1,27 +1,30 @@
 // Fused per-token kernel on the sm_100a tensor cores (tcgen05 MMA, accumulators in TMEM).
 //
-// Per query token t, over its active 128-slot tiles (aclnnSparseLightningIndexerKLLossGrad,
-// section "计算公式"):
-//   pass A  gather K rows -> smem; S^T[128 keys x N1] = K . q^T          (tcgen05, TMEM)
-//           epilogue (one thread per key slot): I = w . ReLU(S) and online max / sum;
-//           I is parked in softmax_out.
-//   combine m, Z over the token.
-//   pass B  gather K rows again; S^T recomputed (tcgen05); epilogue: y = e^(I-m)/Z ->
-//           softmax_out, dI = y - p, dW_h += dI ReLU(S_h) (fp32, per thread),
-//           dS = dI * w * 1[S > 0] -> bf16/fp16 smem tile [N1 x 128 keys]
-//           dq^T[D x N1] += K^T . dS^T                                    (tcgen05, TMEM)
-//           dK^T[D x 128 keys] = q^T . dS                                 (tcgen05, TMEM)
-//           epilogue: dK^T rows (one thread per d) scatter-added with red.global.add.f32,
-//           32 consecutive d per warp instruction (128-byte lines), or stored per slot in
-//           deterministic mode.
-//   dW reduced over the token in a fixed order; dq^T read back from TMEM.
-// Recomputing S in pass B costs a fourth product per tile (8 instead of 6 N1*D*K FLOP per
-// token) but keeps the per-thread state to one fp32 accumulator per head; the L2 scatter
-// of dK, not the tensor pipe, bounds this kernel.
+// For each query token t of the CTA's range and each of its active 128-slot tiles
+// (aclnnSparseLightningIndexerKLLossGrad, section "计算公式"):
+//   pass A  K rows of the tile gathered to smem; S^T[128 keys x N1] = K . q^T (tcgen05);
+//           I = w . ReLU(S) per slot, online max / sum; I parked in softmax_out.
+//   after the last pass-A tile: max and sum combined over the token.
+//   pass B  K rows gathered again; S^T recomputed; y = e^(I-m)/Z -> softmax_out, dI = y - p,
+//           dW_h += dI ReLU(S_h) (fp32), dS = dI * w * 1[S > 0] -> bf16/fp16 smem tile;
+//           dq^T[D x N1] += K^T . dS^T and dK^T[D x 128 keys] = q^T . dS (tcgen05);
+//           dK^T scattered into the fp32 key rows with red.global.add.f32, 32 consecutive d
+//           per warp instruction (one 128-byte line), or stored per slot (deterministic mode).
+//   after the last pass-B tile: dW reduced in a fixed order, dq^T read back from TMEM.
 //
-// Warp roles (320 threads): warp 0 gathers (cp.async, 16-byte row chunks, zero-fill for
-// invalid slots), warp 1 issues the MMAs (one thread) and owns TMEM, warps 2..9 are two
-// epilogue warpgroups that take the tiles of each pass in turn.
+// Schedule. The L2 fp32 reduction rate bounds this kernel, so the scatter must never
+// idle: all roles walk one deterministic item sequence in which pass A of the CTA's next
+// token alternates with pass B of the current one (phase k = B(t_{k-1}) interleaved with
+// A(t_k)). Every item gathers one K tile and computes one S tile.
+//
+// Warp roles (384 threads, 168 registers each):
+//   warps 0-2   producers: each warp gathers a third of the rows of every tile with cp.async
+//               (16-byte chunks of the 256-byte key rows, zero-fill for invalid slots);
+//               warp 0 also loads q.
+//   warp 3      MMA issuer (one thread) and TMEM owner; the S product runs one item ahead.
+//   warps 4-7   scatter group: dK^T tiles from TMEM to the fp32 key rows.
+//   warps 8-11  softmax group: pass-A and pass-B epilogues, dW, dq readback.
+// The two 4-warp groups each cover the four TMEM lane quadrants (warp id % 4).
 //
 // Shared-memory tiles use the 128-byte swizzle in 8-row atoms, so one K tile serves as the
 // K-major A operand of the S product and as the MN-major A operand of the dq product; the q
@@ -38,8 +41,7 @@
 namespace slikl {
 namespace {
 
-constexpr int kThreads = 320;
-constexpr int kEpiThreads = 256;
+constexpr int kThreads = 384;
 constexpr long long kWaitCycles = 1ll << 31;
 constexpr int kTmemCols = 512;
 constexpr int kStageBytes = 128 * 256;      // 128 key rows x 128 d (two 64-d column blocks)
@@ -121,6 +123,21 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *v) {
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float *v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+        ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])),
+          "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])),
+          "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+          "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
+          "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
+          "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15]))
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
     tmem_ld16(taddr, v);
     tmem_ld16(taddr + 16, v + 16);
@@ -147,23 +164,27 @@ __device__ __forceinline__ uint32_t sw128(int row, int col_elem) {
 }
 
 struct Barriers {
-    uint64_t kv_full[4], kv_empty[4];
-    uint64_t q_full[2], q_empty[2];
-    uint64_t s_full[2], s_empty[2];
-    uint64_t ds_full[2], ds_empty[2];
-    uint64_t dk_full[2], dk_empty[2];
-    uint64_t dq_full, dq_empty;
+    uint64_t kv_full[4], kv_empty[4];     // K stages: producers -> MMA -> producers
+    uint64_t q_full[2], q_empty[2];       // q tiles: producer 0 -> MMA -> producer 0
+    uint64_t s_full[2], s_empty[2];       // S^T in TMEM: MMA -> softmax group -> MMA
+    uint64_t ds_full[2];                  // dS tile in smem: softmax group -> MMA
+    uint64_t rows_full[2];                // key rows of a dS tile: softmax -> scatter group
+    uint64_t dk_full[2], dk_empty[2];     // dK^T in TMEM: MMA -> scatter group -> MMA/softmax
+    uint64_t dq_full, dq_empty;           // dq^T in TMEM: MMA -> softmax group -> MMA
     uint64_t drain;
-    uint64_t epi;        // all 8 epilogue warps (reusable barrier)
-    uint64_t wgb[2];     // the 4 warps of one epilogue warpgroup
+    uint64_t sm_sync;                     // the 4 softmax warps (reusable barrier)
 };
 
 struct SmemPlan {
-    uint32_t stages, kv, q, ds, w, rows, red, bar, total;
+    uint32_t stages, kv, q, ds, w, rows, red, ring, bar, total;
 };
 
+// Per producer warp, 4 slots of: 128 slot indices, key base, key count (+ padding).
+constexpr int kRingSlot = 136;            // int32 entries per slot
+constexpr int kRowsStride = 132;          // int32 entries per key-row buffer (16-byte multiple)
+
 template <int N1P>
-__host__ __device__ inline SmemPlan plan_smem(int K, int stages) {
+__host__ __device__ inline SmemPlan plan_smem(int stages) {
     SmemPlan s{};
     uint32_t off = 0;
     auto take = [&](uint32_t bytes, uint32_t align) {
@@ -172,14 +193,14 @@ __host__ __device__ inline SmemPlan plan_smem(int K, int stages) {
         off += bytes;
         return o;
     };
-    (void)K;
     s.stages = stages;
     s.kv = take(stages * kStageBytes, 1024);
     s.q = take(2 * N1P * 256, 1024);                 // two buffers, 2 column blocks each
     s.ds = take(2 * N1P * 256, 1024);                // two buffers [N1P heads x 128 keys]
-    s.w = take(N1P * 4, 16);
-    s.rows = take(2 * 128 * 4, 16);
-    s.red = take(8 * 64 * 4 + 64, 16);
+    s.w = take(2 * N1P * 4, 16);                     // w of two tokens
+    s.rows = take(2 * kRowsStride * 4, 16);          // key rows of two dS tiles
+    s.red = take(4 * 64 * 4, 16);
+    s.ring = take(3 * 4 * kRingSlot * 4, 16);
     s.bar = take(sizeof(Barriers) + 16, 8);
     s.total = off + 1024;                            // slack for aligning the dynamic base
     return s;
@@ -188,7 +209,7 @@ __host__ __device__ inline SmemPlan plan_smem(int K, int stages) {
 struct Ctl {
     volatile int abort;
     uint32_t tmem_base;
-    float stat_m[8], stat_z[8];
+    float stat_m[4], stat_z[4];
 };
 
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Ctl *ctl,
@@ -228,16 +249,100 @@ __device__ __forceinline__ uint16_t to_bits16<__half>(float v) {
     return __half_as_ushort(__float2half_rn(v));
 }
 
+
+// ------------------------------------------------------------------------------------------
+// Item schedule shared by every role
+// ------------------------------------------------------------------------------------------
+struct Item {
+    int kind;        // 0 = pass A, 1 = pass B, -1 = none
+    int t;           // token row
+    int tile;        // 128-slot tile index within the token
+    int ord;         // ordinal of the token among the CTA's active tokens
+    bool first;      // first tile of this token in this pass
+    bool last;       // last tile of this token in this pass
+};
+
+// Phase 0 = A(t_0); phase k = B(t_(k-1)) and A(t_k) alternated (B first), then whichever
+// remains; the final phase = B(t_last).
+// Within a token the tiles are visited from a CTA-dependent starting tile (a rotation of the
+// tile order): CTAs working on neighbouring tokens then scatter into different key rows at
+// the same time instead of contending for the same L2 lines.
+struct Sched {
+    const uint64_t *tiles;
+    int t_next, t_end, nt;
+    int ta, oa, ra; uint64_t ma, ma_all; bool a_on, a_first, a_exists;
+    int tb, ob, rb; uint64_t mb; bool b_on, b_first;
+    int next_ord;
+    bool turn_b;
+
+    __device__ uint64_t rot(uint64_t m, int r) const {
+        if (r == 0) return m;
+        const uint64_t full = nt >= 64 ? ~0ull : ((1ull << nt) - 1);
+        return ((m >> r) | (m << (nt - r))) & full;
+    }
+
+    __device__ bool find_a() {
+        for (; t_next < t_end; ++t_next) {
+            const uint64_t m = tiles[t_next];
+            if (m) {
+                ta = t_next++;
+                oa = next_ord++;
+                ra = (int)((blockIdx.x * 7u + (unsigned)ta * 3u) % (unsigned)nt);
+                ma = ma_all = rot(m, ra);
+                a_on = true;
+                a_first = true;
+                return true;
+            }
+        }
+        a_on = false;
+        return false;
+    }
+    __device__ void init(const uint64_t *tl, int t0, int t1, int ntiles) {
+        tiles = tl; t_next = t0; t_end = t1; next_ord = 0; nt = ntiles;
+        b_on = false; turn_b = true;
+        a_exists = find_a();
+    }
+    __device__ Item next() {
+        Item it;
+        it.kind = -1;
+        if (!a_on && !b_on) return it;
+        const bool take_b = b_on && (!a_on || turn_b);
+        turn_b = !turn_b;
+        if (take_b) {
+            it.kind = 1; it.t = tb; it.ord = ob; it.first = b_first;
+            it.tile = (__ffsll((long long)mb) - 1 + rb) % nt;
+            mb &= mb - 1;
+            it.last = mb == 0;
+            b_first = false;
+            if (it.last) b_on = false;
+        } else {
+            it.kind = 0; it.t = ta; it.ord = oa; it.first = a_first;
+            it.tile = (__ffsll((long long)ma) - 1 + ra) % nt;
+            ma &= ma - 1;
+            it.last = ma == 0;
+            a_first = false;
+            if (it.last) a_on = false;
+        }
+        if (!a_on && !b_on) {
+            // phase ends: its A token becomes the B token of the next phase
+            if (a_exists) { tb = ta; ob = oa; rb = ra; mb = ma_all; b_on = true; b_first = true; }
+            a_exists = find_a();
+            turn_b = true;
+        }
+        return it;
+    }
+};
+
 // ------------------------------------------------------------------------------------------
 // The kernel
 // ------------------------------------------------------------------------------------------
-template <int N1P, int D, typename T, int LAG>
+template <int N1P, int D, typename T>
 __global__ void __launch_bounds__(kThreads, 1) fused_sm100(Params P, int stages) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int K = P.K;
-    const SmemPlan SP = plan_smem<N1P>(K, stages);
+    const SmemPlan SP = plan_smem<N1P>(stages);
     Barriers *bars = reinterpret_cast<Barriers *>(smem + SP.bar);
     __shared__ Ctl ctl;
     constexpr int kFmt = std::is_same<T, __nv_bfloat16>::value ? 1 : 0;
@@ -245,6 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_sm100(Params P, int stages)
     constexpr uint32_t kIdescDq = idesc_f16(kFmt, 128, N1P, 1, 0);
     constexpr uint32_t kIdescDk = idesc_f16(kFmt, 128, 128, 1, 1);
     constexpr int kDChunks = D / 8;          // 16-byte chunks per key row
+    constexpr int kC = N1P < 32 ? N1P : 32;  // S columns per TMEM load
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t0 = P.meta[kMetaHeader + 2 * blockIdx.x];
@@ -254,25 +360,23 @@ __global__ void __launch_bounds__(kThreads, 1) fused_sm100(Params P, int stages)
     if (threadIdx.x == 0) {
         ctl.abort = 0;
         for (int s = 0; s < stages; ++s) {
-            mbar_init(&bars->kv_full[s], 1);
+            mbar_init(&bars->kv_full[s], 96);       // one arrival per producer thread
             mbar_init(&bars->kv_empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&bars->q_full[b], 1);
+            mbar_init(&bars->q_full[b], 32);
             mbar_init(&bars->q_empty[b], 1);
             mbar_init(&bars->s_full[b], 1);
             mbar_init(&bars->s_empty[b], 4);
             mbar_init(&bars->ds_full[b], 4);
-            mbar_init(&bars->ds_empty[b], 1);
+            mbar_init(&bars->rows_full[b], 4);
             mbar_init(&bars->dk_full[b], 1);
             mbar_init(&bars->dk_empty[b], 4);
         }
         mbar_init(&bars->dq_full, 1);
-        mbar_init(&bars->dq_empty, 8);
+        mbar_init(&bars->dq_empty, 4);
         mbar_init(&bars->drain, 1);
-        mbar_init(&bars->epi, 8);
-        mbar_init(&bars->wgb[0], 4);
-        mbar_init(&bars->wgb[1], 4);
+        mbar_init(&bars->sm_sync, 4);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     // zero the q buffers once: padded heads and, for D = 64, the upper column block stay 0;
@@ -286,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_sm100(Params P, int stages)
                     make_uint4(0, 0, 0, 0);
     }
     fence_proxy_async();
-    if (warp == 1) {
+    if (warp == 3) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                      ::"r"(smem_u32(&ctl.tmem_base)), "r"(kTmemCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
@@ -297,90 +401,123 @@ __global__ void __launch_bounds__(kThreads, 1) fused_sm100(Params P, int stages)
     const uint32_t tmem = ctl.tmem_base;
     const uint32_t tm_s = tmem;              // S^T buffers: columns [0, 2*N1P)
     const uint32_t tm_dq = tmem + 128;       // dq^T: columns [128, 128 + N1P)
+    const uint32_t tm_dw = tmem + 192;       // per-slot dW partial sums: columns [192, 192 + N1P)
     const uint32_t tm_dk = tmem + 256;       // dK^T buffers: columns [256, 512)
+    int32_t *rows_s = reinterpret_cast<int32_t *>(smem + SP.rows);   // [2][kRowsStride]
 
-    if (warp == 0) {
-        // =============================== producer ===============================
-        uint64_t *pend[LAG + 1];
-        int npend = 0;
-        uint32_t gk = 0, tq = 0;
-        const char *kbase_ptr = static_cast<const char *>(P.k);
+    Sched sc;
+    sc.init(P.tok_tiles, t0, t1, (K + 127) / 128);
+
+    if (warp < 3) {
+        // =============================== producers ===============================
+        // Every producer warp walks every item in order and waits on every stage phase (a warp
+        // that skipped items could be fooled by the phase parity of a reused stage); each warp
+        // copies its own third of the tile's row groups. Every lane ends an item with
+        // cp.async.mbarrier.arrive.noinc, so a stage turns full (96 arrivals) when all of its
+        // copies have landed, without any producer waiting for them. The slot indices, key
+        // base and key count of item g + 2 travel with item g's copies into a 4-slot ring in
+        // shared memory; item g reads them after the full barrier of item g - 2.
         const int rsub = lane / kDChunks;                 // row within a group of rows
         const int chunk = lane % kDChunks;
         constexpr int kRowsPerPass = 32 / kDChunks;       // 2 (D=128) or 4 (D=64)
-        auto signal_done = [&](bool all) {
-            if (all) cp_async_wait<0>(); else cp_async_wait<LAG>();
-            fence_proxy_async();
-            __syncwarp();
-            int n = all ? npend : npend - LAG;
-            if (lane == 0)
-                for (int i = 0; i < n; ++i) mbar_arrive(pend[i]);
-            for (int i = 0; i + n < npend; ++i) pend[i] = pend[i + n];
-            npend -= n;
-        };
-        auto push = [&](uint64_t *bar) {
-            cp_async_commit();
-            pend[npend++] = bar;
-            if (npend > LAG) signal_done(false);
-        };
+        const char *kbase_ptr = static_cast<const char *>(P.k);
+        int32_t *ring = reinterpret_cast<int32_t *>(smem + SP.ring) + warp * 4 * kRingSlot;
         bool ok = true;
-        for (int t = t0; t < t1 && ok; ++t) {
-            const uint64_t mask = P.tok_tiles[t];
-            if (!mask) continue;
-            const int32_t kb = P.tok_kbase[t], kl = P.tok_klen[t];
-            const int32_t *irow = P.idx + (int64_t)t * K;
-            // q tile (rows h < N1) into q buffer tq % 2
-            const int qb = tq & 1;
-            if (!wait_bar(&bars->q_empty[qb], ((tq >> 1) & 1) ^ 1, &ctl, P.status)) { ok = false; break; }
-            {
-                const char *qsrc = static_cast<const char *>(P.q) + (int64_t)t * P.N1 * D * 2;
+        auto arrive_on_copies = [&](uint64_t *bar) {
+            asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+                         : "memory");
+        };
+        // 4-byte copies (zero-filled past the end of the token's slots): lane l copies slots
+        // l, l+32, l+64, l+96; lane 0 also the key base and key count
+        auto fetch_idx = [&](const Item &it, int slot) {
+            int32_t *dst = ring + slot * kRingSlot;
+            const int32_t *irow = P.idx + (int64_t)it.t * K;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int j = it.tile * 128 + lane + 32 * u;
+                const bool in = j < K;
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;"
+                             ::"r"(smem_u32(dst + lane + 32 * u)), "l"(in ? irow + j : irow), "r"(in ? 4 : 0)
+                             : "memory");
+            }
+            if (lane == 0) {
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst + 128)),
+                             "l"(P.tok_kbase + it.t) : "memory");
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst + 129)),
+                             "l"(P.tok_klen + it.t) : "memory");
+            }
+        };
+        Item it0 = sc.next();
+        Item it1 = it0.kind >= 0 ? sc.next() : it0;
+        Item it2 = it1.kind >= 0 ? sc.next() : it1;
+        if (it0.kind >= 0) fetch_idx(it0, 0);
+        if (it1.kind >= 0) fetch_idx(it1, 1);
+        cp_async_commit();
+        cp_async_wait<0>();
+        __syncwarp();
+        uint32_t g = 0;
+        while (ok && it0.kind >= 0) {
+            if (warp == 0 && it0.kind == 0 && it0.first) {
+                // q tile of a new token (rows h < N1) into q buffer ord % 2
+                const int qb = it0.ord & 1;
+                if (!wait_bar(&bars->q_empty[qb], ((it0.ord >> 1) & 1) ^ 1, &ctl, P.status)) { ok = false; break; }
+                const char *qsrc = static_cast<const char *>(P.q) + (int64_t)it0.t * P.N1 * D * 2;
                 const uint32_t qdst = smem_u32(smem + SP.q + qb * N1P * 256);
                 for (int h = rsub; h < P.N1; h += kRowsPerPass) {
                     const int cb = chunk >> 3;
                     cp_async16(qdst + cb * (N1P * 128) + sw128(h, (chunk & 7) * 8),
                                qsrc + (int64_t)h * D * 2 + chunk * 16, 16);
                 }
-                push(&bars->q_full[qb]);
+                arrive_on_copies(&bars->q_full[qb]);
             }
-            // pass A then pass B: the same gather twice
-            for (int pass = 0; pass < 2 && ok; ++pass) {
-                uint64_t m = mask;
-                while (m) {
-                    const int tile = __ffsll((long long)m) - 1;
-                    m &= m - 1;
-                    const int s = gk % stages;
-                    if (!wait_bar(&bars->kv_empty[s], ((gk / stages) & 1) ^ 1, &ctl, P.status)) { ok = false; break; }
-                    const uint32_t dst = smem_u32(smem + SP.kv + s * kStageBytes);
-                    for (int r = rsub; r < 128; r += kRowsPerPass) {
-                        const int j = tile * 128 + r;
-                        const int32_t v = j < K ? __ldg(irow + j) : -1;
-                        const bool valid = v >= 0 && v < kl;
-                        const char *src = kbase_ptr + (valid ? ((int64_t)(kb + v) * D * 2 + chunk * 16) : 0);
-                        const int cb = chunk >> 3;
-                        cp_async16(dst + cb * 16384 + sw128(r, (chunk & 7) * 8), src, valid ? 16 : 0);
-                    }
-                    push(&bars->kv_full[s]);
-                    ++gk;
-                }
+            // the ring slot of item g travelled with item g - 2
+            if (g >= 2) {
+                const uint32_t gp = g - 2;
+                if (!wait_bar(&bars->kv_full[gp % stages], (gp / stages) & 1, &ctl, P.status)) { ok = false; break; }
             }
-            ++tq;
+            const int s = g % stages;
+            if (!wait_bar(&bars->kv_empty[s], ((g / stages) & 1) ^ 1, &ctl, P.status)) { ok = false; break; }
+            const int32_t *slot = ring + (g & 3) * kRingSlot;
+            const int32_t kb = slot[128], kl = slot[129];
+            const int jbase = it0.tile * 128;
+            const uint32_t dst = smem_u32(smem + SP.kv + s * kStageBytes) + (chunk >> 3) * 16384;
+            // this warp's row groups i = warp, warp + 3, ... (a compact loop: the instruction
+            // cache of a sub-partition is shared with two other warp roles)
+#pragma unroll 2
+            for (int i = warp; i < 128 / kRowsPerPass; i += 3) {
+                const int r = rsub + kRowsPerPass * i;
+                const int32_t v = slot[r];
+                const bool valid = jbase + r < K && v >= 0 && v < kl;
+                const char *src = kbase_ptr + (valid ? ((int64_t)(kb + v) * (D * 2) + chunk * 16) : 0);
+                cp_async16(dst + sw128(r, (chunk & 7) * 8), src, valid ? 16 : 0);
+            }
+            if (it2.kind >= 0) fetch_idx(it2, (g + 2) & 3);
+            arrive_on_copies(&bars->kv_full[s]);
+            it0 = it1;
+            it1 = it2;
+            if (it2.kind >= 0) it2 = sc.next();
+            ++g;
         }
-        signal_done(true);
-    } else if (warp == 1) {
+        cp_async_wait<0>();
+    } else if (warp == 3) {
         // =============================== MMA issuer ===============================
-        uint32_t gk = 0, ga = 0, gb = 0, tq = 0;
+        uint32_t gk = 0, gd = 0, nb = 0;       // items, pass-B items, finished B tokens
         bool ok = true;
         const uint32_t kv0 = smem_u32(smem + SP.kv);
         const uint32_t q0 = smem_u32(smem + SP.q);
         const uint32_t ds0 = smem_u32(smem + SP.ds);
-        // S^T[128 keys x N1P] = K_tile . q^T into S buffer ga & 1; returns the K stage used
-        auto issue_s = [&](uint32_t qaddr, int &stage) -> bool {
-            const int s = gk % stages, b = ga & 1;
+        // S^T of item gk into S buffer gk % 2 (pass-A stages are released right away)
+        auto issue_s = [&](const Item &it, int &stage) -> bool {
+            const int s = gk % stages, b = gk & 1;
+            const int qb = it.ord & 1;
+            if (it.kind == 0 && it.first &&
+                !wait_bar(&bars->q_full[qb], (it.ord >> 1) & 1, &ctl, P.status)) return false;
             if (!wait_bar(&bars->kv_full[s], (gk / stages) & 1, &ctl, P.status)) return false;
-            if (!wait_bar(&bars->s_empty[b], ((ga >> 1) & 1) ^ 1, &ctl, P.status)) return false;
+            if (!wait_bar(&bars->s_empty[b], ((gk >> 1) & 1) ^ 1, &ctl, P.status)) return false;
             tc_fence_after();
             if (lane == 0) {
                 const uint32_t kaddr = kv0 + s * kStageBytes;
+                const uint32_t qaddr = q0 + qb * N1P * 256;
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
                     const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
@@ -389,45 +526,34 @@ __global__ void __launch_bounds__(kThreads, 1) fused_sm100(Params P, int stages)
                              sdesc(qaddr + qoff, 16, 1024), kIdescS, ks > 0);
                 }
                 umma_commit(&bars->s_full[b]);
+                if (it.kind == 0) umma_commit(&bars->kv_empty[s]);
             }
             __syncwarp();
             stage = s;
-            ++gk; ++ga;
+            ++gk;
             return true;
         };
-        for (int t = t0; t < t1 && ok; ++t) {
-            const uint64_t mask = P.tok_tiles[t];
-            if (!mask) continue;
-            const int ntile = __popcll(mask);
-            const int qb = tq & 1;
-            const uint32_t qaddr = q0 + qb * N1P * 256;
-            if (!wait_bar(&bars->q_full[qb], (tq >> 1) & 1, &ctl, P.status)) { ok = false; break; }
-            // ---- pass A: S only; the stage is free once the product is done ----
-            for (int i = 0; i < ntile && ok; ++i) {
-                int st;
-                if (!issue_s(qaddr, st)) { ok = false; break; }
-                if (lane == 0) umma_commit(&bars->kv_empty[st]);
-                __syncwarp();
-            }
-            if (!ok) break;
-            // ---- pass B: S again (one tile ahead), dq^T += K^T . dS^T, dK^T = q^T . dS ----
-            if (!wait_bar(&bars->dq_empty, (tq & 1) ^ 1, &ctl, P.status)) { ok = false; break; }
-            int st_cur = 0, st_next = 0;
-            if (!issue_s(qaddr, st_cur)) { ok = false; break; }
-            for (int i = 0; i < ntile; ++i) {
-                if (i + 1 < ntile && !issue_s(qaddr, st_next)) { ok = false; break; }
-                const int b = gb & 1;
-                if (!wait_bar(&bars->ds_full[b], (gb >> 1) & 1, &ctl, P.status)) { ok = false; break; }
-                if (!wait_bar(&bars->dk_empty[b], ((gb >> 1) & 1) ^ 1, &ctl, P.status)) { ok = false; break; }
+        Item cur = sc.next();
+        int st_cur = 0, st_nxt = 0;
+        if (cur.kind >= 0 && !issue_s(cur, st_cur)) ok = false;
+        while (ok && cur.kind >= 0) {
+            const Item nxt = sc.next();
+            if (nxt.kind >= 0 && !issue_s(nxt, st_nxt)) { ok = false; break; }
+            if (cur.kind == 1) {
+                const int b = gd & 1;
+                if (cur.first && !wait_bar(&bars->dq_empty, (nb & 1) ^ 1, &ctl, P.status)) { ok = false; break; }
+                if (!wait_bar(&bars->ds_full[b], (gd >> 1) & 1, &ctl, P.status)) { ok = false; break; }
+                if (!wait_bar(&bars->dk_empty[b], ((gd >> 1) & 1) ^ 1, &ctl, P.status)) { ok = false; break; }
                 tc_fence_after();
                 if (lane == 0) {
                     const uint32_t kaddr = kv0 + st_cur * kStageBytes;
                     const uint32_t dsaddr = ds0 + b * N1P * 256;
+                    const uint32_t qaddr = q0 + (cur.ord & 1) * N1P * 256;
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks) {        // 128 keys, 16 per step
                         const uint64_t a = sdesc(kaddr + ks * 2048, 16384, 1024);
                         const uint64_t bd = sdesc(dsaddr + (ks >> 2) * (N1P * 128) + (ks & 3) * 32, 16, 1024);
-                        umma_f16(tm_dq, a, bd, kIdescDq, (i > 0 || ks > 0) ? 1u : 0u);
+                        umma_f16(tm_dq, a, bd, kIdescDq, (!cur.first || ks > 0) ? 1u : 0u);
                     }
                     umma_commit(&bars->kv_empty[st_cur]);
 #pragma unroll
@@ -437,19 +563,17 @@ __global__ void __launch_bounds__(kThreads, 1) fused_sm100(Params P, int stages)
                         umma_f16(tm_dk + b * 128, a, bd, kIdescDk, ks > 0);
                     }
                     umma_commit(&bars->dk_full[b]);
-                    umma_commit(&bars->ds_empty[b]);
+                    if (cur.last) {
+                        umma_commit(&bars->dq_full);
+                        umma_commit(&bars->q_empty[cur.ord & 1]);
+                    }
                 }
                 __syncwarp();
-                st_cur = st_next;
-                ++gb;
+                if (cur.last) ++nb;
+                ++gd;
             }
-            if (!ok) break;
-            if (lane == 0) {
-                umma_commit(&bars->dq_full);
-                umma_commit(&bars->q_empty[qb]);
-            }
-            __syncwarp();
-            ++tq;
+            cur = nxt;
+            st_cur = st_nxt;
         }
         // drain: wait for every MMA issued by this thread before TMEM is released
         if (lane == 0) umma_commit(&bars->drain);
@@ -458,246 +582,308 @@ __global__ void __launch_bounds__(kThreads, 1) fused_sm100(Params P, int stages)
             long long start = clock64();
             while (!mbar_try_wait(&bars->drain, 0) && clock64() - start < kWaitCycles) {}
         }
-    } else {
-        // =============================== epilogue ===============================
-        const int ew = warp - 2;                 // 0..7
-        const int wg = ew >> 2;                  // warpgroup 0 / 1
-        const int quad = warp & 3;               // TMEM lane quadrant of this warp
-        const int lrow = quad * 32 + lane;       // key slot in tile (pass A/B) or d (scatter)
-        const int et = threadIdx.x - 64;         // 0..255
+    } else if (warp < 8) {
+        // =============================== scatter group ===============================
+        const int quad = warp & 3;
+        const int d = quad * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-        float *ws = reinterpret_cast<float *>(smem + SP.w);
-        int32_t *rows_s = reinterpret_cast<int32_t *>(smem + SP.rows);
-        float *red = reinterpret_cast<float *>(smem + SP.red);
-        uint8_t *ds_tiles = smem + SP.ds;
-        uint32_t ga = 0, gb = 0, tq = 0, ph_epi = 0, ph_wg = 0;
+        uint32_t gd = 0;
         bool ok = true;
-        constexpr int kC = N1P < 32 ? N1P : 32;  // S columns per TMEM load
-        for (int t = t0; t < t1 && ok; ++t) {
-            const uint64_t mask = P.tok_tiles[t];
-            const int32_t kl = P.tok_klen[t], kbs = P.tok_kbase[t];
-            const int32_t *irow = P.idx + (int64_t)t * K;
-            const float *prow = P.p + (int64_t)t * K;
-            float *yrow = P.y + (int64_t)t * K;
-            if (!mask) {
-                for (int j = et; j < K; j += kEpiThreads) yrow[j] = 0.f;
-                for (int e = et; e < P.N1 * D; e += kEpiThreads)
-                    reinterpret_cast<T *>(P.dq)[(int64_t)t * P.N1 * D + e] = T(0.f);
-                for (int h = et; h < P.N1; h += kEpiThreads) P.dw[(int64_t)t * P.N1 + h] = 0.f;
-                continue;
-            }
-            // previous token done with ws / red, then w_t in place
-            if (!group_sync(&bars->epi, ph_epi, &ctl, P.status)) { ok = false; break; }
-            for (int h = et; h < N1P; h += kEpiThreads) ws[h] = h < P.N1 ? P.w[(int64_t)t * P.N1 + h] : 0.f;
-            if (!group_sync(&bars->epi, ph_epi, &ctl, P.status)) { ok = false; break; }
-
-            // ---------------- pass A: I = w . ReLU(S), online max / sum ----------------
-            float m_t = -INFINITY, z_t = 0.f;
-            uint64_t mm = mask;
-            while (mm) {
-                const int tile = __ffsll((long long)mm) - 1;
-                mm &= mm - 1;
-                if ((ga & 1) == (uint32_t)wg) {
-                    const int sb = ga & 1;
-                    const int j = tile * 128 + lrow;
-                    const int32_t v = j < K ? irow[j] : -1;
-                    const bool valid = v >= 0 && v < kl;
-                    if (v != -1 && !valid) set_status(P.status, SLIKL_DEV_INDEX_OUT_OF_RANGE);
-                    if (!wait_bar(&bars->s_full[sb], (ga >> 1) & 1, &ctl, P.status)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t sa = tm_s + sb * N1P + lane_addr;
-                    float sv[32];
-                    float I = 0.f;
+        while (ok) {
+            const Item it = sc.next();
+            if (it.kind < 0) break;
+            if (it.kind != 1) continue;
+            const int b = gd & 1;
+            if (!wait_bar(&bars->rows_full[b], (gd >> 1) & 1, &ctl, P.status)) { ok = false; break; }
+            if (!wait_bar(&bars->dk_full[b], (gd >> 1) & 1, &ctl, P.status)) { ok = false; break; }
+            tc_fence_after();
+            if (quad * 32 < D) {
+                // 4 chunks of 32 keys, one compact loop body (the instruction cache of a
+                // sub-partition is shared with two other warp roles)
+                const int4 *rs4 = reinterpret_cast<const int4 *>(rows_s + b * kRowsStride);
+                const int64_t slot0 = (int64_t)it.t * K + it.tile * 128;
+                const uint32_t da = tm_dk + b * 128 + lane_addr;
+#pragma unroll 1
+                for (int ch = 0; ch < 4; ++ch) {
+                    float vals[32];
+                    tmem_ld32(da + ch * 32, vals);
+                    int32_t rr[32];
 #pragma unroll
-                    for (int c = 0; c < N1P; c += kC) {
-                        if (kC == 32) tmem_ld32(sa + c, sv); else tmem_ld16(sa + c, sv);
-                        tmem_wait_ld();
+                    for (int u = 0; u < 8; ++u) {
+                        const int4 q4 = rs4[ch * 8 + u];
+                        rr[4 * u] = q4.x; rr[4 * u + 1] = q4.y; rr[4 * u + 2] = q4.z; rr[4 * u + 3] = q4.w;
+                    }
+                    tmem_wait_ld();
+                    if (!P.deterministic) {
 #pragma unroll
-                        for (int h = 0; h < kC; ++h) I = fmaf(ws[c + h], fmaxf(sv[h], 0.f), I);
+                        for (int c = 0; c < 32; ++c)
+                            if (rr[c] >= 0) red_add_f32(P.dk_acc + (int64_t)rr[c] * D + d, vals[c]);
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            if (rr[c] >= 0) P.partials[(slot0 + ch * 32 + c) * D + d] = vals[c];
                     }
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&bars->s_empty[sb]);
-                    if (valid) {
-                        if (I > m_t) {
-                            z_t = (m_t == -INFINITY) ? 0.f : z_t * __expf(m_t - I);
-                            m_t = I;
-                        }
-                        z_t += __expf(I - m_t);
-                    }
-                    if (j < K) yrow[j] = valid ? I : -INFINITY;       // parked for pass B
                 }
-                ++ga;
             }
-            if (!ok) break;
-
-            // ---------------- softmax statistics over the token ----------------
-            float mw = m_t;
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->dk_empty[b]);
+            ++gd;
+        }
+    } else {
+        // =============================== softmax group ===============================
+        const int ew = warp - 8;                 // 0..3
+        const int quad = warp & 3;
+        const int lrow = quad * 32 + lane;       // key slot in the tile, or d for dq
+        const int et = threadIdx.x - 256;        // 0..127
+        const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+        float *wsm = reinterpret_cast<float *>(smem + SP.w);      // [2][N1P]
+        float *red = reinterpret_cast<float *>(smem + SP.red);    // [4][64]
+        uint8_t *ds_tiles = smem + SP.ds;
+        uint32_t gk = 0, gd = 0, nb = 0, ph = 0;
+        bool ok = true;
+        // tokens of the range without any active tile: zero outputs
+        for (int t = t0; t < t1; ++t) {
+            if (P.tok_tiles[t]) continue;
+            for (int j = et; j < K; j += 128) P.y[(int64_t)t * K + j] = 0.f;
+            for (int e = et; e < P.N1 * D; e += 128)
+                reinterpret_cast<T *>(P.dq)[(int64_t)t * P.N1 * D + e] = T(0.f);
+            for (int h = et; h < P.N1; h += 128) P.dw[(int64_t)t * P.N1 + h] = 0.f;
+        }
+        float m_a = -INFINITY, z_a = 0.f;        // pass-A token: running max / sum
+        float M_n = -INFINITY, iZ_n = 0.f;       // its combined statistics, handed to pass B
+        float M_b = -INFINITY, iZ_b = 0.f;       // pass-B token
+        // per-slot inputs of the next item are loaded while the current one is processed
+        struct Pre { int32_t v, kl, kb; float p, I; bool haveI; };
+        auto prefetch = [&](const Item &nx, const Item &cu, Pre &o) {
+            const int jn = nx.tile * 128 + lrow;
+            const int64_t ro = (int64_t)nx.t * K;
+            o.kl = P.tok_klen[nx.t];
+            o.kb = P.tok_kbase[nx.t];
+            o.v = jn < K ? P.idx[ro + jn] : -1;
+            o.p = (nx.kind == 1 && jn < K) ? P.p[ro + jn] : 0.f;
+            // the parked logit of a pass-B tile is written by the pass-A item of the same
+            // tile; when that is the current item it is read later, after it has been parked
+            o.haveI = nx.kind == 1 && !(cu.kind == 0 && cu.t == nx.t && cu.tile == nx.tile);
+            o.I = (o.haveI && jn < K) ? P.y[ro + jn] : 0.f;
+        };
+        Item it = sc.next();
+        Pre cur{};
+        if (it.kind >= 0) {
+            Item none;
+            none.kind = -1;
+            prefetch(it, none, cur);
+        }
+        while (ok && it.kind >= 0) {
+            const Item nx = sc.next();
+            Pre nxt{};
+            // pass-A items load the next item's inputs right away; pass-B items after their
+            // proxy fence (which would otherwise also wait for these loads)
+            if (nx.kind >= 0 && it.kind == 0) prefetch(nx, it, nxt);
+            const int sb = gk & 1;
+            const float *ws = wsm + (it.ord & 1) * N1P;
+            const int32_t kl = cur.kl;
+            const int j = it.tile * 128 + lrow;
+            const int64_t row_off = (int64_t)it.t * K;
+            if (it.kind == 0) {
+                // ---------------- pass A item ----------------
+                if (it.first) {
+                    // w of the new token into its buffer (the token two ordinals back is done)
+                    for (int h = et; h < N1P; h += 128)
+                        wsm[(it.ord & 1) * N1P + h] = h < P.N1 ? P.w[(int64_t)it.t * P.N1 + h] : 0.f;
+                    if (!group_sync(&bars->sm_sync, ph, &ctl, P.status)) { ok = false; break; }
+                    m_a = -INFINITY;
+                    z_a = 0.f;
+                }
+                const int32_t v = cur.v;
+                const bool valid = v >= 0 && v < kl;
+                if (v != -1 && !valid) set_status(P.status, SLIKL_DEV_INDEX_OUT_OF_RANGE);
+                if (!wait_bar(&bars->s_full[sb], (gk >> 1) & 1, &ctl, P.status)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t sa = tm_s + sb * N1P + lane_addr;
+                float sv[32];
+                float I = 0.f;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) mw = fmaxf(mw, __shfl_xor_sync(0xffffffffu, mw, o));
-            if (lane == 0) ctl.stat_m[ew] = mw;
-            if (!group_sync(&bars->epi, ph_epi, &ctl, P.status)) { ok = false; break; }
-            float M = -INFINITY;
+                for (int c = 0; c < N1P; c += kC) {
+                    if (kC == 32) tmem_ld32(sa + c, sv); else tmem_ld16(sa + c, sv);
+                    float wv[32];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) M = fmaxf(M, ctl.stat_m[i]);
-            const float zs = (m_t == -INFINITY) ? 0.f : z_t * __expf(m_t - M);
-            float zw = zs;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) zw += __shfl_xor_sync(0xffffffffu, zw, o);
-            if (lane == 0) ctl.stat_z[ew] = zw;
-            if (!group_sync(&bars->epi, ph_epi, &ctl, P.status)) { ok = false; break; }
-            float Z = 0.f;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) Z += ctl.stat_z[i];
-            const float invZ = Z > 0.f ? 1.f / Z : 0.f;
-
-            // ---------------- pass B: y, dI, dS, dW; dK scatter ----------------
-            float dW[N1P];
-#pragma unroll
-            for (int h = 0; h < N1P; ++h) dW[h] = 0.f;
-            mm = mask;
-            while (mm) {
-                const int tile = __ffsll((long long)mm) - 1;
-                mm &= mm - 1;
-                if ((gb & 1) == (uint32_t)wg) {
-                    const int b = wg;
-                    const int sb = ga & 1;
-                    const int j = tile * 128 + lrow;
-                    const int32_t v = j < K ? irow[j] : -1;
-                    const bool valid = v >= 0 && v < kl;
-                    float dI = 0.f;
-                    if (j < K) {
-                        const float I = yrow[j];
-                        const float y = valid ? __expf(I - M) * invZ : 0.f;
-                        yrow[j] = y;
-                        dI = valid ? y - prow[j] : 0.f;
+                    for (int h = 0; h < kC; h += 4) {
+                        const float4 w4 = *reinterpret_cast<const float4 *>(ws + c + h);
+                        wv[h] = w4.x; wv[h + 1] = w4.y; wv[h + 2] = w4.z; wv[h + 3] = w4.w;
                     }
-                    if (!wait_bar(&bars->ds_empty[b], ((gb >> 1) & 1) ^ 1, &ctl, P.status)) { ok = false; break; }
-                    if (!wait_bar(&bars->s_full[sb], (ga >> 1) & 1, &ctl, P.status)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t sa = tm_s + sb * N1P + lane_addr;
-                    uint8_t *dsb = ds_tiles + b * N1P * 256 + (lrow >> 6) * (N1P * 128);
-                    const int jj = lrow & 63;
-                    float sv[32];
+                    tmem_wait_ld();
+                    float i4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int c = 0; c < N1P; c += kC) {
-                        if (kC == 32) tmem_ld32(sa + c, sv); else tmem_ld16(sa + c, sv);
-                        tmem_wait_ld();
+                    for (int h = 0; h < kC; ++h) i4[h & 3] = fmaf(wv[h], fmaxf(sv[h], 0.f), i4[h & 3]);
+                    I += (i4[0] + i4[1]) + (i4[2] + i4[3]);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->s_empty[sb]);
+                if (valid) {
+                    if (I > m_a) {
+                        z_a = (m_a == -INFINITY) ? 0.f : z_a * __expf(m_a - I);
+                        m_a = I;
+                    }
+                    z_a += __expf(I - m_a);
+                }
+                if (j < K) P.y[row_off + j] = valid ? I : -INFINITY;       // parked for pass B
+                if (it.last) {
+                    // combine max and sum over the 128 threads (fixed order)
+                    float mw = m_a;
 #pragma unroll
-                        for (int h = 0; h < kC; ++h) {
-                            const float sval = sv[h];
-                            dW[c + h] = fmaf(dI, fmaxf(sval, 0.f), dW[c + h]);
-                            const float d = sval > 0.f ? dI * ws[c + h] : 0.f;
-                            *reinterpret_cast<uint16_t *>(dsb + sw128(c + h, jj)) = to_bits16<T>(d);
+                    for (int o = 16; o > 0; o >>= 1) mw = fmaxf(mw, __shfl_xor_sync(0xffffffffu, mw, o));
+                    if (lane == 0) ctl.stat_m[ew] = mw;
+                    if (!group_sync(&bars->sm_sync, ph, &ctl, P.status)) { ok = false; break; }
+                    float M = -INFINITY;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) M = fmaxf(M, ctl.stat_m[i]);
+                    float zw = (m_a == -INFINITY) ? 0.f : z_a * __expf(m_a - M);
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) zw += __shfl_xor_sync(0xffffffffu, zw, o);
+                    if (lane == 0) ctl.stat_z[ew] = zw;
+                    if (!group_sync(&bars->sm_sync, ph, &ctl, P.status)) { ok = false; break; }
+                    float Z = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) Z += ctl.stat_z[i];
+                    M_n = M;
+                    iZ_n = Z > 0.f ? 1.f / Z : 0.f;
+                    // stat_m / stat_z are rewritten only after two more group syncs
+                }
+            } else {
+                // ---------------- pass B item ----------------
+                if (it.first) {
+                    M_b = M_n;
+                    iZ_b = iZ_n;
+                }
+                const int b = gd & 1;
+                const int32_t v = cur.v;
+                const bool valid = v >= 0 && v < kl;
+                float dI = 0.f, y = 0.f;
+                if (j < K) {
+                    const float I = cur.haveI ? cur.I : P.y[row_off + j];
+                    y = valid ? __expf(I - M_b) * iZ_b : 0.f;
+                    dI = valid ? y - cur.p : 0.f;
+                }
+                // dS tile / key rows of buffer b free once the scatter of its previous use ended
+                if (!wait_bar(&bars->dk_empty[b], ((gd >> 1) & 1) ^ 1, &ctl, P.status)) { ok = false; break; }
+                if (!wait_bar(&bars->s_full[sb], (gk >> 1) & 1, &ctl, P.status)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t sa = tm_s + sb * N1P + lane_addr;
+                const uint32_t dwa = tm_dw + lane_addr;
+                uint8_t *dsb = ds_tiles + b * N1P * 256 + (lrow >> 6) * (N1P * 128);
+                const int jj = lrow & 63;
+                // 16 heads at a time: dS to smem; this slot's dW partial sums stay in TMEM
+#pragma unroll 1
+                for (int c = 0; c < N1P; c += 16) {
+                    float sv[16], acc[16], wv[16];
+                    tmem_ld16(sa + c, sv);
+                    if (!it.first) tmem_ld16(dwa + c, acc);
+#pragma unroll
+                    for (int h = 0; h < 16; h += 4) {
+                        const float4 w4 = *reinterpret_cast<const float4 *>(ws + c + h);
+                        wv[h] = w4.x; wv[h + 1] = w4.y; wv[h + 2] = w4.z; wv[h + 3] = w4.w;
+                    }
+                    tmem_wait_ld();
+                    uint8_t *dsc = dsb + c * 128;
+#pragma unroll
+                    for (int h = 0; h < 16; ++h) {
+                        const float sval = sv[h];
+                        const float a0 = it.first ? 0.f : acc[h];
+                        acc[h] = fmaf(dI, fmaxf(sval, 0.f), a0);
+                        const float dsv = sval > 0.f ? dI * wv[h] : 0.f;
+                        *reinterpret_cast<uint16_t *>(dsc + sw128(h, jj)) = to_bits16<T>(dsv);
+                    }
+                    tmem_st16(dwa + c, acc);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->s_empty[sb]);
+                rows_s[b * kRowsStride + lrow] = valid ? cur.kb + v : -1;
+                fence_proxy_async();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&bars->ds_full[b]);
+                    mbar_arrive(&bars->rows_full[b]);
+                }
+                if (j < K) P.y[row_off + j] = y;
+                if (nx.kind >= 0) prefetch(nx, it, nxt);
+                ++gd;
+                if (it.last) {
+                    // softmax_out of the token's inactive tiles
+                    const uint64_t mask = P.tok_tiles[it.t];
+                    const int ntiles = (K + 127) / 128;
+                    for (int tl = 0; tl < ntiles; ++tl) {
+                        if ((mask >> tl) & 1) continue;
+                        for (int jz = tl * 128 + et; jz < (tl + 1) * 128 && jz < K; jz += 128) P.y[row_off + jz] = 0.f;
+                    }
+                    // dW: this slot's partial sums from TMEM; butterfly reduce-scatter within each
+                    // warp, then the 4 warps in order
+                    constexpr int kV = N1P < 32 ? 32 : N1P;
+                    float vv[kV];
+#pragma unroll
+                    for (int h = 0; h < kV; ++h) vv[h] = 0.f;
+#pragma unroll
+                    for (int c = 0; c < N1P; c += 16) tmem_ld16(tm_dw + lane_addr + c, vv + c);
+                    tmem_wait_ld();
+                    int len = kV;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) {
+                        const int half = len >> 1;
+                        const bool upper = (lane & o) != 0;
+#pragma unroll
+                        for (int h = 0; h < kV / 2; ++h) {
+                            if (h < half) {
+                                const float mine = upper ? vv[h + half] : vv[h];
+                                const float other = upper ? vv[h] : vv[h + half];
+                                vv[h] = mine + __shfl_xor_sync(0xffffffffu, other, o);
+                            }
                         }
+                        len = half;
                     }
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&bars->s_empty[sb]);
-                    rows_s[b * 128 + lrow] = valid ? kbs + v : -1;
-                    fence_proxy_async();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&bars->ds_full[b]);
-                    // rows_s of this tile visible to the whole group
-                    if (!group_sync(&bars->wgb[wg], ph_wg, &ctl, P.status)) { ok = false; break; }
-                    if (!wait_bar(&bars->dk_full[b], (gb >> 1) & 1, &ctl, P.status)) { ok = false; break; }
+                    int base = 0, span = kV;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) {
+                        span >>= 1;
+                        if (lane & o) base += span;
+                    }
+#pragma unroll
+                    for (int h = 0; h < kV / 32; ++h) red[ew * 64 + base + h] = vv[h];
+                    if (!group_sync(&bars->sm_sync, ph, &ctl, P.status)) { ok = false; break; }
+                    for (int h = et; h < P.N1; h += 128) {
+                        float a = 0.f;
+                        for (int i = 0; i < 4; ++i) a += red[i * 64 + h];
+                        P.dw[(int64_t)it.t * P.N1 + h] = a;
+                    }
+                    // dq^T readback (lane = d): columns = heads
+                    if (!wait_bar(&bars->dq_full, nb & 1, &ctl, P.status)) { ok = false; break; }
                     tc_fence_after();
                     if (quad * 32 < D) {
-                        const uint32_t da = tm_dk + b * 128 + lane_addr;
-                        const int d = lrow;
+                        T *dqrow = reinterpret_cast<T *>(P.dq) + (int64_t)it.t * P.N1 * D;
                         float dv[32];
-#pragma unroll 1
-                        for (int c0 = 0; c0 < 128; c0 += 32) {
-                            tmem_ld32(da + c0, dv);
+#pragma unroll
+                        for (int c0 = 0; c0 < N1P; c0 += kC) {
+                            if (kC == 32) tmem_ld32(tm_dq + lane_addr + c0, dv); else tmem_ld16(tm_dq + lane_addr + c0, dv);
                             tmem_wait_ld();
 #pragma unroll
-                            for (int c = 0; c < 32; ++c) {
-                                const int32_t r = rows_s[b * 128 + c0 + c];
-                                if (r >= 0) {
-                                    if (P.deterministic)
-                                        P.partials[((int64_t)t * K + tile * 128 + c0 + c) * D + d] = dv[c];
-                                    else
-                                        red_add_f32(P.dk_acc + (int64_t)r * D + d, dv[c]);
-                                }
+                            for (int c = 0; c < kC; ++c) {
+                                const int h = c0 + c;
+                                if (h < P.N1) dqrow[(int64_t)h * D + lrow] = T(dv[c]);
                             }
                         }
                     }
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&bars->dk_empty[b]);
-                    // rows_s reads done before its next write
-                    if (!group_sync(&bars->wgb[wg], ph_wg, &ctl, P.status)) { ok = false; break; }
-                }
-                ++gb;
-                ++ga;
-            }
-            if (!ok) break;
-            // slots of inactive tiles: softmax_out = 0
-            {
-                const int ntiles = (K + 127) / 128;
-                for (int tile = 0; tile < ntiles; ++tile) {
-                    if ((mask >> tile) & 1) continue;
-                    for (int j = tile * 128 + et; j < (tile + 1) * 128 && j < K; j += kEpiThreads) yrow[j] = 0.f;
+                    if (lane == 0) mbar_arrive(&bars->dq_empty);
+                    ++nb;
+                    // red is rewritten only after the next token's group syncs
                 }
             }
-            // ---------------- dW: fixed-order reduction over the 256 threads ----------------
-            // butterfly reduce-scatter within the warp, then the 8 warps in index order
-            {
-                constexpr int kV = N1P < 32 ? 32 : N1P;
-                float vv[kV];
-#pragma unroll
-                for (int h = 0; h < kV; ++h) vv[h] = h < N1P ? dW[h] : 0.f;
-                int len = kV;
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    const int half = len >> 1;
-                    const bool upper = (lane & o) != 0;
-#pragma unroll
-                    for (int h = 0; h < kV / 2; ++h) {
-                        if (h < half) {
-                            const float mine = upper ? vv[h + half] : vv[h];
-                            const float other = upper ? vv[h] : vv[h + half];
-                            vv[h] = mine + __shfl_xor_sync(0xffffffffu, other, o);
-                        }
-                    }
-                    len = half;
-                }
-                int base = 0, span = kV;
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    span >>= 1;
-                    if (lane & o) base += span;
-                }
-#pragma unroll
-                for (int h = 0; h < kV / 32; ++h) red[ew * 64 + base + h] = vv[h];
-            }
-            if (!group_sync(&bars->epi, ph_epi, &ctl, P.status)) { ok = false; break; }
-            for (int h = et; h < P.N1; h += kEpiThreads) {
-                float a = 0.f;
-                for (int i = 0; i < 8; ++i) a += red[i * 64 + h];
-                P.dw[(int64_t)t * P.N1 + h] = a;
-            }
-            // ---------------- dq^T readback ----------------
-            if (!wait_bar(&bars->dq_full, tq & 1, &ctl, P.status)) { ok = false; break; }
-            tc_fence_after();
-            if (quad * 32 < D) {
-                constexpr int kHalf = N1P / 2;               // heads read by this warpgroup
-                const uint32_t qa = tm_dq + wg * kHalf + lane_addr;
-                float dv[32];
-                const int d = lrow;
-                T *dqrow = reinterpret_cast<T *>(P.dq) + (int64_t)t * P.N1 * D;
-                if (kHalf >= 32) tmem_ld32(qa, dv); else tmem_ld16(qa, dv);
-                tmem_wait_ld();
-#pragma unroll
-                for (int c = 0; c < (kHalf < 32 ? kHalf : 32); ++c) {
-                    const int h = wg * kHalf + c;
-                    if (h < P.N1) dqrow[(int64_t)h * D + d] = T(dv[c]);
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->dq_empty);
-            ++tq;
+            ++gk;
+            it = nx;
+            cur = nxt;
         }
     }
 
@@ -705,7 +891,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_sm100(Params P, int stages)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) {
+    if (warp == 3) {
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                      "r"(kTmemCols));
     }
@@ -713,33 +899,13 @@ __global__ void __launch_bounds__(kThreads, 1) fused_sm100(Params P, int stages)
 
 template <int N1P, int D, typename T>
 cudaError_t launch_t(const Params &P, int workers, cudaStream_t s) {
-    int stages = 4;
-    SmemPlan sp = plan_smem<N1P>(P.K, stages);
-    while (sp.total > 226 * 1024 && stages > 2) {
-        --stages;
-        sp = plan_smem<N1P>(P.K, stages);
-    }
+    const int stages = 4;
+    const SmemPlan sp = plan_smem<N1P>(stages);
     if (sp.total > 226 * 1024) return cudaErrorInvalidConfiguration;
-    // The producer signals a gathered tile LAG groups late; in pass B the MMA warp holds two
-    // stages (S of tile i+1 is issued before the dq product of tile i), so LAG <= stages - 2
-    // keeps the producer from waiting on a stage that only a later signal could free.
-    cudaError_t e;
-    if (stages == 4) {
-        auto k = fused_sm100<N1P, D, T, 2>;
-        e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp.total);
-        if (e != cudaSuccess) return e;
-        k<<<workers, kThreads, sp.total, s>>>(P, stages);
-    } else if (stages == 3) {
-        auto k = fused_sm100<N1P, D, T, 1>;
-        e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp.total);
-        if (e != cudaSuccess) return e;
-        k<<<workers, kThreads, sp.total, s>>>(P, stages);
-    } else {
-        auto k = fused_sm100<N1P, D, T, 0>;
-        e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp.total);
-        if (e != cudaSuccess) return e;
-        k<<<workers, kThreads, sp.total, s>>>(P, stages);
-    }
+    auto k = fused_sm100<N1P, D, T>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp.total);
+    if (e != cudaSuccess) return e;
+    k<<<workers, kThreads, sp.total, s>>>(P, stages);
     return cudaGetLastError();
 }
 
