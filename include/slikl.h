@@ -76,7 +76,9 @@ typedef int32_t slikl_status;
  *                    cu_seqlens_q [B+1] on the device with cu_seqlens_q[0] = 0 and
  *                    cu_seqlens_q[B] = T1; S1 is ignored.
  *   layout_k = BSND: k/dk [B,S2,1,D], requires S2 > 0; T2 is ignored (taken as B*S2).
- *   layout_k = TND:  k/dk [T2,1,D], cu_seqlens_k [B+1] on the device, cu_seqlens_k[B] = T2.
+ *   layout_k = TND:  k/dk [T2,1,D], cu_seqlens_k [B+1] on the device, cu_seqlens_k[B] = T2;
+ *                    S2 > 0 promises that no batch has more than S2 key rows (it lets the
+ *                    key-major dK path size its records; 0 = no promise, that path is off).
  *
  * The key tensor has one head (N2 = 1): the page's formulas carry no key-head index.
  * Valid indices of a batch-b token are local to batch b's key range: key row =
@@ -92,7 +94,7 @@ typedef struct {
     int32_t layout_k;        /* SLIKL_BSND or SLIKL_TND */
     int32_t deterministic;   /* 0 or 1 */
     int64_t B;               /* batches (TND: number of sequences = len(cu_seqlens) - 1) */
-    int64_t S1, S2;          /* BSND query / key lengths */
+    int64_t S1, S2;          /* BSND query / key lengths; TND keys: S2 = longest key range or 0 */
     int64_t T1, T2;          /* TND total query / key rows */
     int64_t N1, D, topk;     /* query heads, head dim, top-k slots per token */
 } slikl_problem;
@@ -139,10 +141,49 @@ SLIKL_API slikl_status slikl_grad(const slikl_problem *problem, const slikl_tens
                         void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * dK paths (slikl_options.dk_path). Both give the same dK up to the order of fp32 additions.
+ *   SLIKL_DK_SCATTER   every named slot adds its dK row into an fp32 accumulator with
+ *                      atomic adds (the page's default), or, deterministic = 1, stores it for
+ *                      the key-major sort and fixed-order reduction;
+ *   SLIKL_DK_KEYMAJOR  the fused kernel stores, per named (query row, key), dI and the heads
+ *                      with S > 0; a second tensor-core kernel then forms dK one 256-key block
+ *                      at a time from every query row that names a key of the block.
+ *                      Needs N1 <= 64, deterministic = 0 and a key-range bound
+ *                      (BSND: S2; TND: problem->S2 > 0) of at most 16384 keys; its workspace
+ *                      holds T1 x roundup(S2, 256) records of 8 (N1 <= 32) or 16 bytes.
+ *   SLIKL_DK_AUTO      the key-major path when it is possible, the key range is at most 16x
+ *                      topk and its records take at most 8 GiB; else the scatter path.
+ * The workspace size depends on the path: size and launch with the same options.
+ */
+#define SLIKL_DK_AUTO     0
+#define SLIKL_DK_SCATTER  1
+#define SLIKL_DK_KEYMAJOR 2
+
+typedef struct {
+    int32_t dk_path;     /* SLIKL_DK_AUTO, SLIKL_DK_SCATTER or SLIKL_DK_KEYMAJOR */
+    void *fused_begin;   /* optional cudaEvent_t recorded just before the fused kernel, or NULL */
+    void *fused_end;     /* optional cudaEvent_t recorded just after it, or NULL */
+} slikl_options;
+
+/*
+ * slikl_grad_workspace_size / slikl_grad with options (NULL options = SLIKL_DK_AUTO, no
+ * events; slikl_grad_workspace_size and slikl_grad are these calls with NULL options).
+ * Errors: as the plain calls; SLIKL_ERR_PARAM_INVALID also for an unknown dk_path or
+ * SLIKL_DK_KEYMAJOR on a problem that path cannot run.
+ */
+SLIKL_API slikl_status slikl_grad_workspace_size_ex(const slikl_problem *problem,
+                                                    const slikl_options *options,
+                                                    size_t *workspace_bytes);
+SLIKL_API slikl_status slikl_grad_ex(const slikl_problem *problem, const slikl_tensors *tensors,
+                                     void *workspace, size_t workspace_bytes, void *stream,
+                                     const slikl_options *options);
+
+/*
  * slikl_grad with a measurement aid: when fused_begin / fused_end are not NULL they are
  * cudaEvent_t handles (created by the caller) recorded on `stream` immediately before and
  * after the fused per-token kernel, so its duration can be read with cudaEventElapsedTime.
- * Everything else, including errors, is as slikl_grad (which is this call with NULL events).
+ * Everything else, including errors, is as slikl_grad (which is this call with NULL events);
+ * the same as slikl_grad_ex with SLIKL_DK_AUTO and these events.
  */
 SLIKL_API slikl_status slikl_grad_with_events(const slikl_problem *problem,
                                               const slikl_tensors *tensors, void *workspace,
@@ -155,6 +196,9 @@ SLIKL_API slikl_status slikl_grad_with_events(const slikl_problem *problem,
 #define SLIKL_DEV_BAD_CU_SEQLENS_K    0x4u  /* cu_seqlens_k not 0..T2 non-decreasing; the key
                                                ranges of the batches were emptied            */
 #define SLIKL_DEV_WAIT_TIMEOUT        0x8u  /* an internal bounded wait gave up; outputs invalid */
+#define SLIKL_DEV_KEY_RANGE_ABOVE_S2  0x10u /* key-major dK path: a batch holds more key rows
+                                               than problem->S2 promised (TND); the rows of
+                                               that batch are left out, outputs invalid    */
 
 /*
  * Copies the status word of the last slikl_grad call that used `workspace` (device) into

@@ -35,8 +35,15 @@ SLIKL_DEV_INDEX_OUT_OF_RANGE = 0x1
 SLIKL_DEV_BAD_CU_SEQLENS_Q = 0x2
 SLIKL_DEV_BAD_CU_SEQLENS_K = 0x4
 SLIKL_DEV_WAIT_TIMEOUT = 0x8
+SLIKL_DEV_KEY_RANGE_ABOVE_S2 = 0x10
+
+SLIKL_DK_AUTO = 0
+SLIKL_DK_SCATTER = 1
+SLIKL_DK_KEYMAJOR = 2
+_DK_PATHS = {"auto": SLIKL_DK_AUTO, "scatter": SLIKL_DK_SCATTER, "keymajor": SLIKL_DK_KEYMAJOR}
 
 EXPORTED = ("slikl_grad_workspace_size", "slikl_grad", "slikl_grad_with_events",
+            "slikl_grad_workspace_size_ex", "slikl_grad_ex",
             "slikl_read_device_status",
             "slikl_grad_metadata_size", "slikl_grad_metadata_workspace_size",
             "slikl_grad_metadata", "slikl_status_string", "slikl_grad_noalloc")
@@ -56,6 +63,19 @@ class slikl_tensors(ctypes.Structure):
     _fields_ = [(name, ctypes.c_void_p) for name in
                 ("q", "k", "w", "attn_softmax_l1norm", "sparse_indices", "cu_seqlens_q",
                  "cu_seqlens_k", "dq", "dk", "dw", "softmax_out")]
+
+
+class slikl_options(ctypes.Structure):
+    _fields_ = [("dk_path", ctypes.c_int32), ("fused_begin", ctypes.c_void_p),
+                ("fused_end", ctypes.c_void_p)]
+
+
+def make_options(dk_path="auto", fused_begin: int = 0, fused_end: int = 0) -> slikl_options:
+    o = slikl_options()
+    o.dk_path = _DK_PATHS[dk_path] if isinstance(dk_path, str) else int(dk_path)
+    o.fused_begin = fused_begin or None
+    o.fused_end = fused_end or None
+    return o
 
 
 class SliklError(RuntimeError):
@@ -79,6 +99,10 @@ def load_library() -> ctypes.CDLL:
         lib.slikl_grad.argtypes = [P(slikl_problem), P(slikl_tensors), VP, ctypes.c_size_t, VP]
         lib.slikl_grad_with_events.argtypes = [P(slikl_problem), P(slikl_tensors), VP,
                                                ctypes.c_size_t, VP, VP, VP]
+        lib.slikl_grad_workspace_size_ex.argtypes = [P(slikl_problem), P(slikl_options),
+                                                     P(ctypes.c_size_t)]
+        lib.slikl_grad_ex.argtypes = [P(slikl_problem), P(slikl_tensors), VP, ctypes.c_size_t,
+                                      VP, P(slikl_options)]
         lib.slikl_read_device_status.argtypes = [VP, VP, P(ctypes.c_uint32)]
         lib.slikl_grad_metadata_size.argtypes = [ctypes.c_int32]
         lib.slikl_grad_metadata_size.restype = ctypes.c_int64
@@ -90,7 +114,7 @@ def load_library() -> ctypes.CDLL:
         lib.slikl_status_string.argtypes = [ctypes.c_int32]
         lib.slikl_status_string.restype = ctypes.c_char_p
         for name in ("slikl_grad_workspace_size", "slikl_grad", "slikl_grad_with_events",
-                     "slikl_read_device_status",
+                     "slikl_grad_workspace_size_ex", "slikl_grad_ex", "slikl_read_device_status",
                      "slikl_grad_metadata_workspace_size", "slikl_grad_metadata"):
             getattr(lib, name).restype = ctypes.c_int32
         _lib = lib
@@ -127,6 +151,26 @@ def slikl_grad_with_events(problem: slikl_problem, tensors: slikl_tensors, works
                                                fused_begin or None, fused_end or None)
     if rc != SLIKL_OK:
         raise SliklError(rc, "slikl_grad_with_events")
+
+
+def slikl_grad_workspace_size_ex(problem: slikl_problem, options: Optional[slikl_options]) -> int:
+    n = ctypes.c_size_t(0)
+    rc = load_library().slikl_grad_workspace_size_ex(
+        ctypes.byref(problem), ctypes.byref(options) if options is not None else None,
+        ctypes.byref(n))
+    if rc != SLIKL_OK:
+        raise SliklError(rc, "slikl_grad_workspace_size_ex")
+    return int(n.value)
+
+
+def slikl_grad_ex(problem: slikl_problem, tensors: slikl_tensors, workspace: int,
+                  workspace_bytes: int, stream: int = 0,
+                  options: Optional[slikl_options] = None) -> None:
+    rc = load_library().slikl_grad_ex(ctypes.byref(problem), ctypes.byref(tensors), workspace,
+                                      workspace_bytes, stream,
+                                      ctypes.byref(options) if options is not None else None)
+    if rc != SLIKL_OK:
+        raise SliklError(rc, "slikl_grad_ex")
 
 
 def slikl_read_device_status(workspace: int, stream: int = 0) -> int:
@@ -174,8 +218,11 @@ _DT = {torch.bfloat16: SLIKL_BF16, torch.float16: SLIKL_FP16}
 
 def make_problem(q: torch.Tensor, k: torch.Tensor, sparse_indices: torch.Tensor,
                  layout_q: str = "BSND", layout_k: str = "BSND", deterministic: bool = False,
-                 B: Optional[int] = None) -> slikl_problem:
-    """Problem struct from tensor shapes (BSND q [B,S1,N1,D]; TND q [T1,N1,D])."""
+                 B: Optional[int] = None, key_range_bound: int = 0) -> slikl_problem:
+    """Problem struct from tensor shapes (BSND q [B,S1,N1,D]; TND q [T1,N1,D]).
+
+    For TND keys, `key_range_bound` (> 0) promises that no batch has more key rows; it goes
+    to problem.S2 and lets the key-major dK path run."""
     pr = slikl_problem()
     if q.dtype not in _DT or k.dtype != q.dtype:
         raise ValueError("q and k must share dtype float16 or bfloat16")
@@ -196,6 +243,7 @@ def make_problem(q: torch.Tensor, k: torch.Tensor, sparse_indices: torch.Tensor,
         pr.T2 = k.shape[0] * k.shape[1]
     else:
         pr.T2 = k.shape[0]
+        pr.S2 = int(key_range_bound)
     pr.topk = sparse_indices.shape[-1]
     return pr
 
@@ -210,18 +258,21 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
 
 def grad(q, k, w, attn_softmax_l1norm, sparse_indices, layout_q="BSND", layout_k="BSND",
          cu_seqlens_q=None, cu_seqlens_k=None, deterministic=False, stream=None, out=None,
-         workspace=None):
-    """Run slikl_grad on CUDA tensors. Returns dict(dq, dk, dw, softmax_out, workspace).
+         workspace=None, dk_path="auto", key_range_bound=0):
+    """Run slikl_grad_ex on CUDA tensors. Returns dict(dq, dk, dw, softmax_out, workspace).
 
-    `out` may supply preallocated dq/dk/dw/softmax_out, `workspace` a uint8 CUDA buffer.
+    `out` may supply preallocated dq/dk/dw/softmax_out, `workspace` a uint8 CUDA buffer;
+    `dk_path` is "auto", "scatter" or "keymajor"; `key_range_bound` as in make_problem.
     """
     B = None
     if layout_q == "TND":
         B = cu_seqlens_q.numel() - 1
     elif layout_k == "TND":
         B = cu_seqlens_k.numel() - 1
-    pr = make_problem(q, k, sparse_indices, layout_q, layout_k, deterministic, B)
-    nbytes = slikl_grad_workspace_size(pr)
+    pr = make_problem(q, k, sparse_indices, layout_q, layout_k, deterministic, B,
+                      key_range_bound)
+    opt = make_options(dk_path)
+    nbytes = slikl_grad_workspace_size_ex(pr, opt)
     if workspace is None or workspace.numel() < nbytes:
         workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device)
     if out is None:
@@ -236,17 +287,26 @@ def grad(q, k, w, attn_softmax_l1norm, sparse_indices, layout_q="BSND", layout_k
     tn.dq, tn.dk, tn.dw = _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dw"])
     tn.softmax_out = _ptr(out["softmax_out"])
     s = stream if stream is not None else torch.cuda.current_stream(q.device)
-    slikl_grad(pr, tn, workspace.data_ptr(), workspace.numel(), s.cuda_stream)
+    slikl_grad_ex(pr, tn, workspace.data_ptr(), workspace.numel(), s.cuda_stream, opt)
     res = dict(out)
     res["workspace"] = workspace
     return res
 
 
-def grad_workload(wl, device="cuda", deterministic=False, stream=None):
+def key_range_bound_of(wl) -> int:
+    """Longest key range of a workload's batches (host data), for TND problems."""
+    if wl.cu_seqlens_k is None:
+        return 0
+    c = wl.cu_seqlens_k.tolist()
+    return max((c[i + 1] - c[i] for i in range(len(c) - 1)), default=0)
+
+
+def grad_workload(wl, device="cuda", deterministic=False, stream=None, dk_path="auto"):
     """Move a slikl_inputs.Workload to the device and run grad()."""
     dev = torch.device(device)
     t = {n: getattr(wl, n).to(dev) for n in ("q", "k", "w", "p", "idx")}
     cuq = wl.cu_seqlens_q.to(dev) if wl.cu_seqlens_q is not None else None
     cuk = wl.cu_seqlens_k.to(dev) if wl.cu_seqlens_k is not None else None
     return grad(t["q"], t["k"], t["w"], t["p"], t["idx"], wl.layout, wl.layout, cuq, cuk,
-                deterministic=deterministic, stream=stream)
+                deterministic=deterministic, stream=stream, dk_path=dk_path,
+                key_range_bound=key_range_bound_of(wl))

@@ -14,6 +14,7 @@ namespace {
 
 struct Derived {
     int64_t T1, T2;
+    KmShape km;
 };
 
 slikl_status validate(const slikl_problem *pr, Derived *out) {
@@ -45,6 +46,49 @@ slikl_status validate(const slikl_problem *pr, Derived *out) {
         return SLIKL_ERR_PARAM_INVALID;
     out->T1 = T1;
     out->T2 = T2;
+    out->km = KmShape{};
+    return SLIKL_OK;
+}
+
+// Longest key range the key-major path may assume: S2 for BSND keys; for TND keys the
+// caller's bound in problem->S2 (0 = none given).
+int64_t key_range_bound(const slikl_problem *pr) { return pr->S2 > 0 ? pr->S2 : 0; }
+
+// Whether the key-major dK path can run this problem: the tensor-core kernels (N1 <= 64), a
+// known key-range bound of at most 16384 keys, atomic mode.
+bool km_possible(const slikl_problem *pr) {
+    const int64_t s2 = key_range_bound(pr);
+    return pr->N1 <= 64 && pr->deterministic == 0 && s2 > 0 && s2 <= 16384;
+}
+
+// Picks the dK path. The key-major path does work in proportion to the (query row, 256-key
+// block) pairs that are named at all and the scatter path in proportion to the named slots;
+// with the key range at most 16x top-k the first is the cheaper on B200 (measured rates: a
+// key-major row of 256 keys costs about as much tensor time as 16 fp32 slot scatters).
+slikl_status choose_dk_path(const slikl_problem *pr, Derived *dv, int32_t path) {
+    if (path != SLIKL_DK_AUTO && path != SLIKL_DK_SCATTER && path != SLIKL_DK_KEYMAJOR)
+        return SLIKL_ERR_PARAM_INVALID;
+    const bool possible = km_possible(pr);
+    if (path == SLIKL_DK_KEYMAJOR && !possible) return SLIKL_ERR_PARAM_INVALID;
+    bool use = false;
+    if (possible) {
+        const int64_t s2m = (key_range_bound(pr) + 255) / 256 * 256;
+        const int rb = pr->N1 > 32 ? 16 : 8;
+        const double rec_bytes = (double)dv->T1 * (double)s2m * rb;
+        use = path == SLIKL_DK_KEYMAJOR ||
+              (path == SLIKL_DK_AUTO && key_range_bound(pr) <= 16 * pr->topk &&
+               rec_bytes <= 8.0 * (1ull << 30));
+        if (use) {
+            KmShape k{};
+            k.km = 1;
+            k.S2m = (int)s2m;
+            k.kbound = key_range_bound(pr);
+            k.rec_bytes = rb;
+            k.nkpw = (int)((s2m / 256 + 31) / 32);
+            k.units_max = (s2m / 256) * ((dv->T1 + 31) / 32 + pr->B);
+            dv->km = k;
+        }
+    }
     return SLIKL_OK;
 }
 
@@ -77,7 +121,7 @@ Params make_params(const slikl_problem *pr, const Derived &dv, const slikl_tenso
         P.idx = tn->sparse_indices; P.cu_q = tn->cu_seqlens_q; P.cu_k = tn->cu_seqlens_k;
         P.dq = tn->dq; P.dk = tn->dk; P.dw = tn->dw; P.y = tn->softmax_out;
     }
-    WsLayout L = make_layout(dv.T1, dv.T2, pr->topk, pr->D, pr->deterministic);
+    WsLayout L = make_layout(dv.T1, dv.T2, pr->topk, pr->D, pr->deterministic, dv.km, pr->B);
     char *base = static_cast<char *>(ws);
     P.status = reinterpret_cast<uint32_t *>(base + L.status);
     P.meta = reinterpret_cast<int32_t *>(base + L.meta);
@@ -94,6 +138,20 @@ Params make_params(const slikl_problem *pr, const Derived &dv, const slikl_tenso
     P.vals1 = reinterpret_cast<int32_t *>(base + L.vals1);
     P.hist = reinterpret_cast<int32_t *>(base + L.hist);
     P.row_ptr = reinterpret_cast<int32_t *>(base + L.row_ptr);
+    P.km = dv.km.km;
+    if (P.km) {
+        P.S2m = dv.km.S2m;
+        P.kbound = dv.km.kbound;
+        P.nkpw = dv.km.nkpw;
+        P.rec_bytes = dv.km.rec_bytes;
+        P.units_max = dv.km.units_max;
+        P.tok_pairs = reinterpret_cast<uint32_t *>(base + L.tok_pairs);
+        P.rec = base + L.rec;
+        P.units = reinterpret_cast<int4 *>(base + L.units);
+        P.unit_off = reinterpret_cast<int64_t *>(base + L.unit_off);
+        P.unit_prefix = reinterpret_cast<int64_t *>(base + L.unit_prefix);
+        P.km_range = reinterpret_cast<int32_t *>(base + L.km_range);
+    }
     return P;
 }
 
@@ -122,39 +180,60 @@ using namespace slikl;
 
 extern "C" {
 
-slikl_status slikl_grad_workspace_size(const slikl_problem *problem, size_t *workspace_bytes) {
+slikl_status slikl_grad_workspace_size_ex(const slikl_problem *problem,
+                                          const slikl_options *options, size_t *workspace_bytes) {
     if (!workspace_bytes) return SLIKL_ERR_INNER_NULLPTR;
     Derived dv;
     slikl_status st = validate(problem, &dv);
     if (st != SLIKL_OK) return st;
+    st = choose_dk_path(problem, &dv, options ? options->dk_path : SLIKL_DK_AUTO);
+    if (st != SLIKL_OK) return st;
     *workspace_bytes = make_layout(dv.T1, dv.T2, problem->topk, problem->D,
-                                   problem->deterministic).total;
+                                   problem->deterministic, dv.km, problem->B).total;
     return SLIKL_OK;
+}
+
+slikl_status slikl_grad_workspace_size(const slikl_problem *problem, size_t *workspace_bytes) {
+    return slikl_grad_workspace_size_ex(problem, nullptr, workspace_bytes);
 }
 
 slikl_status slikl_grad(const slikl_problem *problem, const slikl_tensors *tensors,
                         void *workspace, size_t workspace_bytes, void *stream) {
-    return slikl_grad_with_events(problem, tensors, workspace, workspace_bytes, stream, nullptr,
-                                  nullptr);
+    return slikl_grad_ex(problem, tensors, workspace, workspace_bytes, stream, nullptr);
 }
 
 slikl_status slikl_grad_with_events(const slikl_problem *problem, const slikl_tensors *tensors,
                                     void *workspace, size_t workspace_bytes, void *stream,
                                     void *fused_begin, void *fused_end) {
+    slikl_options o{};
+    o.dk_path = SLIKL_DK_AUTO;
+    o.fused_begin = fused_begin;
+    o.fused_end = fused_end;
+    return slikl_grad_ex(problem, tensors, workspace, workspace_bytes, stream, &o);
+}
+
+slikl_status slikl_grad_ex(const slikl_problem *problem, const slikl_tensors *tensors,
+                           void *workspace, size_t workspace_bytes, void *stream,
+                           const slikl_options *options) {
     Derived dv;
     slikl_status st = validate(problem, &dv);
+    if (st != SLIKL_OK) return st;
+    st = choose_dk_path(problem, &dv, options ? options->dk_path : SLIKL_DK_AUTO);
     if (st != SLIKL_OK) return st;
     st = check_tensors(problem, tensors, true);
     if (st != SLIKL_OK) return st;
     if (!workspace) return SLIKL_ERR_PARAM_NULLPTR;
     if (reinterpret_cast<uintptr_t>(workspace) & 255) return SLIKL_ERR_PARAM_INVALID;
-    WsLayout L = make_layout(dv.T1, dv.T2, problem->topk, problem->D, problem->deterministic);
+    WsLayout L = make_layout(dv.T1, dv.T2, problem->topk, problem->D, problem->deterministic,
+                             dv.km, problem->B);
     if (workspace_bytes < L.total) return SLIKL_ERR_WORKSPACE_TOO_SMALL;
     bool ok = false;
     int sms = current_sm_count(&ok);
     if (!ok) return SLIKL_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     Params P = make_params(problem, dv, tensors, workspace);
+    void *fused_begin = options ? options->fused_begin : nullptr;
+    void *fused_end = options ? options->fused_end : nullptr;
 
     const int workers = sms < kMaxWorkers ? sms : kMaxWorkers;
     if (cudaMemsetAsync(P.status, 0, 256, s) != cudaSuccess) return SLIKL_ERR_CUDA;
@@ -162,15 +241,18 @@ slikl_status slikl_grad_with_events(const slikl_problem *problem, const slikl_te
         cudaMemsetAsync(P.dk_acc, 0, sizeof(float) * (size_t)dv.T2 * problem->D, s) != cudaSuccess)
         return SLIKL_ERR_CUDA;
     if (launch_metadata(P, workers, 1, s) != cudaSuccess) return SLIKL_ERR_CUDA;
+    if (P.km && launch_km_metadata(P, workers, s) != cudaSuccess) return SLIKL_ERR_CUDA;
     if (fused_begin && cudaEventRecord(static_cast<cudaEvent_t>(fused_begin), s) != cudaSuccess)
         return SLIKL_ERR_CUDA;
     if (dv.T1 > 0) {
         bool handled = false;
         if (launch_fused_sm100(P, workers, s, &handled) != cudaSuccess) return SLIKL_ERR_CUDA;
         if (!handled && launch_fused_simt(P, workers, s) != cudaSuccess) return SLIKL_ERR_CUDA;
+        if (P.km && !handled) return SLIKL_ERR_CUDA;   // key-major records need the sm100 kernel
     }
     if (fused_end && cudaEventRecord(static_cast<cudaEvent_t>(fused_end), s) != cudaSuccess)
         return SLIKL_ERR_CUDA;
+    if (P.km && dv.T1 > 0 && launch_dk_keymajor(P, workers, s) != cudaSuccess) return SLIKL_ERR_CUDA;
     cudaError_t e = P.deterministic ? launch_deterministic_reduce(P, s) : launch_cast(P, s);
     return e == cudaSuccess ? SLIKL_OK : SLIKL_ERR_CUDA;
 }

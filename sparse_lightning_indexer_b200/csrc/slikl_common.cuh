@@ -41,12 +41,35 @@ struct Params {
     int32_t *keys0, *vals0, *keys1, *vals1;   // radix-sort buffers [T1*K]
     int32_t *hist;        // [256 * sort_blocks]
     int32_t *row_ptr;     // [T2 + 2]
+    // key-major dK path (km = 1): the fused kernel stores one record per named (token, key)
+    // and the key-major kernel forms dK block by block from them
+    int km;
+    int S2m;              // record row length in keys: longest key range rounded up to 256
+    int64_t kbound;       // the longest key range the caller promised
+    int nkpw;             // 32-bit words per token in tok_pairs
+    int rec_bytes;        // 8 (N1 <= 32) or 16 (N1 <= 64)
+    uint32_t *tok_pairs;  // [T1][nkpw] bit kp: the token names a key of [256 kp, 256 kp + 256)
+    void *rec;            // [T1][S2m] records {dI, ReLU(S) > 0 mask of the heads}
+    int4 *units;          // [units_max] {first token, first key row, local key | keys << 16,
+                          //              token mask}: 32 tokens x one 256-key block pair
+    int64_t *unit_off;    // [B + 1] first unit of each batch; unit_off[B] = unit count
+    int64_t *unit_prefix; // [units_max + 1] exclusive prefix of the unit costs
+    int32_t *km_range;    // [kMaxWorkers + 1] first unit of each worker of the key-major kernel
+    int64_t units_max;
+};
+
+// Shape of the key-major dK path of one call (km = 0: scatter path).
+struct KmShape {
+    int km;
+    int S2m, nkpw, rec_bytes;
+    int64_t units_max, kbound;
 };
 
 // Byte offsets of the workspace regions; every region starts 256-byte aligned.
 struct WsLayout {
     size_t status, meta, tok_kbase, tok_klen, tok_cost, tok_tiles, cost_prefix;
     size_t dk_acc, partials, keys0, vals0, keys1, vals1, hist, row_ptr;
+    size_t tok_pairs, rec, units, unit_off, unit_prefix, km_range;
     size_t total;
 };
 
@@ -54,7 +77,8 @@ constexpr int kSortTile = 4096;          // elements per block of one radix-sort
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-inline WsLayout make_layout(int64_t T1, int64_t T2, int64_t K, int64_t D, int det) {
+inline WsLayout make_layout(int64_t T1, int64_t T2, int64_t K, int64_t D, int det,
+                            const KmShape &km = KmShape{}, int64_t B = 0) {
     WsLayout L{};
     size_t off = 0;
     auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
@@ -75,6 +99,13 @@ inline WsLayout make_layout(int64_t T1, int64_t T2, int64_t K, int64_t D, int de
     L.vals1 = take(det ? sizeof(int32_t) * n : 0);
     L.hist = take(det ? sizeof(int32_t) * 256 * sort_blocks : 0);
     L.row_ptr = take(det ? sizeof(int32_t) * (size_t)(T2 + 2) : 0);
+    const bool k = km.km != 0;
+    L.tok_pairs = take(k ? sizeof(uint32_t) * (size_t)T1 * km.nkpw : 0);
+    L.rec = take(k ? (size_t)T1 * (size_t)km.S2m * km.rec_bytes : 0);
+    L.units = take(k ? 16 * (size_t)km.units_max : 0);
+    L.unit_off = take(k ? sizeof(int64_t) * (size_t)(B + 1) : 0);
+    L.unit_prefix = take(k ? sizeof(int64_t) * (size_t)(km.units_max + 1) : 0);
+    L.km_range = take(k ? sizeof(int32_t) * (kMaxWorkers + 1) : 0);
     L.total = off;
     return L;
 }
@@ -121,5 +152,7 @@ cudaError_t launch_fused_simt(const Params &P, int workers, cudaStream_t s);
 cudaError_t launch_fused_sm100(const Params &P, int workers, cudaStream_t s, bool *handled);
 cudaError_t launch_cast(const Params &P, cudaStream_t s);
 cudaError_t launch_deterministic_reduce(const Params &P, cudaStream_t s);
+cudaError_t launch_km_metadata(const Params &P, int workers, cudaStream_t s);
+cudaError_t launch_dk_keymajor(const Params &P, int workers, cudaStream_t s);
 
 }  // namespace slikl

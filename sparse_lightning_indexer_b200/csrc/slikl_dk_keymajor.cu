@@ -1,0 +1,400 @@
+// Key-major dK on the sm_100a tensor cores (tcgen05 MMA, accumulators in TMEM).
+//
+// The operator adds dK_topk(t) = dS_t^T . q_t into the key rows named by each query row t
+// (aclnnSparseLightningIndexerKLLossGrad, section "计算公式"). Grouped by key instead of by
+// query row, the same sum reads
+//
+//   dK_j = sum over the rows t that name key j of  sum_h dS_t[h, j] q_t[h, :]
+//
+// The fused kernel leaves one record per named (t, j): dI_tj and the set of heads with
+// S_tjh > 0. dS_tjh = dI_tj * w_th * [S_tjh > 0] is rebuilt from it here (the same fp32
+// product and rounding as the fused kernel's dS), and for one 256-key block pair the
+// products of all rows that name a key of the pair accumulate in TMEM:
+//
+//   dK^T [D x 256 keys] += q_t^T [D x heads] . dS_t [heads x 256 keys]   (M = 128, N = 256)
+//
+// so a key row takes one fp32 add per run of work units instead of one per naming slot.
+//
+// Work units are 32 query rows of one batch x one 256-key block pair (tables built by the
+// key-major metadata kernels). Each CTA takes a contiguous, cost-balanced range of units;
+// consecutive units on the same pair form a run that accumulates in one of two TMEM
+// buffers and is flushed once, with red.global.add.f32 of 32 consecutive d per warp
+// instruction, into the fp32 dK rows.
+//
+// Warp roles (512 threads):
+//   warp 0      producer: per query row, TMA of q_t (128-byte swizzle, zero heads past N1)
+//               and a bulk copy of the pair's 256 records (lane 0); w_t through registers
+//   warp 1      MMA issuer and TMEM owner
+//   warps 2-3   idle
+//   warps 4-7   flush: finished dK^T buffers from TMEM to the fp32 key rows
+//   warps 8-15  dS builders: one key of the pair per thread, written as a 128-byte K-major
+//               row (heads contiguous) with the 128-byte swizzle
+//
+// Every mbarrier wait is bounded; on expiry the CTA sets SLIKL_DEV_WAIT_TIMEOUT, the roles
+// stop, in-flight copies and MMAs are waited for (again bounded), TMEM is freed.
+#include <type_traits>
+
+#include "slikl_sm100.cuh"
+
+namespace slikl {
+namespace {
+
+using namespace sm100;
+
+constexpr int kKmThreads = 512;
+constexpr int kKmStages = 4;
+constexpr int kKmTmemCols = 512;         // two dK^T buffers of 256 columns
+
+struct KmBarriers {
+    uint64_t full[kKmStages];            // q, w, records landed (producer, TMA bytes)
+    uint64_t dsr[kKmStages];             // dS tile written (8 builder warps)
+    uint64_t empty[kKmStages];           // stage consumed by the MMA (tcgen05.commit)
+    uint64_t accf[2];                    // dK^T buffer complete (tcgen05.commit)
+    uint64_t acce[2];                    // dK^T buffer flushed (4 flush warps)
+    uint64_t drain;
+};
+
+struct KmPlan {
+    uint32_t q, ds, rec, w, bar, total;
+};
+
+__host__ __device__ constexpr uint32_t round_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
+
+template <int N1P, int RB>
+__host__ __device__ constexpr KmPlan km_plan() {
+    // [stage][2 column blocks][N1P heads][128 B] | [stage][256 keys][128 B] |
+    // [stage][256 records] | [stage][N1P] | barriers
+    return KmPlan{0u,
+                  kKmStages * N1P * 256u,
+                  kKmStages * N1P * 256u + kKmStages * 256u * 128u,
+                  kKmStages * N1P * 256u + kKmStages * 256u * 128u + kKmStages * 256u * RB,
+                  round_up(kKmStages * N1P * 256u + kKmStages * 256u * 128u +
+                               kKmStages * 256u * RB + kKmStages * N1P * 4u, 8),
+                  round_up(kKmStages * N1P * 256u + kKmStages * 256u * 128u +
+                               kKmStages * 256u * RB + kKmStages * N1P * 4u, 8) +
+                      (uint32_t)sizeof(KmBarriers) + 1024u};
+}
+
+struct KmItem {
+    int t;           // query row
+    int key0;        // first key row of the pair (identifies the run)
+    int kloc;        // first key of the pair within the batch's key range
+    int nkeys;       // keys of the pair inside the batch's key range
+    bool first;      // first row of a run
+    bool last;       // last row of a run
+};
+
+// The item sequence of a CTA: every set bit of every unit in [u0, u1), in order. Every role
+// walks it on its own.
+struct KmIter {
+    const int4 *U;
+    int u, u1;
+    int4 cu, nu;
+    uint32_t m;
+    bool has_nu;
+    int prev_key0;
+
+    __device__ void find_next(int from) {
+        has_nu = false;
+        for (int k = from; k < u1; ++k) {
+            const int4 x = U[k];
+            if (x.w) { nu = x; u = k; has_nu = true; return; }
+        }
+        u = u1;
+    }
+    __device__ void init(const int4 *units, int a, int b) {
+        U = units; u1 = b; prev_key0 = -1; m = 0;
+        find_next(a);
+        if (has_nu) {
+            cu = nu;
+            m = (uint32_t)cu.w;
+            find_next(u + 1);
+        }
+    }
+    __device__ bool next(KmItem &it) {
+        if (!m) return false;
+        const int bit = __ffs((int)m) - 1;
+        m &= m - 1;
+        it.t = cu.x + bit;
+        it.key0 = cu.y;
+        it.kloc = cu.z & 0xFFFF;
+        it.nkeys = (int)((uint32_t)cu.z >> 16);
+        it.first = cu.y != prev_key0;
+        prev_key0 = cu.y;
+        if (m == 0) {
+            if (has_nu) {
+                it.last = nu.y != cu.y;
+                cu = nu;
+                m = (uint32_t)cu.w;
+                find_next(u + 1);
+            } else {
+                it.last = true;
+            }
+        } else {
+            it.last = false;
+        }
+        return true;
+    }
+};
+
+template <typename T>
+__device__ __forceinline__ uint32_t pack2(float a, float b);
+template <>
+__device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float a, float b) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t *>(&v);
+}
+template <>
+__device__ __forceinline__ uint32_t pack2<__half>(float a, float b) {
+    const __half2 v = __floats2half2_rn(a, b);
+    return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+template <int N1P, int D, typename T>
+__global__ void __launch_bounds__(kKmThreads, 1)
+    dk_keymajor(Params P, const __grid_constant__ CUtensorMap qmap) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    constexpr int RB = N1P > 32 ? 16 : 8;
+    constexpr KmPlan SP = km_plan<N1P, RB>();
+    constexpr int kFmt = std::is_same<T, __nv_bfloat16>::value ? 1 : 0;
+    constexpr uint32_t kIdesc = idesc_f16(kFmt, 128, 256, 1, 0);
+    constexpr uint32_t kTx = (D / 64) * N1P * 128 + 256 * RB;   // q boxes + records
+    KmBarriers *bars = reinterpret_cast<KmBarriers *>(smem + SP.bar);
+    __shared__ volatile int abort_flag;
+    __shared__ uint32_t tmem_base;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int u0 = P.km_range[blockIdx.x], u1 = P.km_range[blockIdx.x + 1];
+
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        for (int s = 0; s < kKmStages; ++s) {
+            mbar_init(&bars->full[s], 1);
+            mbar_init(&bars->dsr[s], 8);
+            mbar_init(&bars->empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars->accf[b], 1);
+            mbar_init(&bars->acce[b], 4);
+        }
+        mbar_init(&bars->drain, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (D == 64) {
+        // the upper column block of every q stage stays zero (rows d >= 64 of q^T)
+        for (uint32_t i = threadIdx.x; i < kKmStages * N1P * 128 / 16; i += kKmThreads) {
+            const uint32_t st = i / (N1P * 8), r = i % (N1P * 8);
+            reinterpret_cast<uint4 *>(smem + SP.q + st * N1P * 256 + N1P * 128)[r] =
+                make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(&tmem_base)), "r"(kKmTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tacc = tmem_base;
+
+    KmIter iter;
+    iter.init(P.units, u0, u1);
+    KmItem it;
+
+    if (warp == 0) {
+        // =============================== producer ===============================
+        // w_t goes through registers (its rows need only 4-byte alignment), loaded one item
+        // ahead; q_t and the records by TMA / bulk copy, issued by lane 0
+        auto load_w = [&](int t, float *wv) {
+#pragma unroll
+            for (int k = 0; k < (N1P + 31) / 32; ++k) {
+                const int h = lane + 32 * k;
+                wv[k] = h < P.N1 ? P.w[(int64_t)t * P.N1 + h] : 0.f;
+            }
+        };
+        float wcur[(N1P + 31) / 32], wnxt[(N1P + 31) / 32];
+        uint32_t i = 0;
+        bool ok = true, have = iter.next(it);
+        if (have) load_w(it.t, wcur);
+        while (have) {
+            KmItem nx;
+            const bool have_nx = iter.next(nx);
+            if (have_nx) load_w(nx.t, wnxt);
+            const int s = i % kKmStages;
+            if (!wait_bar(&bars->empty[s], ((i / kKmStages) & 1) ^ 1, &abort_flag, P.status)) { ok = false; break; }
+            float *wd = reinterpret_cast<float *>(smem + SP.w + s * N1P * 4);
+#pragma unroll
+            for (int k = 0; k < (N1P + 31) / 32; ++k)
+                if (lane + 32 * k < N1P) wd[lane + 32 * k] = wcur[k];
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&bars->full[s], kTx);
+                const uint32_t qd = smem_u32(smem + SP.q + s * N1P * 256);
+                tma_load_3d(qd, &qmap, 0, 0, it.t, &bars->full[s]);
+                if (D == 128) tma_load_3d(qd + N1P * 128, &qmap, 64, 0, it.t, &bars->full[s]);
+                bulk_g2s(smem_u32(smem + SP.rec + s * 256 * RB),
+                         static_cast<const char *>(P.rec) + ((int64_t)it.t * P.S2m + it.kloc) * RB,
+                         256 * RB, &bars->full[s]);
+            }
+            __syncwarp();
+            ++i;
+            it = nx;
+            have = have_nx;
+#pragma unroll
+            for (int k = 0; k < (N1P + 31) / 32; ++k) wcur[k] = wnxt[k];
+        }
+        if (!ok && lane == 0) {
+            // wait (bounded) for the copies already issued before the CTA leaves
+            for (uint32_t j = i > kKmStages ? i - kKmStages : 0; j < i; ++j) {
+                const long long st = clock64();
+                while (!mbar_try_wait(&bars->full[j % kKmStages], (j / kKmStages) & 1) &&
+                       clock64() - st < kWaitCycles) {}
+            }
+        }
+    } else if (warp == 1) {
+        // =============================== MMA issuer ===============================
+        uint32_t i = 0, nrun = 0;
+        while (iter.next(it)) {
+            const int s = i % kKmStages;
+            const int ab = nrun & 1;
+            if (!wait_bar(&bars->dsr[s], (i / kKmStages) & 1, &abort_flag, P.status)) break;
+            if (it.first && !wait_bar(&bars->acce[ab], ((nrun >> 1) & 1) ^ 1, &abort_flag, P.status)) break;
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t qa = smem_u32(smem + SP.q + s * N1P * 256);
+                const uint32_t da = smem_u32(smem + SP.ds + s * 256 * 128);
+#pragma unroll
+                for (int ks = 0; ks < N1P / 16; ++ks) {
+                    const uint64_t a = sdesc(qa + ks * 2048, N1P * 128, 1024);   // q^T, MN-major
+                    const uint64_t b = sdesc(da + ks * 32, 16, 1024);            // dS, K-major
+                    umma_f16(tacc + ab * 256, a, b, kIdesc, (it.first && ks == 0) ? 0u : 1u);
+                }
+                umma_commit(&bars->empty[s]);
+                if (it.last) umma_commit(&bars->accf[ab]);
+            }
+            __syncwarp();
+            if (it.last) ++nrun;
+            ++i;
+        }
+        if (lane == 0) umma_commit(&bars->drain);
+        __syncwarp();
+        const long long st = clock64();
+        while (!mbar_try_wait(&bars->drain, 0) && clock64() - st < kWaitCycles) {}
+    } else if (warp >= 4 && warp < 8) {
+        // =============================== flush ===============================
+        const int quad = warp & 3;
+        const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+        uint32_t nrun = 0;
+        while (iter.next(it)) {
+            if (!it.last) continue;
+            const int ab = nrun & 1;
+            if (!wait_bar(&bars->accf[ab], (nrun >> 1) & 1, &abort_flag, P.status)) break;
+            tc_fence_after();
+            if (quad * 32 < D) {
+                float *dst = P.dk_acc + (int64_t)it.key0 * D + quad * 32 + lane;
+#pragma unroll 1
+                for (int c = 0; c < 256; c += 32) {
+                    if (c >= it.nkeys) break;
+                    float v[32];
+                    tmem_ld32(tacc + ab * 256 + lane_addr + c, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int k = 0; k < 32; ++k)
+                        if (c + k < it.nkeys) red_add_f32(dst + (int64_t)(c + k) * D, v[k]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->acce[ab]);
+            ++nrun;
+        }
+    } else if (warp >= 8) {
+        // =============================== dS builders ===============================
+        const int e = threadIdx.x - 256;          // key of the pair, 0..255
+        uint32_t i = 0;
+        while (iter.next(it)) {
+            const int s = i % kKmStages;
+            if (!wait_bar(&bars->full[s], (i / kKmStages) & 1, &abort_flag, P.status)) break;
+            uint32_t m0, m1 = 0;
+            float dI;
+            const uint8_t *rp = smem + SP.rec + s * 256 * RB + e * RB;
+            if (RB == 16) {
+                const uint4 r = *reinterpret_cast<const uint4 *>(rp);
+                m0 = r.x; m1 = r.y; dI = __uint_as_float(r.z);
+            } else {
+                const uint2 r = *reinterpret_cast<const uint2 *>(rp);
+                m0 = r.x; dI = __uint_as_float(r.y);
+            }
+            const float *ws = reinterpret_cast<const float *>(smem + SP.w + s * N1P * 4);
+            uint8_t *row = smem + SP.ds + s * 256 * 128 + e * 128;
+#pragma unroll
+            for (int c = 0; c < N1P / 8; ++c) {       // 8 heads = one 16-byte chunk
+                const float4 wa = *reinterpret_cast<const float4 *>(ws + 8 * c);
+                const float4 wb = *reinterpret_cast<const float4 *>(ws + 8 * c + 4);
+                const uint32_t mb = ((c < 4 ? m0 : m1) >> ((c & 3) * 8)) & 0xFFu;
+                const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+                float d[8];
+#pragma unroll
+                for (int h = 0; h < 8; ++h) d[h] = ((mb >> h) & 1u) ? dI * wv[h] : 0.f;
+                const uint4 o = make_uint4(pack2<T>(d[0], d[1]), pack2<T>(d[2], d[3]),
+                                           pack2<T>(d[4], d[5]), pack2<T>(d[6], d[7]));
+                *reinterpret_cast<uint4 *>(row + (((c ^ e) & 7) << 4)) = o;
+            }
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->dsr[s]);
+            ++i;
+        }
+    }
+
+    // ---------------- teardown ----------------
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tacc),
+                     "r"(kKmTmemCols));
+    }
+}
+
+template <int N1P, int D, typename T>
+cudaError_t launch_km_t(const Params &P, int workers, cudaStream_t s) {
+    constexpr int RB = N1P > 32 ? 16 : 8;
+    constexpr KmPlan sp = km_plan<N1P, RB>();
+    static_assert(sp.total <= 227 * 1024, "key-major kernel shared memory");
+    CUtensorMap qmap;
+    cudaError_t e = encode_q_map<N1P, T>(P, &qmap);
+    if (e != cudaSuccess) return e;
+    auto k = dk_keymajor<N1P, D, T>;
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp.total);
+    if (e != cudaSuccess) return e;
+    k<<<workers, kKmThreads, sp.total, s>>>(P, qmap);
+    return cudaGetLastError();
+}
+
+template <int N1P, int D>
+cudaError_t launch_km_d(const Params &P, int workers, cudaStream_t s) {
+    return P.dtype == SLIKL_BF16 ? launch_km_t<N1P, D, __nv_bfloat16>(P, workers, s)
+                                 : launch_km_t<N1P, D, __half>(P, workers, s);
+}
+
+template <int N1P>
+cudaError_t launch_km_n(const Params &P, int workers, cudaStream_t s) {
+    return P.D == 128 ? launch_km_d<N1P, 128>(P, workers, s) : launch_km_d<N1P, 64>(P, workers, s);
+}
+
+}  // namespace
+
+// Shapes: N1 <= 64, D in {64, 128}.
+cudaError_t launch_dk_keymajor(const Params &P, int workers, cudaStream_t s) {
+    if (P.N1 > 64 || (P.D != 64 && P.D != 128)) return cudaErrorInvalidValue;
+    if (P.N1 <= 16) return launch_km_n<16>(P, workers, s);
+    if (P.N1 <= 32) return launch_km_n<32>(P, workers, s);
+    return launch_km_n<64>(P, workers, s);
+}
+
+}  // namespace slikl

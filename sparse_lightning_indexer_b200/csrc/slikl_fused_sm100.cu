@@ -36,132 +36,16 @@
 // is freed and the kernel returns.
 #include <type_traits>
 
-#include "slikl_common.cuh"
+#include "slikl_sm100.cuh"
 
 namespace slikl {
 namespace {
 
+using namespace sm100;
+
 constexpr int kThreads = 384;
-constexpr long long kWaitCycles = 1ll << 31;
 constexpr int kTmemCols = 512;
 constexpr int kStageBytes = 128 * 256;      // 128 key rows x 128 d (two 64-d column blocks)
-
-// ------------------------------------------------------------------------------------------
-// PTX wrappers
-// ------------------------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ void fence_proxy_async() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-                 "r"(src_bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                         uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-__device__ __forceinline__ void umma_commit(uint64_t *bar) {
-    asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-        ::"r"(smem_u32(bar))
-        : "memory");
-}
-__device__ __forceinline__ void tmem_wait_ld() {
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-// 32 lanes x 32 bit, 16 / 32 consecutive columns per thread
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *v) {
-    uint32_t r[16];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float *v) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
-        ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])),
-          "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])),
-          "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
-          "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
-          "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
-          "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15]))
-        : "memory");
-}
-__device__ __forceinline__ void tmem_wait_st() {
-    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
-    tmem_ld16(taddr, v);
-    tmem_ld16(taddr + 16, v + 16);
-}
-
-// Shared-memory matrix descriptor (sm_100): start >> 4 in [0,14), leading byte offset >> 4
-// in [16,30), stride byte offset >> 4 in [32,46), version 1 at bit 46, 128-byte swizzle
-// (value 2) in [61,64).
-__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
-}
-// Instruction descriptor, kind::f16 with fp32 accumulate: D format bit 4, A/B format at
-// bits 7 / 10 (0 = f16, 1 = bf16), A / B MN-major at bits 15 / 16, N >> 3 at 17, M >> 4 at 24.
-__host__ __device__ constexpr uint32_t idesc_f16(int fmt, int m, int n, int a_mn, int b_mn) {
-    return (1u << 4) | ((uint32_t)fmt << 7) | ((uint32_t)fmt << 10) | ((uint32_t)a_mn << 15) |
-           ((uint32_t)b_mn << 16) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
-}
-
-// Byte offset of element (row, col) of a tile of 128-byte rows (64 bf16 per row) in 8-row
-// atoms with the 128-byte swizzle (16-byte chunk index XOR row % 8).
-__device__ __forceinline__ uint32_t sw128(int row, int col_elem) {
-    return (uint32_t)(row * 128 + ((((col_elem >> 3) ^ row) & 7) << 4) + (col_elem & 7) * 2);
-}
 
 struct Barriers {
     uint64_t kv_full[4], kv_empty[4];     // K stages: producers -> MMA -> producers
@@ -211,44 +95,6 @@ struct Ctl {
     uint32_t tmem_base;
     float stat_m[4], stat_z[4];
 };
-
-__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Ctl *ctl,
-                                         uint32_t *status) {
-    if (mbar_try_wait(bar, parity)) return true;
-    long long start = clock64();
-    while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (ctl->abort) return false;
-        if (clock64() - start > kWaitCycles) {
-            ctl->abort = 1;
-            set_status(status, SLIKL_DEV_WAIT_TIMEOUT);
-            return false;
-        }
-    }
-}
-
-// Reusable barrier over a fixed set of warps (lane 0 of each arrives); bounded like wait_bar,
-// so a CTA that aborts never strands warps at a hardware barrier.
-__device__ __forceinline__ bool group_sync(uint64_t *bar, uint32_t &phase, Ctl *ctl,
-                                           uint32_t *status) {
-    __syncwarp();
-    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
-    const bool ok = wait_bar(bar, phase & 1, ctl, status);
-    ++phase;
-    return ok;
-}
-
-template <typename T>
-__device__ __forceinline__ uint16_t to_bits16(float v);
-template <>
-__device__ __forceinline__ uint16_t to_bits16<__nv_bfloat16>(float v) {
-    return __bfloat16_as_ushort(__float2bfloat16_rn(v));
-}
-template <>
-__device__ __forceinline__ uint16_t to_bits16<__half>(float v) {
-    return __half_as_ushort(__float2half_rn(v));
-}
-
 
 // ------------------------------------------------------------------------------------------
 // Item schedule shared by every role
@@ -336,8 +182,9 @@ struct Sched {
 // ------------------------------------------------------------------------------------------
 // The kernel
 // ------------------------------------------------------------------------------------------
-template <int N1P, int D, typename T>
-__global__ void __launch_bounds__(kThreads, 1) fused_sm100(Params P, int stages) {
+template <int N1P, int D, typename T, bool kRec>
+__global__ void __launch_bounds__(kThreads, 1)
+    fused_sm100(Params P, int stages, const __grid_constant__ CUtensorMap qmap) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -351,6 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_sm100(Params P, int stages)
     constexpr uint32_t kIdescDk = idesc_f16(kFmt, 128, 128, 1, 1);
     constexpr int kDChunks = D / 8;          // 16-byte chunks per key row
     constexpr int kC = N1P < 32 ? N1P : 32;  // S columns per TMEM load
+    constexpr int kRecBytes = N1P > 32 ? 16 : 8;  // record: ReLU mask word(s), dI
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t0 = P.meta[kMetaHeader + 2 * blockIdx.x];
@@ -364,14 +212,14 @@ __global__ void __launch_bounds__(kThreads, 1) fused_sm100(Params P, int stages)
             mbar_init(&bars->kv_empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&bars->q_full[b], 32);
+            mbar_init(&bars->q_full[b], 1);      // producer 0 (expect_tx) + TMA bytes
             mbar_init(&bars->q_empty[b], 1);
             mbar_init(&bars->s_full[b], 1);
             mbar_init(&bars->s_empty[b], 4);
             mbar_init(&bars->ds_full[b], 4);
             mbar_init(&bars->rows_full[b], 4);
             mbar_init(&bars->dk_full[b], 1);
-            mbar_init(&bars->dk_empty[b], 4);
+            mbar_init(&bars->dk_empty[b], kRec ? 1 : 4);
         }
         mbar_init(&bars->dq_full, 1);
         mbar_init(&bars->dq_empty, 4);
@@ -414,9 +262,11 @@ __global__ void __launch_bounds__(kThreads, 1) fused_sm100(Params P, int stages)
         // that skipped items could be fooled by the phase parity of a reused stage); each warp
         // copies its own third of the tile's row groups. Every lane ends an item with
         // cp.async.mbarrier.arrive.noinc, so a stage turns full (96 arrivals) when all of its
-        // copies have landed, without any producer waiting for them. The slot indices, key
-        // base and key count of item g + 2 travel with item g's copies into a 4-slot ring in
-        // shared memory; item g reads them after the full barrier of item g - 2.
+        // copies have landed, without any producer waiting for them (that arrival also waits
+        // for every earlier cp.async of the thread, so nothing else is copied with cp.async).
+        // The slot indices, key base and key count of an item are loaded into registers four
+        // items ahead and stored into a 4-slot ring in shared memory two items ahead; warp 0
+        // also loads q by TMA.
         const int rsub = lane / kDChunks;                 // row within a group of rows
         const int chunk = lane % kDChunks;
         constexpr int kRowsPerPass = 32 / kDChunks;       // 2 (D=128) or 4 (D=64)
@@ -427,78 +277,97 @@ __global__ void __launch_bounds__(kThreads, 1) fused_sm100(Params P, int stages)
             asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
                          : "memory");
         };
-        // 4-byte copies (zero-filled past the end of the token's slots): lane l copies slots
-        // l, l+32, l+64, l+96; lane 0 also the key base and key count
-        auto fetch_idx = [&](const Item &it, int slot) {
-            int32_t *dst = ring + slot * kRingSlot;
+        struct IdxRegs { int32_t v[4]; int32_t kb, kl; };
+        // lane l loads slots l, l+32, l+64, l+96 of the item's tile (-1 past the token's end)
+        auto ldg_idx = [&](const Item &it, IdxRegs &r) {
             const int32_t *irow = P.idx + (int64_t)it.t * K;
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int j = it.tile * 128 + lane + 32 * u;
-                const bool in = j < K;
-                asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;"
-                             ::"r"(smem_u32(dst + lane + 32 * u)), "l"(in ? irow + j : irow), "r"(in ? 4 : 0)
-                             : "memory");
+                r.v[u] = j < K ? irow[j] : -1;
             }
-            if (lane == 0) {
-                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst + 128)),
-                             "l"(P.tok_kbase + it.t) : "memory");
-                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst + 129)),
-                             "l"(P.tok_klen + it.t) : "memory");
-            }
+            r.kb = P.tok_kbase[it.t];
+            r.kl = P.tok_klen[it.t];
+        };
+        auto sts_idx = [&](const IdxRegs &r, int slot) {
+            int32_t *d = ring + slot * kRingSlot;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) d[lane + 32 * u] = r.v[u];
+            if (lane == 0) { d[128] = r.kb; d[129] = r.kl; }
         };
         Item it0 = sc.next();
         Item it1 = it0.kind >= 0 ? sc.next() : it0;
         Item it2 = it1.kind >= 0 ? sc.next() : it1;
-        if (it0.kind >= 0) fetch_idx(it0, 0);
-        if (it1.kind >= 0) fetch_idx(it1, 1);
-        cp_async_commit();
-        cp_async_wait<0>();
-        __syncwarp();
+        Item it3 = it2.kind >= 0 ? sc.next() : it2;
+        IdxRegs r2{}, r3{};
+        if (it0.kind >= 0) { IdxRegs r; ldg_idx(it0, r); sts_idx(r, 0); }
+        if (it1.kind >= 0) { IdxRegs r; ldg_idx(it1, r); sts_idx(r, 1); }
+        if (it2.kind >= 0) ldg_idx(it2, r2);
+        if (it3.kind >= 0) ldg_idx(it3, r3);
+        int q_last = -1;                                  // ordinal of the last q load issued
         uint32_t g = 0;
         while (ok && it0.kind >= 0) {
+            __syncwarp();                                 // ring stores of earlier items
             if (warp == 0 && it0.kind == 0 && it0.first) {
-                // q tile of a new token (rows h < N1) into q buffer ord % 2
+                // q tile of a new token (heads past N1 read as zero) into q buffer ord % 2
                 const int qb = it0.ord & 1;
-                if (!wait_bar(&bars->q_empty[qb], ((it0.ord >> 1) & 1) ^ 1, &ctl, P.status)) { ok = false; break; }
-                const char *qsrc = static_cast<const char *>(P.q) + (int64_t)it0.t * P.N1 * D * 2;
-                const uint32_t qdst = smem_u32(smem + SP.q + qb * N1P * 256);
-                for (int h = rsub; h < P.N1; h += kRowsPerPass) {
-                    const int cb = chunk >> 3;
-                    cp_async16(qdst + cb * (N1P * 128) + sw128(h, (chunk & 7) * 8),
-                               qsrc + (int64_t)h * D * 2 + chunk * 16, 16);
+                if (!wait_bar(&bars->q_empty[qb], ((it0.ord >> 1) & 1) ^ 1, &ctl.abort, P.status)) { ok = false; break; }
+                if (lane == 0) {
+                    const uint32_t qdst = smem_u32(smem + SP.q + qb * N1P * 256);
+                    mbar_arrive_expect_tx(&bars->q_full[qb], (D / 64) * N1P * 128);
+                    tma_load_3d(qdst, &qmap, 0, 0, it0.t, &bars->q_full[qb]);
+                    if (D == 128) tma_load_3d(qdst + N1P * 128, &qmap, 64, 0, it0.t, &bars->q_full[qb]);
                 }
-                arrive_on_copies(&bars->q_full[qb]);
-            }
-            // the ring slot of item g travelled with item g - 2
-            if (g >= 2) {
-                const uint32_t gp = g - 2;
-                if (!wait_bar(&bars->kv_full[gp % stages], (gp / stages) & 1, &ctl, P.status)) { ok = false; break; }
+                q_last = it0.ord;
             }
             const int s = g % stages;
-            if (!wait_bar(&bars->kv_empty[s], ((g / stages) & 1) ^ 1, &ctl, P.status)) { ok = false; break; }
+            if (!wait_bar(&bars->kv_empty[s], ((g / stages) & 1) ^ 1, &ctl.abort, P.status)) { ok = false; break; }
             const int32_t *slot = ring + (g & 3) * kRingSlot;
             const int32_t kb = slot[128], kl = slot[129];
             const int jbase = it0.tile * 128;
             const uint32_t dst = smem_u32(smem + SP.kv + s * kStageBytes) + (chunk >> 3) * 16384;
-            // this warp's row groups i = warp, warp + 3, ... (a compact loop: the instruction
-            // cache of a sub-partition is shared with two other warp roles)
-#pragma unroll 2
-            for (int i = warp; i < 128 / kRowsPerPass; i += 3) {
-                const int r = rsub + kRowsPerPass * i;
-                const int32_t v = slot[r];
-                const bool valid = jbase + r < K && v >= 0 && v < kl;
-                const char *src = kbase_ptr + (valid ? ((int64_t)(kb + v) * (D * 2) + chunk * 16) : 0);
-                cp_async16(dst + sw128(r, (chunk & 7) * 8), src, valid ? 16 : 0);
+            // this warp's row groups i = warp, warp + 3, ...: all slot indices into registers
+            // first, then the copies back to back (a shared-memory load issued after a copy
+            // waits behind it in the memory pipeline)
+            constexpr int kGroups = 128 / kRowsPerPass;       // 64 (D=128) or 32 (D=64)
+            constexpr int kPer = (kGroups + 2) / 3;
+            int32_t vv[kPer];
+#pragma unroll
+            for (int j = 0; j < kPer; ++j) {
+                const int i = warp + 3 * j;
+                vv[j] = i < kGroups ? slot[rsub + kRowsPerPass * i] : -1;
             }
-            if (it2.kind >= 0) fetch_idx(it2, (g + 2) & 3);
+#pragma unroll
+            for (int j = 0; j < kPer; ++j) {
+                const int i = warp + 3 * j;
+                if (i < kGroups) {
+                    const int r = rsub + kRowsPerPass * i;
+                    const int32_t v = vv[j];
+                    const bool valid = jbase + r < K && v >= 0 && v < kl;
+                    const char *src = kbase_ptr + (valid ? ((int64_t)(kb + v) * (D * 2) + chunk * 16) : 0);
+                    cp_async16(dst + sw128(r, (chunk & 7) * 8), src, valid ? 16 : 0);
+                }
+            }
             arrive_on_copies(&bars->kv_full[s]);
+            // ring slot of item g + 2 from the loads issued two items ago; loads of item g + 4
+            if (it2.kind >= 0) sts_idx(r2, (g + 2) & 3);
             it0 = it1;
             it1 = it2;
-            if (it2.kind >= 0) it2 = sc.next();
+            it2 = it3;
+            r2 = r3;
+            if (it3.kind >= 0) {
+                it3 = sc.next();
+                if (it3.kind >= 0) ldg_idx(it3, r3);
+            }
             ++g;
         }
         cp_async_wait<0>();
+        if (!ok && q_last >= 0 && lane == 0) {
+            // the CTA stops: wait (bounded) for the last q load before the buffer goes away
+            const long long st = clock64();
+            while (!mbar_try_wait(&bars->q_full[q_last & 1], (q_last >> 1) & 1) &&
+                   clock64() - st < kWaitCycles) {}
+        }
     } else if (warp == 3) {
         // =============================== MMA issuer ===============================
         uint32_t gk = 0, gd = 0, nb = 0;       // items, pass-B items, finished B tokens
@@ -511,9 +380,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_sm100(Params P, int stages)
             const int s = gk % stages, b = gk & 1;
             const int qb = it.ord & 1;
             if (it.kind == 0 && it.first &&
-                !wait_bar(&bars->q_full[qb], (it.ord >> 1) & 1, &ctl, P.status)) return false;
-            if (!wait_bar(&bars->kv_full[s], (gk / stages) & 1, &ctl, P.status)) return false;
-            if (!wait_bar(&bars->s_empty[b], ((gk >> 1) & 1) ^ 1, &ctl, P.status)) return false;
+                !wait_bar(&bars->q_full[qb], (it.ord >> 1) & 1, &ctl.abort, P.status)) return false;
+            if (!wait_bar(&bars->kv_full[s], (gk / stages) & 1, &ctl.abort, P.status)) return false;
+            if (!wait_bar(&bars->s_empty[b], ((gk >> 1) & 1) ^ 1, &ctl.abort, P.status)) return false;
             tc_fence_after();
             if (lane == 0) {
                 const uint32_t kaddr = kv0 + s * kStageBytes;
@@ -541,9 +410,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_sm100(Params P, int stages)
             if (nxt.kind >= 0 && !issue_s(nxt, st_nxt)) { ok = false; break; }
             if (cur.kind == 1) {
                 const int b = gd & 1;
-                if (cur.first && !wait_bar(&bars->dq_empty, (nb & 1) ^ 1, &ctl, P.status)) { ok = false; break; }
-                if (!wait_bar(&bars->ds_full[b], (gd >> 1) & 1, &ctl, P.status)) { ok = false; break; }
-                if (!wait_bar(&bars->dk_empty[b], ((gd >> 1) & 1) ^ 1, &ctl, P.status)) { ok = false; break; }
+                if (cur.first && !wait_bar(&bars->dq_empty, (nb & 1) ^ 1, &ctl.abort, P.status)) { ok = false; break; }
+                if (!wait_bar(&bars->ds_full[b], (gd >> 1) & 1, &ctl.abort, P.status)) { ok = false; break; }
+                if (!kRec && !wait_bar(&bars->dk_empty[b], ((gd >> 1) & 1) ^ 1, &ctl.abort, P.status)) { ok = false; break; }
                 tc_fence_after();
                 if (lane == 0) {
                     const uint32_t kaddr = kv0 + st_cur * kStageBytes;
@@ -556,13 +425,17 @@ __global__ void __launch_bounds__(kThreads, 1) fused_sm100(Params P, int stages)
                         umma_f16(tm_dq, a, bd, kIdescDq, (!cur.first || ks > 0) ? 1u : 0u);
                     }
                     umma_commit(&bars->kv_empty[st_cur]);
+                    if constexpr (kRec) {
+                        umma_commit(&bars->dk_empty[b]);     // dS tile b read by the dq product
+                    } else {
 #pragma unroll
-                    for (int ks = 0; ks < N1P / 16; ++ks) {  // N1P heads, 16 per step
-                        const uint64_t a = sdesc(qaddr + ks * 2048, N1P * 128, 1024);
-                        const uint64_t bd = sdesc(dsaddr + ks * 2048, N1P * 128, 1024);
-                        umma_f16(tm_dk + b * 128, a, bd, kIdescDk, ks > 0);
+                        for (int ks = 0; ks < N1P / 16; ++ks) {  // N1P heads, 16 per step
+                            const uint64_t a = sdesc(qaddr + ks * 2048, N1P * 128, 1024);
+                            const uint64_t bd = sdesc(dsaddr + ks * 2048, N1P * 128, 1024);
+                            umma_f16(tm_dk + b * 128, a, bd, kIdescDk, ks > 0);
+                        }
+                        umma_commit(&bars->dk_full[b]);
                     }
-                    umma_commit(&bars->dk_full[b]);
                     if (cur.last) {
                         umma_commit(&bars->dq_full);
                         umma_commit(&bars->q_empty[cur.ord & 1]);
@@ -584,6 +457,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_sm100(Params P, int stages)
         }
     } else if (warp < 8) {
         // =============================== scatter group ===============================
+        // (idle when dK is formed key-major from records)
+        if constexpr (!kRec) {
         const int quad = warp & 3;
         const int d = quad * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
@@ -594,8 +469,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_sm100(Params P, int stages)
             if (it.kind < 0) break;
             if (it.kind != 1) continue;
             const int b = gd & 1;
-            if (!wait_bar(&bars->rows_full[b], (gd >> 1) & 1, &ctl, P.status)) { ok = false; break; }
-            if (!wait_bar(&bars->dk_full[b], (gd >> 1) & 1, &ctl, P.status)) { ok = false; break; }
+            if (!wait_bar(&bars->rows_full[b], (gd >> 1) & 1, &ctl.abort, P.status)) { ok = false; break; }
+            if (!wait_bar(&bars->dk_full[b], (gd >> 1) & 1, &ctl.abort, P.status)) { ok = false; break; }
             tc_fence_after();
             if (quad * 32 < D) {
                 // 4 chunks of 32 keys, one compact loop body (the instruction cache of a
@@ -629,6 +504,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_sm100(Params P, int stages)
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->dk_empty[b]);
             ++gd;
+        }
         }
     } else {
         // =============================== softmax group ===============================
@@ -691,19 +567,35 @@ __global__ void __launch_bounds__(kThreads, 1) fused_sm100(Params P, int stages)
                     // w of the new token into its buffer (the token two ordinals back is done)
                     for (int h = et; h < N1P; h += 128)
                         wsm[(it.ord & 1) * N1P + h] = h < P.N1 ? P.w[(int64_t)it.t * P.N1 + h] : 0.f;
-                    if (!group_sync(&bars->sm_sync, ph, &ctl, P.status)) { ok = false; break; }
+                    if constexpr (kRec) {
+                        // zero the records of every 256-key block pair the token names; pass B
+                        // then adds the named keys (the group syncs that end pass A order
+                        // these stores before those)
+                        const uint32_t *pw = P.tok_pairs + (int64_t)it.t * P.nkpw;
+                        for (int wd = 0; wd < P.nkpw; ++wd) {
+                            uint32_t bits = pw[wd];
+                            while (bits) {
+                                const int kp = wd * 32 + __ffs(bits) - 1;
+                                bits &= bits - 1;
+                                uint4 *dst = reinterpret_cast<uint4 *>(
+                                    static_cast<char *>(P.rec) + ((int64_t)it.t * P.S2m + 256 * kp) * kRecBytes);
+                                for (int i = et; i < 256 * kRecBytes / 16; i += 128) dst[i] = make_uint4(0, 0, 0, 0);
+                            }
+                        }
+                    }
+                    if (!group_sync(&bars->sm_sync, ph, &ctl.abort, P.status)) { ok = false; break; }
                     m_a = -INFINITY;
                     z_a = 0.f;
                 }
                 const int32_t v = cur.v;
                 const bool valid = v >= 0 && v < kl;
                 if (v != -1 && !valid) set_status(P.status, SLIKL_DEV_INDEX_OUT_OF_RANGE);
-                if (!wait_bar(&bars->s_full[sb], (gk >> 1) & 1, &ctl, P.status)) { ok = false; break; }
+                if (!wait_bar(&bars->s_full[sb], (gk >> 1) & 1, &ctl.abort, P.status)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t sa = tm_s + sb * N1P + lane_addr;
                 float sv[32];
                 float I = 0.f;
-#pragma unroll
+#pragma unroll 1
                 for (int c = 0; c < N1P; c += kC) {
                     if (kC == 32) tmem_ld32(sa + c, sv); else tmem_ld16(sa + c, sv);
                     float wv[32];
@@ -735,7 +627,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_sm100(Params P, int stages)
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) mw = fmaxf(mw, __shfl_xor_sync(0xffffffffu, mw, o));
                     if (lane == 0) ctl.stat_m[ew] = mw;
-                    if (!group_sync(&bars->sm_sync, ph, &ctl, P.status)) { ok = false; break; }
+                    if (!group_sync(&bars->sm_sync, ph, &ctl.abort, P.status)) { ok = false; break; }
                     float M = -INFINITY;
 #pragma unroll
                     for (int i = 0; i < 4; ++i) M = fmaxf(M, ctl.stat_m[i]);
@@ -743,7 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_sm100(Params P, int stages)
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) zw += __shfl_xor_sync(0xffffffffu, zw, o);
                     if (lane == 0) ctl.stat_z[ew] = zw;
-                    if (!group_sync(&bars->sm_sync, ph, &ctl, P.status)) { ok = false; break; }
+                    if (!group_sync(&bars->sm_sync, ph, &ctl.abort, P.status)) { ok = false; break; }
                     float Z = 0.f;
 #pragma unroll
                     for (int i = 0; i < 4; ++i) Z += ctl.stat_z[i];
@@ -767,13 +659,14 @@ __global__ void __launch_bounds__(kThreads, 1) fused_sm100(Params P, int stages)
                     dI = valid ? y - cur.p : 0.f;
                 }
                 // dS tile / key rows of buffer b free once the scatter of its previous use ended
-                if (!wait_bar(&bars->dk_empty[b], ((gd >> 1) & 1) ^ 1, &ctl, P.status)) { ok = false; break; }
-                if (!wait_bar(&bars->s_full[sb], (gk >> 1) & 1, &ctl, P.status)) { ok = false; break; }
+                if (!wait_bar(&bars->dk_empty[b], ((gd >> 1) & 1) ^ 1, &ctl.abort, P.status)) { ok = false; break; }
+                if (!wait_bar(&bars->s_full[sb], (gk >> 1) & 1, &ctl.abort, P.status)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t sa = tm_s + sb * N1P + lane_addr;
                 const uint32_t dwa = tm_dw + lane_addr;
                 uint8_t *dsb = ds_tiles + b * N1P * 256 + (lrow >> 6) * (N1P * 128);
                 const int jj = lrow & 63;
+                uint64_t smask = 0;                 // heads with S > 0 (record mode)
                 // 16 heads at a time: dS to smem; this slot's dW partial sums stay in TMEM
 #pragma unroll 1
                 for (int c = 0; c < N1P; c += 16) {
@@ -787,26 +680,43 @@ __global__ void __launch_bounds__(kThreads, 1) fused_sm100(Params P, int stages)
                     }
                     tmem_wait_ld();
                     uint8_t *dsc = dsb + c * 128;
+                    uint32_t m16 = 0;
 #pragma unroll
                     for (int h = 0; h < 16; ++h) {
                         const float sval = sv[h];
                         const float a0 = it.first ? 0.f : acc[h];
                         acc[h] = fmaf(dI, fmaxf(sval, 0.f), a0);
                         const float dsv = sval > 0.f ? dI * wv[h] : 0.f;
+                        if (kRec) m16 |= (sval > 0.f ? 1u : 0u) << h;
                         *reinterpret_cast<uint16_t *>(dsc + sw128(h, jj)) = to_bits16<T>(dsv);
                     }
+                    if (kRec) smask |= (uint64_t)m16 << c;
                     tmem_st16(dwa + c, acc);
                 }
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars->s_empty[sb]);
-                rows_s[b * kRowsStride + lrow] = valid ? cur.kb + v : -1;
+                if (!kRec) rows_s[b * kRowsStride + lrow] = valid ? cur.kb + v : -1;
                 fence_proxy_async();
                 __syncwarp();
                 if (lane == 0) {
                     mbar_arrive(&bars->ds_full[b]);
-                    mbar_arrive(&bars->rows_full[b]);
+                    if (!kRec) mbar_arrive(&bars->rows_full[b]);
+                }
+                if constexpr (kRec) {
+                    // record of this (token, key): the mask words are the same for every slot
+                    // naming the key; dI is added, so repeated slots of a key sum their dI
+                    if (valid && v < P.S2m) {
+                        char *rp = static_cast<char *>(P.rec) + ((int64_t)it.t * P.S2m + v) * kRecBytes;
+                        if (kRecBytes == 16) {
+                            *reinterpret_cast<uint2 *>(rp) = make_uint2((uint32_t)smask, (uint32_t)(smask >> 32));
+                            red_add_f32(reinterpret_cast<float *>(rp + 8), dI);
+                        } else {
+                            *reinterpret_cast<uint32_t *>(rp) = (uint32_t)smask;
+                            red_add_f32(reinterpret_cast<float *>(rp + 4), dI);
+                        }
+                    }
                 }
                 if (j < K) P.y[row_off + j] = y;
                 if (nx.kind >= 0) prefetch(nx, it, nxt);
@@ -819,8 +729,6 @@ __global__ void __launch_bounds__(kThreads, 1) fused_sm100(Params P, int stages)
                         if ((mask >> tl) & 1) continue;
                         for (int jz = tl * 128 + et; jz < (tl + 1) * 128 && jz < K; jz += 128) P.y[row_off + jz] = 0.f;
                     }
-                    // dW: this slot's partial sums from TMEM; butterfly reduce-scatter within each
-                    // warp, then the 4 warps in order
                     constexpr int kV = N1P < 32 ? 32 : N1P;
                     float vv[kV];
 #pragma unroll
@@ -851,14 +759,14 @@ __global__ void __launch_bounds__(kThreads, 1) fused_sm100(Params P, int stages)
                     }
 #pragma unroll
                     for (int h = 0; h < kV / 32; ++h) red[ew * 64 + base + h] = vv[h];
-                    if (!group_sync(&bars->sm_sync, ph, &ctl, P.status)) { ok = false; break; }
+                    if (!group_sync(&bars->sm_sync, ph, &ctl.abort, P.status)) { ok = false; break; }
                     for (int h = et; h < P.N1; h += 128) {
                         float a = 0.f;
                         for (int i = 0; i < 4; ++i) a += red[i * 64 + h];
                         P.dw[(int64_t)it.t * P.N1 + h] = a;
                     }
                     // dq^T readback (lane = d): columns = heads
-                    if (!wait_bar(&bars->dq_full, nb & 1, &ctl, P.status)) { ok = false; break; }
+                    if (!wait_bar(&bars->dq_full, nb & 1, &ctl.abort, P.status)) { ok = false; break; }
                     tc_fence_after();
                     if (quad * 32 < D) {
                         T *dqrow = reinterpret_cast<T *>(P.dq) + (int64_t)it.t * P.N1 * D;
@@ -902,10 +810,13 @@ cudaError_t launch_t(const Params &P, int workers, cudaStream_t s) {
     const int stages = 4;
     const SmemPlan sp = plan_smem<N1P>(stages);
     if (sp.total > 226 * 1024) return cudaErrorInvalidConfiguration;
-    auto k = fused_sm100<N1P, D, T>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp.total);
+    auto k = P.km ? fused_sm100<N1P, D, T, true> : fused_sm100<N1P, D, T, false>;
+    CUtensorMap qmap;
+    cudaError_t e = encode_q_map<N1P, T>(P, &qmap);
     if (e != cudaSuccess) return e;
-    k<<<workers, kThreads, sp.total, s>>>(P, stages);
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp.total);
+    if (e != cudaSuccess) return e;
+    k<<<workers, kThreads, sp.total, s>>>(P, stages, qmap);
     return cudaGetLastError();
 }
 

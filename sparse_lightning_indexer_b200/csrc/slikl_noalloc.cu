@@ -39,8 +39,11 @@ slikl_status slikl_grad_noalloc(const slikl_problem *problem, const slikl_tensor
                                 void *stream) {
     if (!problem) return SLIKL_ERR_PARAM_NULLPTR;
     if (problem->deterministic) return SLIKL_ERR_PARAM_INVALID;   // needs far more scratch
+    // the scatter dK path: its scratch does not grow with the key range
+    slikl_options opt{};
+    opt.dk_path = SLIKL_DK_SCATTER;
     size_t need = 0;
-    slikl_status st = slikl_grad_workspace_size(problem, &need);
+    slikl_status st = slikl_grad_workspace_size_ex(problem, &opt, &need);
     if (st != SLIKL_OK) return st;
     if (need > kNoAllocScratchBytes) return SLIKL_ERR_WORKSPACE_TOO_SMALL;
     if (!tensors) return SLIKL_ERR_PARAM_NULLPTR;
@@ -58,7 +61,7 @@ slikl_status slikl_grad_noalloc(const slikl_problem *problem, const slikl_tensor
         }
         scratch = g_scratch_addr[dev];
     }
-    return slikl_grad(problem, tensors, scratch, kNoAllocScratchBytes, stream);
+    return slikl_grad_ex(problem, tensors, scratch, kNoAllocScratchBytes, stream, &opt);
 }
 
 }  // extern "C"

@@ -49,8 +49,8 @@ def assert_close(name, got, ref):
         assert a <= mtol * m, f"{name}: max-abs {a:.3e} > {mtol} * {m:.3e}"
 
 
-def run_gpu(wl, deterministic=False):
-    res = sli.grad_workload(wl, deterministic=deterministic)
+def run_gpu(wl, deterministic=False, dk_path="auto"):
+    res = sli.grad_workload(wl, deterministic=deterministic, dk_path=dk_path)
     torch.cuda.synchronize()
     flags = sli.slikl_read_device_status(res["workspace"].data_ptr())
     T1, T2, N1, D, K = wl.T1, wl.T2, wl.N1, wl.D, wl.K
@@ -111,12 +111,23 @@ SMALL = [
 ]
 
 
+MODES = [(False, "scatter"), (False, "keymajor"), (True, "scatter")]
+MODE_IDS = ["scatter", "keymajor", "det"]
+
+
+def keymajor_possible(case):
+    return case["N1"] <= 64
+
+
 @pytest.mark.parametrize("case", SMALL, ids=lambda c: f"s{c['seed']}")
-@pytest.mark.parametrize("det", [False, True], ids=["atomic", "det"])
-def test_small_parity(case, det):
+@pytest.mark.parametrize("mode", MODES, ids=MODE_IDS)
+def test_small_parity(case, mode):
+    det, path = mode
+    if path == "keymajor" and not keymajor_possible(case):
+        pytest.skip("key-major dK path needs N1 <= 64")
     wl = si.small(**case)
     ref = oracle.grad(wl)
-    got = run_gpu(wl, deterministic=det)
+    got = run_gpu(wl, deterministic=det, dk_path=path)
     assert got["flags"] == 0
     check_exact(wl, got)
     check_against(wl, got, ref)
@@ -125,11 +136,27 @@ def test_small_parity(case, det):
 def test_config0_full_parity():
     wl = si.config(0)
     ref = oracle.grad(wl)
-    for det in (False, True):
-        got = run_gpu(wl, deterministic=det)
+    for det, path in MODES + [(False, "auto")]:
+        got = run_gpu(wl, deterministic=det, dk_path=path)
         assert got["flags"] == 0
         check_exact(wl, got)
         check_against(wl, got, ref)
+
+
+def test_keymajor_key_range_bound_too_small_flagged():
+    """TND keys with a promised key-range bound below a batch's real key count: the batch is
+    left out of the key-major records and the call flags it instead of faulting."""
+    wl = si.small(seed=23, layout="TND", B=3, S1=30, S2=700, N1=16, D=128, K=64,
+                  pattern="causal")
+    real = sli.key_range_bound_of(wl)
+    dev = torch.device("cuda")
+    t = {n: getattr(wl, n).to(dev) for n in ("q", "k", "w", "p", "idx")}
+    res = sli.grad(t["q"], t["k"], t["w"], t["p"], t["idx"], "TND", "TND",
+                   wl.cu_seqlens_q.to(dev), wl.cu_seqlens_k.to(dev), dk_path="keymajor",
+                   key_range_bound=max(1, real - 100))
+    torch.cuda.synchronize()
+    flags = sli.slikl_read_device_status(res["workspace"].data_ptr())
+    assert flags & sli.SLIKL_DEV_KEY_RANGE_ABOVE_S2
 
 
 def masked(wl, tokens):
@@ -159,19 +186,20 @@ def cfg(cid):
     return _CFG_CACHE[cid]
 
 
-@pytest.mark.parametrize("cid", [1, 2, 3, 4])
-def test_full_size_sampled_parity(cid):
+@pytest.mark.parametrize("cid,path", [(1, "auto"), (2, "auto"), (3, "auto"), (4, "auto"),
+                                      (1, "scatter"), (4, "scatter")])
+def test_full_size_sampled_parity(cid, path):
     wl = cfg(cid)
     toks = sample_tokens(wl, 48, seed=cid)
     ref = oracle.grad(wl, tokens=toks)
-    got = run_gpu(wl)
+    got = run_gpu(wl, dk_path=path)
     assert got["flags"] == 0
     check_exact(wl, got)
     for name in ("y", "dw", "dq"):
         assert_close(name, got[name][toks], ref[name][toks])
     # full dk on the masked problem of the same shape
     wm = masked(wl, toks)
-    gm = run_gpu(wm)
+    gm = run_gpu(wm, dk_path=path)
     assert gm["flags"] == 0
     check_exact(wm, gm)
     assert_close("dk", gm["dk"], ref["dk"])
