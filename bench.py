@@ -145,6 +145,26 @@ def raw_elapsed_ms(a, b):
     return ms
 
 
+def combine_over_ranks(local, world, device):
+    """Max over ranks of each per-rank time (seconds); local list of floats. With one rank the
+    values are returned as they are. Every rank must call this (it is a collective)."""
+    if world <= 1:
+        return list(local)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(local), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def fused_algorithmic_flop(wl, dk_path):
+    """Algorithmic FLOPs of one fused-kernel launch at the nominal slot count: the S and dq
+    products (2 N1 D each per slot), plus the dK product (2 N1 D) when the fused kernel forms dK
+    itself (scatter path). The second S product of pass B is recomputation, not counted."""
+    per_slot = 4.0 if dk_path == "keymajor" else 6.0
+    return per_slot * wl.N1 * wl.D * wl.K * wl.T1
+
+
 def oracle_rate(wl, ntok, seed=0):
     """fp64 oracle on a seeded sample of ntok query tokens; returns (tokens/s, cores, secs)."""
     import oracle  # CPU baseline leg only
@@ -190,8 +210,9 @@ def main():
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--deterministic", action="store_true")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--ref-tokens", type=int, default=96)
-    ap.add_argument("--cpu-baseline-tokens", type=int, default=1024)
+    ap.add_argument("--ref-tokens", type=int, default=512)
+    ap.add_argument("--cpu-baseline-tokens", type=int, default=12000)
+    ap.add_argument("--dk-path", default="auto", choices=["auto", "scatter", "keymajor"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -221,8 +242,11 @@ def main():
     cuq = wl.cu_seqlens_q.to(dev) if wl.cu_seqlens_q is not None else None
     cuk = wl.cu_seqlens_k.to(dev) if wl.cu_seqlens_k is not None else None
     B = wl.B if wl.layout == "TND" else None
-    pr = sli.make_problem(q, k, idx, wl.layout, wl.layout, args.deterministic, B)
-    nbytes = sli.slikl_grad_workspace_size(pr)
+    pr = sli.make_problem(q, k, idx, wl.layout, wl.layout, args.deterministic, B,
+                          sli.key_range_bound_of(wl))
+    base_opt = sli.make_options(args.dk_path)
+    dk_path = "keymajor" if sli.slikl_grad_dk_path(pr, base_opt) == sli.SLIKL_DK_KEYMAJOR else "scatter"
+    nbytes = sli.slikl_grad_workspace_size_ex(pr, base_opt)
     ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
     out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dw=torch.empty_like(w),
                softmax_out=torch.empty_like(p))
@@ -242,11 +266,8 @@ def main():
     sid = stream.cuda_stream
 
     def step(evs=None):
-        if evs is None:
-            sli.slikl_grad(pr, tn, ws.data_ptr(), nbytes, sid)
-        else:
-            sli.slikl_grad_with_events(pr, tn, ws.data_ptr(), nbytes, sid, int(evs[0]),
-                                       int(evs[1]))
+        opt = base_opt if evs is None else sli.make_options(args.dk_path, *(int(e) for e in evs))
+        sli.slikl_grad_ex(pr, tn, ws.data_ptr(), nbytes, sid, opt)
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
@@ -261,7 +282,7 @@ def main():
         time.sleep(0.3)
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
-        kev = [(raw_event(), raw_event()) for _ in range(args.steps)]
+        kev = [tuple(raw_event() for _ in range(4)) for _ in range(args.steps)]
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
@@ -274,7 +295,8 @@ def main():
         if world > 1:
             dist.barrier()
         step_ms = [a.elapsed_time(b) for a, b in ev]
-        kern_ms = [raw_elapsed_ms(a, b) for a, b in kev]
+        kern_ms = [raw_elapsed_ms(e[0], e[1]) for e in kev]
+        dk_ms = [raw_elapsed_ms(e[2], e[3]) for e in kev]
         flags = sli.slikl_read_device_status(ws.data_ptr(), sid)
 
         # end to end through the public API with pinned host buffers
@@ -291,7 +313,7 @@ def main():
             a.record(stream)
             for dst, src in ((q2, hq), (k2, hk), (w2, hw), (p2, hp), (i2, hi)):
                 dst.copy_(src, non_blocking=True)
-            sli.slikl_grad(pr, tn2, ws.data_ptr(), nbytes, sid)
+            sli.slikl_grad_ex(pr, tn2, ws.data_ptr(), nbytes, sid, base_opt)
             for n, t in out.items():
                 hout[n].copy_(t, non_blocking=True)
             b.record(stream)
@@ -300,26 +322,22 @@ def main():
                 e2e_ms.append(a.elapsed_time(b))
         clk = clocks.stop()
 
-    t_total = sum(step_ms) / 1e3
-    t_e2e = sum(e2e_ms) / 1e3
-    if world > 1:
-        tt = torch.tensor([t_total, t_e2e, sum(kern_ms) / 1e3], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_total, t_e2e, t_kern = tt.tolist()
-    else:
-        t_kern = sum(kern_ms) / 1e3
+    t_total, t_e2e, t_kern, t_dk = combine_over_ranks(
+        [sum(step_ms) / 1e3, sum(e2e_ms) / 1e3, sum(kern_ms) / 1e3, sum(dk_ms) / 1e3], world, dev)
     tokens = wl.T1 * args.steps * world
     value = tokens / t_total
     peaks, peak_src = load_peaks()
     k_avg = t_kern / args.steps
+    dk_avg = t_dk / args.steps
     flop = stats["flop_nom"]
-    achieved_tf = flop / k_avg / 1e12
+    kflop = fused_algorithmic_flop(wl, dk_path)
+    achieved_tf = kflop / k_avg / 1e12
     peak_tf = peaks["bf16_tflops"]
     step_avg = t_total / args.steps
     t_roof = max(flop / (peak_tf * 1e12), stats["bytes"] / (peaks["hbm_gbs"] * 1e9))
     # our kernels per call: 3 work-split + fused + (cast | sort init, 3 per radix pass,
-    # row pointers, segmented reduce)
-    launches_per_step = 5
+    # row pointers, segmented reduce); the key-major path adds 2 metadata kernels and its dK kernel
+    launches_per_step = 5 + (3 if dk_path == "keymajor" else 0)
     if args.deterministic:
         passes = (int(wl.T2).bit_length() + 7) // 8
         launches_per_step = 3 + 1 + 1 + 3 * passes + 2
@@ -337,6 +355,7 @@ def main():
             "data": "synthetic (seeded, shaped like the operator's workloads)",
             "config": {"workload": wl.name, "T1": wl.T1, "T2": wl.T2, "N1": wl.N1, "D": wl.D,
                        "topk": wl.K, "deterministic": bool(args.deterministic),
+                       "dk_path": dk_path,
                        "l2": "flushed before every timed step (256 MiB write, outside the events)",
                        "parallelism": f"replicas x{world}"},
             "tflops_nominal": flop / step_avg / 1e12,
@@ -346,8 +365,11 @@ def main():
                               "peaks": peak_src},
             "roofline": {"bound": "tensor", "achieved": achieved_tf, "peak": peak_tf,
                          "unit": "TFLOP/s", "frac": achieved_tf / peak_tf, "traffic": None,
-                         "kernel": "fused per-token kernel", "peak_source": f"bf16_tflops ({peak_src})"},
-            "fused_kernel_ms": 1e3 * k_avg,
+                         "kernel": "fused_sm100 (fused per-token kernel)",
+                         "algorithmic_flop_per_launch": kflop,
+                         "peak_source": f"bf16_tflops, burst ({peak_src})"},
+            "stages_ms": {"fused": 1e3 * k_avg, "dk": 1e3 * dk_avg,
+                          "memset_and_work_split": 1e3 * (step_avg - k_avg - dk_avg)},
             "e2e": {"value": tokens / t_e2e, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": launches_per_step * args.steps,

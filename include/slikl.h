@@ -163,6 +163,10 @@ typedef struct {
     int32_t dk_path;     /* SLIKL_DK_AUTO, SLIKL_DK_SCATTER or SLIKL_DK_KEYMAJOR */
     void *fused_begin;   /* optional cudaEvent_t recorded just before the fused kernel, or NULL */
     void *fused_end;     /* optional cudaEvent_t recorded just after it, or NULL */
+    void *dk_begin;      /* optional cudaEvent_t recorded before the dK stage that follows the
+                            fused kernel (key-major kernel and cast, the cast alone, or the
+                            deterministic reduction), or NULL */
+    void *dk_end;        /* optional cudaEvent_t recorded after that stage, or NULL */
 } slikl_options;
 
 /*
@@ -177,6 +181,14 @@ SLIKL_API slikl_status slikl_grad_workspace_size_ex(const slikl_problem *problem
 SLIKL_API slikl_status slikl_grad_ex(const slikl_problem *problem, const slikl_tensors *tensors,
                                      void *workspace, size_t workspace_bytes, void *stream,
                                      const slikl_options *options);
+
+/*
+ * The dK path slikl_grad_ex would take for `problem` with `options` (NULL = SLIKL_DK_AUTO):
+ * writes SLIKL_DK_SCATTER or SLIKL_DK_KEYMAJOR to *path. Host only, no CUDA call.
+ * Errors: SLIKL_ERR_INNER_NULLPTR (path NULL) and those of slikl_grad_workspace_size_ex.
+ */
+SLIKL_API slikl_status slikl_grad_dk_path(const slikl_problem *problem,
+                                          const slikl_options *options, int32_t *path);
 
 /*
  * slikl_grad with a measurement aid: when fused_begin / fused_end are not NULL they are

@@ -43,7 +43,7 @@ SLIKL_DK_KEYMAJOR = 2
 _DK_PATHS = {"auto": SLIKL_DK_AUTO, "scatter": SLIKL_DK_SCATTER, "keymajor": SLIKL_DK_KEYMAJOR}
 
 EXPORTED = ("slikl_grad_workspace_size", "slikl_grad", "slikl_grad_with_events",
-            "slikl_grad_workspace_size_ex", "slikl_grad_ex",
+            "slikl_grad_workspace_size_ex", "slikl_grad_ex", "slikl_grad_dk_path",
             "slikl_read_device_status",
             "slikl_grad_metadata_size", "slikl_grad_metadata_workspace_size",
             "slikl_grad_metadata", "slikl_status_string", "slikl_grad_noalloc")
@@ -67,14 +67,19 @@ class slikl_tensors(ctypes.Structure):
 
 class slikl_options(ctypes.Structure):
     _fields_ = [("dk_path", ctypes.c_int32), ("fused_begin", ctypes.c_void_p),
-                ("fused_end", ctypes.c_void_p)]
+                ("fused_end", ctypes.c_void_p), ("dk_begin", ctypes.c_void_p),
+                ("dk_end", ctypes.c_void_p)]
 
 
-def make_options(dk_path="auto", fused_begin: int = 0, fused_end: int = 0) -> slikl_options:
+def make_options(dk_path="auto", fused_begin: int = 0, fused_end: int = 0, dk_begin: int = 0,
+                 dk_end: int = 0) -> slikl_options:
+    """Options of slikl_grad_ex; the event arguments are cudaEvent_t handles (ints) or 0."""
     o = slikl_options()
     o.dk_path = _DK_PATHS[dk_path] if isinstance(dk_path, str) else int(dk_path)
     o.fused_begin = fused_begin or None
     o.fused_end = fused_end or None
+    o.dk_begin = dk_begin or None
+    o.dk_end = dk_end or None
     return o
 
 
@@ -103,6 +108,8 @@ def load_library() -> ctypes.CDLL:
                                                      P(ctypes.c_size_t)]
         lib.slikl_grad_ex.argtypes = [P(slikl_problem), P(slikl_tensors), VP, ctypes.c_size_t,
                                       VP, P(slikl_options)]
+        lib.slikl_grad_dk_path.argtypes = [P(slikl_problem), P(slikl_options), P(ctypes.c_int32)]
+        lib.slikl_grad_dk_path.restype = ctypes.c_int32
         lib.slikl_read_device_status.argtypes = [VP, VP, P(ctypes.c_uint32)]
         lib.slikl_grad_metadata_size.argtypes = [ctypes.c_int32]
         lib.slikl_grad_metadata_size.restype = ctypes.c_int64
@@ -171,6 +178,17 @@ def slikl_grad_ex(problem: slikl_problem, tensors: slikl_tensors, workspace: int
                                       ctypes.byref(options) if options is not None else None)
     if rc != SLIKL_OK:
         raise SliklError(rc, "slikl_grad_ex")
+
+
+def slikl_grad_dk_path(problem: slikl_problem, options: Optional[slikl_options] = None) -> int:
+    """SLIKL_DK_SCATTER or SLIKL_DK_KEYMAJOR: the dK path slikl_grad_ex would take."""
+    v = ctypes.c_int32(0)
+    rc = load_library().slikl_grad_dk_path(
+        ctypes.byref(problem), ctypes.byref(options) if options is not None else None,
+        ctypes.byref(v))
+    if rc != SLIKL_OK:
+        raise SliklError(rc, "slikl_grad_dk_path")
+    return int(v.value)
 
 
 def slikl_read_device_status(workspace: int, stream: int = 0) -> int:

@@ -148,6 +148,7 @@ Params make_params(const slikl_problem *pr, const Derived &dv, const slikl_tenso
         P.tok_pairs = reinterpret_cast<uint32_t *>(base + L.tok_pairs);
         P.rec = base + L.rec;
         P.units = reinterpret_cast<int4 *>(base + L.units);
+        P.units_c = reinterpret_cast<int4 *>(base + L.units_c);
         P.unit_off = reinterpret_cast<int64_t *>(base + L.unit_off);
         P.unit_prefix = reinterpret_cast<int64_t *>(base + L.unit_prefix);
         P.km_range = reinterpret_cast<int32_t *>(base + L.km_range);
@@ -190,6 +191,18 @@ slikl_status slikl_grad_workspace_size_ex(const slikl_problem *problem,
     if (st != SLIKL_OK) return st;
     *workspace_bytes = make_layout(dv.T1, dv.T2, problem->topk, problem->D,
                                    problem->deterministic, dv.km, problem->B).total;
+    return SLIKL_OK;
+}
+
+slikl_status slikl_grad_dk_path(const slikl_problem *problem, const slikl_options *options,
+                                int32_t *path) {
+    if (!path) return SLIKL_ERR_INNER_NULLPTR;
+    Derived dv;
+    slikl_status st = validate(problem, &dv);
+    if (st != SLIKL_OK) return st;
+    st = choose_dk_path(problem, &dv, options ? options->dk_path : SLIKL_DK_AUTO);
+    if (st != SLIKL_OK) return st;
+    *path = dv.km.km ? SLIKL_DK_KEYMAJOR : SLIKL_DK_SCATTER;
     return SLIKL_OK;
 }
 
@@ -252,9 +265,16 @@ slikl_status slikl_grad_ex(const slikl_problem *problem, const slikl_tensors *te
     }
     if (fused_end && cudaEventRecord(static_cast<cudaEvent_t>(fused_end), s) != cudaSuccess)
         return SLIKL_ERR_CUDA;
+    void *dk_begin = options ? options->dk_begin : nullptr;
+    void *dk_end = options ? options->dk_end : nullptr;
+    if (dk_begin && cudaEventRecord(static_cast<cudaEvent_t>(dk_begin), s) != cudaSuccess)
+        return SLIKL_ERR_CUDA;
     if (P.km && dv.T1 > 0 && launch_dk_keymajor(P, workers, s) != cudaSuccess) return SLIKL_ERR_CUDA;
     cudaError_t e = P.deterministic ? launch_deterministic_reduce(P, s) : launch_cast(P, s);
-    return e == cudaSuccess ? SLIKL_OK : SLIKL_ERR_CUDA;
+    if (e != cudaSuccess) return SLIKL_ERR_CUDA;
+    if (dk_end && cudaEventRecord(static_cast<cudaEvent_t>(dk_end), s) != cudaSuccess)
+        return SLIKL_ERR_CUDA;
+    return SLIKL_OK;
 }
 
 slikl_status slikl_read_device_status(const void *workspace, void *stream, uint32_t *flags) {

@@ -52,6 +52,7 @@ struct Params {
     void *rec;            // [T1][S2m] records {dI, ReLU(S) > 0 mask of the heads}
     int4 *units;          // [units_max] {first token, first key row, local key | keys << 16,
                           //              token mask}: 32 tokens x one 256-key block pair
+    int4 *units_c;        // [units_max] the units that hold at least one row, in order
     int64_t *unit_off;    // [B + 1] first unit of each batch; unit_off[B] = unit count
     int64_t *unit_prefix; // [units_max + 1] exclusive prefix of the unit costs
     int32_t *km_range;    // [kMaxWorkers + 1] first unit of each worker of the key-major kernel
@@ -69,7 +70,7 @@ struct KmShape {
 struct WsLayout {
     size_t status, meta, tok_kbase, tok_klen, tok_cost, tok_tiles, cost_prefix;
     size_t dk_acc, partials, keys0, vals0, keys1, vals1, hist, row_ptr;
-    size_t tok_pairs, rec, units, unit_off, unit_prefix, km_range;
+    size_t tok_pairs, rec, units, units_c, unit_off, unit_prefix, km_range;
     size_t total;
 };
 
@@ -103,6 +104,7 @@ inline WsLayout make_layout(int64_t T1, int64_t T2, int64_t K, int64_t D, int de
     L.tok_pairs = take(k ? sizeof(uint32_t) * (size_t)T1 * km.nkpw : 0);
     L.rec = take(k ? (size_t)T1 * (size_t)km.S2m * km.rec_bytes : 0);
     L.units = take(k ? 16 * (size_t)km.units_max : 0);
+    L.units_c = take(k ? 16 * (size_t)km.units_max : 0);
     L.unit_off = take(k ? sizeof(int64_t) * (size_t)(B + 1) : 0);
     L.unit_prefix = take(k ? sizeof(int64_t) * (size_t)(km.units_max + 1) : 0);
     L.km_range = take(k ? sizeof(int32_t) * (kMaxWorkers + 1) : 0);

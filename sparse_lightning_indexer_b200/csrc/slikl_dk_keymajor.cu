@@ -21,14 +21,14 @@
 // buffers and is flushed once, with red.global.add.f32 of 32 consecutive d per warp
 // instruction, into the fp32 dK rows.
 //
-// Warp roles (512 threads):
+// Warp roles (768 threads):
 //   warp 0      producer: per query row, TMA of q_t (128-byte swizzle, zero heads past N1)
 //               and a bulk copy of the pair's 256 records (lane 0); w_t through registers
 //   warp 1      MMA issuer and TMEM owner
 //   warps 2-3   idle
 //   warps 4-7   flush: finished dK^T buffers from TMEM to the fp32 key rows
-//   warps 8-15  dS builders: one key of the pair per thread, written as a 128-byte K-major
-//               row (heads contiguous) with the 128-byte swizzle
+//   warps 8-23  dS builders: two threads per key of the pair, each writing half of its
+//               128-byte K-major row (heads contiguous) with the 128-byte swizzle
 //
 // Every mbarrier wait is bounded; on expiry the CTA sets SLIKL_DEV_WAIT_TIMEOUT, the roles
 // stop, in-flight copies and MMAs are waited for (again bounded), TMEM is freed.
@@ -41,13 +41,13 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kKmThreads = 512;
+constexpr int kKmThreads = 768;
 constexpr int kKmStages = 4;
 constexpr int kKmTmemCols = 512;         // two dK^T buffers of 256 columns
 
 struct KmBarriers {
     uint64_t full[kKmStages];            // q, w, records landed (producer, TMA bytes)
-    uint64_t dsr[kKmStages];             // dS tile written (8 builder warps)
+    uint64_t dsr[kKmStages];             // dS tile written (16 builder warps)
     uint64_t empty[kKmStages];           // stage consumed by the MMA (tcgen05.commit)
     uint64_t accf[2];                    // dK^T buffer complete (tcgen05.commit)
     uint64_t acce[2];                    // dK^T buffer flushed (4 flush warps)
@@ -137,19 +137,6 @@ struct KmIter {
     }
 };
 
-template <typename T>
-__device__ __forceinline__ uint32_t pack2(float a, float b);
-template <>
-__device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float a, float b) {
-    const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
-    return *reinterpret_cast<const uint32_t *>(&v);
-}
-template <>
-__device__ __forceinline__ uint32_t pack2<__half>(float a, float b) {
-    const __half2 v = __floats2half2_rn(a, b);
-    return *reinterpret_cast<const uint32_t *>(&v);
-}
-
 template <int N1P, int D, typename T>
 __global__ void __launch_bounds__(kKmThreads, 1)
     dk_keymajor(Params P, const __grid_constant__ CUtensorMap qmap) {
@@ -172,7 +159,7 @@ __global__ void __launch_bounds__(kKmThreads, 1)
         abort_flag = 0;
         for (int s = 0; s < kKmStages; ++s) {
             mbar_init(&bars->full[s], 1);
-            mbar_init(&bars->dsr[s], 8);
+            mbar_init(&bars->dsr[s], 16);
             mbar_init(&bars->empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -202,7 +189,7 @@ __global__ void __launch_bounds__(kKmThreads, 1)
     const uint32_t tacc = tmem_base;
 
     KmIter iter;
-    iter.init(P.units, u0, u1);
+    iter.init(P.units_c, u0, u1);
     KmItem it;
 
     if (warp == 0) {
@@ -314,35 +301,45 @@ __global__ void __launch_bounds__(kKmThreads, 1)
         }
     } else if (warp >= 8) {
         // =============================== dS builders ===============================
-        const int e = threadIdx.x - 256;          // key of the pair, 0..255
+        // two threads per key of the pair: heads [32 h, 32 h + 32) of key e
+        const int e = (threadIdx.x - 256) >> 1;   // key of the pair, 0..255
+        const int half = threadIdx.x & 1;
+        constexpr int kChunks = N1P / 8;          // 16-byte chunks of 8 heads per row
+        constexpr int kHalfChunks = kChunks < 4 ? kChunks : 4;
+        const bool has_work = half * 4 < kChunks;
         uint32_t i = 0;
         while (iter.next(it)) {
             const int s = i % kKmStages;
             if (!wait_bar(&bars->full[s], (i / kKmStages) & 1, &abort_flag, P.status)) break;
-            uint32_t m0, m1 = 0;
-            float dI;
-            const uint8_t *rp = smem + SP.rec + s * 256 * RB + e * RB;
-            if (RB == 16) {
-                const uint4 r = *reinterpret_cast<const uint4 *>(rp);
-                m0 = r.x; m1 = r.y; dI = __uint_as_float(r.z);
-            } else {
-                const uint2 r = *reinterpret_cast<const uint2 *>(rp);
-                m0 = r.x; dI = __uint_as_float(r.y);
-            }
-            const float *ws = reinterpret_cast<const float *>(smem + SP.w + s * N1P * 4);
-            uint8_t *row = smem + SP.ds + s * 256 * 128 + e * 128;
+            if (has_work) {
+                uint32_t m;
+                float dI;
+                const uint8_t *rp = smem + SP.rec + s * 256 * RB + e * RB;
+                if (RB == 16) {
+                    const uint4 r = *reinterpret_cast<const uint4 *>(rp);
+                    m = half ? r.y : r.x;
+                    dI = __uint_as_float(r.z);
+                } else {
+                    const uint2 r = *reinterpret_cast<const uint2 *>(rp);
+                    m = r.x;
+                    dI = __uint_as_float(r.y);
+                }
+                const float *ws = reinterpret_cast<const float *>(smem + SP.w + s * N1P * 4) + 32 * half;
+                uint8_t *row = smem + SP.ds + s * 256 * 128 + e * 128;
 #pragma unroll
-            for (int c = 0; c < N1P / 8; ++c) {       // 8 heads = one 16-byte chunk
-                const float4 wa = *reinterpret_cast<const float4 *>(ws + 8 * c);
-                const float4 wb = *reinterpret_cast<const float4 *>(ws + 8 * c + 4);
-                const uint32_t mb = ((c < 4 ? m0 : m1) >> ((c & 3) * 8)) & 0xFFu;
-                const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-                float d[8];
+                for (int cc = 0; cc < kHalfChunks; ++cc) {   // 8 heads = one 16-byte chunk
+                    const int c = half * 4 + cc;
+                    const float4 wa = *reinterpret_cast<const float4 *>(ws + 8 * cc);
+                    const float4 wb = *reinterpret_cast<const float4 *>(ws + 8 * cc + 4);
+                    const uint32_t mb = (m >> (cc * 8)) & 0xFFu;
+                    const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+                    float d[8];
 #pragma unroll
-                for (int h = 0; h < 8; ++h) d[h] = ((mb >> h) & 1u) ? dI * wv[h] : 0.f;
-                const uint4 o = make_uint4(pack2<T>(d[0], d[1]), pack2<T>(d[2], d[3]),
-                                           pack2<T>(d[4], d[5]), pack2<T>(d[6], d[7]));
-                *reinterpret_cast<uint4 *>(row + (((c ^ e) & 7) << 4)) = o;
+                    for (int h = 0; h < 8; ++h) d[h] = ((mb >> h) & 1u) ? dI * wv[h] : 0.f;
+                    const uint4 o = make_uint4(pack2<T>(d[0], d[1]), pack2<T>(d[2], d[3]),
+                                               pack2<T>(d[4], d[5]), pack2<T>(d[6], d[7]));
+                    *reinterpret_cast<uint4 *>(row + (((c ^ e) & 7) << 4)) = o;
+                }
             }
             fence_proxy_async();
             __syncwarp();

@@ -80,11 +80,11 @@ __host__ __device__ inline SmemPlan plan_smem(int stages) {
     s.stages = stages;
     s.kv = take(stages * kStageBytes, 1024);
     s.q = take(2 * N1P * 256, 1024);                 // two buffers, 2 column blocks each
-    s.ds = take(2 * N1P * 256, 1024);                // two buffers [N1P heads x 128 keys]
+    s.ds = take(2 * 128 * 128, 1024);                // two buffers [128 keys x 64 heads]
     s.w = take(2 * N1P * 4, 16);                     // w of two tokens
     s.rows = take(2 * kRowsStride * 4, 16);          // key rows of two dS tiles
     s.red = take(4 * 64 * 4, 16);
-    s.ring = take(3 * 4 * kRingSlot * 4, 16);
+    s.ring = take(7 * 4 * kRingSlot * 4, 16);       // up to 7 producer warps
     s.bar = take(sizeof(Barriers) + 16, 8);
     s.total = off + 1024;                            // slack for aligning the dynamic base
     return s;
@@ -109,23 +109,15 @@ struct Item {
 };
 
 // Phase 0 = A(t_0); phase k = B(t_(k-1)) and A(t_k) alternated (B first), then whichever
-// remains; the final phase = B(t_last).
-// Within a token the tiles are visited from a CTA-dependent starting tile (a rotation of the
-// tile order): CTAs working on neighbouring tokens then scatter into different key rows at
-// the same time instead of contending for the same L2 lines.
+// remains; the final phase = B(t_last). Tiles of a token are visited in index order. Every
+// role runs this for every item, so it stays a handful of instructions per item.
 struct Sched {
     const uint64_t *tiles;
-    int t_next, t_end, nt;
-    int ta, oa, ra; uint64_t ma, ma_all; bool a_on, a_first, a_exists;
-    int tb, ob, rb; uint64_t mb; bool b_on, b_first;
+    int t_next, t_end;
+    int ta, oa; uint64_t ma, ma_all; bool a_on, a_first, a_exists;
+    int tb, ob; uint64_t mb; bool b_on, b_first;
     int next_ord;
     bool turn_b;
-
-    __device__ uint64_t rot(uint64_t m, int r) const {
-        if (r == 0) return m;
-        const uint64_t full = nt >= 64 ? ~0ull : ((1ull << nt) - 1);
-        return ((m >> r) | (m << (nt - r))) & full;
-    }
 
     __device__ bool find_a() {
         for (; t_next < t_end; ++t_next) {
@@ -133,8 +125,7 @@ struct Sched {
             if (m) {
                 ta = t_next++;
                 oa = next_ord++;
-                ra = (int)((blockIdx.x * 7u + (unsigned)ta * 3u) % (unsigned)nt);
-                ma = ma_all = rot(m, ra);
+                ma = ma_all = m;
                 a_on = true;
                 a_first = true;
                 return true;
@@ -143,8 +134,8 @@ struct Sched {
         a_on = false;
         return false;
     }
-    __device__ void init(const uint64_t *tl, int t0, int t1, int ntiles) {
-        tiles = tl; t_next = t0; t_end = t1; next_ord = 0; nt = ntiles;
+    __device__ void init(const uint64_t *tl, int t0, int t1) {
+        tiles = tl; t_next = t0; t_end = t1; next_ord = 0;
         b_on = false; turn_b = true;
         a_exists = find_a();
     }
@@ -156,14 +147,14 @@ struct Sched {
         turn_b = !turn_b;
         if (take_b) {
             it.kind = 1; it.t = tb; it.ord = ob; it.first = b_first;
-            it.tile = (__ffsll((long long)mb) - 1 + rb) % nt;
+            it.tile = __ffsll((long long)mb) - 1;
             mb &= mb - 1;
             it.last = mb == 0;
             b_first = false;
             if (it.last) b_on = false;
         } else {
             it.kind = 0; it.t = ta; it.ord = oa; it.first = a_first;
-            it.tile = (__ffsll((long long)ma) - 1 + ra) % nt;
+            it.tile = __ffsll((long long)ma) - 1;
             ma &= ma - 1;
             it.last = ma == 0;
             a_first = false;
@@ -171,7 +162,7 @@ struct Sched {
         }
         if (!a_on && !b_on) {
             // phase ends: its A token becomes the B token of the next phase
-            if (a_exists) { tb = ta; ob = oa; rb = ra; mb = ma_all; b_on = true; b_first = true; }
+            if (a_exists) { tb = ta; ob = oa; mb = ma_all; b_on = true; b_first = true; }
             a_exists = find_a();
             turn_b = true;
         }
@@ -194,11 +185,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     __shared__ Ctl ctl;
     constexpr int kFmt = std::is_same<T, __nv_bfloat16>::value ? 1 : 0;
     constexpr uint32_t kIdescS = idesc_f16(kFmt, 128, N1P, 0, 0);
-    constexpr uint32_t kIdescDq = idesc_f16(kFmt, 128, N1P, 1, 0);
-    constexpr uint32_t kIdescDk = idesc_f16(kFmt, 128, 128, 1, 1);
+    // dq^T [D x 64 heads]: dS^T read MN-major from the [keys x heads] tile (heads past N1P
+    // are zero columns); dK^T [D x 128 keys]: the same tile read K-major
+    constexpr uint32_t kIdescDq = idesc_f16(kFmt, 128, 64, 1, 1);
+    constexpr uint32_t kIdescDk = idesc_f16(kFmt, 128, 128, 1, 0);
     constexpr int kDChunks = D / 8;          // 16-byte chunks per key row
     constexpr int kC = N1P < 32 ? N1P : 32;  // S columns per TMEM load
     constexpr int kRecBytes = N1P > 32 ? 16 : 8;  // record: ReLU mask word(s), dI
+    // producer warps: 0-2, and in record mode also 4-7 (the scatter group has no work there)
+    constexpr int kProd = kRec ? 7 : 3;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t0 = P.meta[kMetaHeader + 2 * blockIdx.x];
@@ -208,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         ctl.abort = 0;
         for (int s = 0; s < stages; ++s) {
-            mbar_init(&bars->kv_full[s], 96);       // one arrival per producer thread
+            mbar_init(&bars->kv_full[s], 32 * kProd);   // one arrival per producer thread
             mbar_init(&bars->kv_empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -227,6 +222,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&bars->sm_sync, 4);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
+    // zero the dS tiles once: heads past N1P stay 0 (the dq product reads 64 heads)
+    for (uint32_t i = threadIdx.x; i < 2 * 16384 / 16; i += kThreads)
+        reinterpret_cast<uint4 *>(smem + SP.ds)[i] = make_uint4(0, 0, 0, 0);
     // zero the q buffers once: padded heads and, for D = 64, the upper column block stay 0;
     // for D = 64 also the upper column block of every K stage (never written by the gather)
     for (uint32_t i = threadIdx.x; i < (uint32_t)(2 * N1P * 256 / 16); i += kThreads)
@@ -254,14 +252,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     int32_t *rows_s = reinterpret_cast<int32_t *>(smem + SP.rows);   // [2][kRowsStride]
 
     Sched sc;
-    sc.init(P.tok_tiles, t0, t1, (K + 127) / 128);
+    sc.init(P.tok_tiles, t0, t1);
 
-    if (warp < 3) {
+    if (warp < 3 || (kRec && warp >= 4 && warp < 8)) {
         // =============================== producers ===============================
         // Every producer warp walks every item in order and waits on every stage phase (a warp
         // that skipped items could be fooled by the phase parity of a reused stage); each warp
-        // copies its own third of the tile's row groups. Every lane ends an item with
-        // cp.async.mbarrier.arrive.noinc, so a stage turns full (96 arrivals) when all of its
+        // copies its share of the tile's row groups. Every lane ends an item with
+        // cp.async.mbarrier.arrive.noinc, so a stage turns full (32 arrivals per producer warp) when all of its
         // copies have landed, without any producer waiting for them (that arrival also waits
         // for every earlier cp.async of the thread, so nothing else is copied with cp.async).
         // The slot indices, key base and key count of an item are loaded into registers four
@@ -271,7 +269,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int chunk = lane % kDChunks;
         constexpr int kRowsPerPass = 32 / kDChunks;       // 2 (D=128) or 4 (D=64)
         const char *kbase_ptr = static_cast<const char *>(P.k);
-        int32_t *ring = reinterpret_cast<int32_t *>(smem + SP.ring) + warp * 4 * kRingSlot;
+        const int pw = warp < 3 ? warp : warp - 1;      // producer index 0 .. kProd - 1
+        int32_t *ring = reinterpret_cast<int32_t *>(smem + SP.ring) + pw * 4 * kRingSlot;
         bool ok = true;
         auto arrive_on_copies = [&](uint64_t *bar) {
             asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
@@ -326,20 +325,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int32_t kb = slot[128], kl = slot[129];
             const int jbase = it0.tile * 128;
             const uint32_t dst = smem_u32(smem + SP.kv + s * kStageBytes) + (chunk >> 3) * 16384;
-            // this warp's row groups i = warp, warp + 3, ...: all slot indices into registers
+            // this warp's row groups i = pw, pw + kProd, ...: all slot indices into registers
             // first, then the copies back to back (a shared-memory load issued after a copy
             // waits behind it in the memory pipeline)
             constexpr int kGroups = 128 / kRowsPerPass;       // 64 (D=128) or 32 (D=64)
-            constexpr int kPer = (kGroups + 2) / 3;
+            constexpr int kPer = (kGroups + kProd - 1) / kProd;
             int32_t vv[kPer];
 #pragma unroll
             for (int j = 0; j < kPer; ++j) {
-                const int i = warp + 3 * j;
+                const int i = pw + kProd * j;
                 vv[j] = i < kGroups ? slot[rsub + kRowsPerPass * i] : -1;
             }
 #pragma unroll
             for (int j = 0; j < kPer; ++j) {
-                const int i = warp + 3 * j;
+                const int i = pw + kProd * j;
                 if (i < kGroups) {
                     const int r = rsub + kRowsPerPass * i;
                     const int32_t v = vv[j];
@@ -416,12 +415,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 if (lane == 0) {
                     const uint32_t kaddr = kv0 + st_cur * kStageBytes;
-                    const uint32_t dsaddr = ds0 + b * N1P * 256;
+                    const uint32_t dsaddr = ds0 + b * 16384;
                     const uint32_t qaddr = q0 + (cur.ord & 1) * N1P * 256;
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks) {        // 128 keys, 16 per step
                         const uint64_t a = sdesc(kaddr + ks * 2048, 16384, 1024);
-                        const uint64_t bd = sdesc(dsaddr + (ks >> 2) * (N1P * 128) + (ks & 3) * 32, 16, 1024);
+                        const uint64_t bd = sdesc(dsaddr + ks * 2048, 16384, 1024);
                         umma_f16(tm_dq, a, bd, kIdescDq, (!cur.first || ks > 0) ? 1u : 0u);
                     }
                     umma_commit(&bars->kv_empty[st_cur]);
@@ -431,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int ks = 0; ks < N1P / 16; ++ks) {  // N1P heads, 16 per step
                             const uint64_t a = sdesc(qaddr + ks * 2048, N1P * 128, 1024);
-                            const uint64_t bd = sdesc(dsaddr + ks * 2048, N1P * 128, 1024);
+                            const uint64_t bd = sdesc(dsaddr + ks * 32, 16, 1024);
                             umma_f16(tm_dk + b * 128, a, bd, kIdescDk, ks > 0);
                         }
                         umma_commit(&bars->dk_full[b]);
@@ -664,8 +663,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const uint32_t sa = tm_s + sb * N1P + lane_addr;
                 const uint32_t dwa = tm_dw + lane_addr;
-                uint8_t *dsb = ds_tiles + b * N1P * 256 + (lrow >> 6) * (N1P * 128);
-                const int jj = lrow & 63;
+                // this slot's row of the [keys x heads] dS tile: 128 bytes, 16-byte chunks swizzled
+                uint8_t *dsrow = ds_tiles + b * 16384 + lrow * 128;
                 uint64_t smask = 0;                 // heads with S > 0 (record mode)
                 // 16 heads at a time: dS to smem; this slot's dW partial sums stay in TMEM
 #pragma unroll 1
@@ -679,17 +678,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                         wv[h] = w4.x; wv[h + 1] = w4.y; wv[h + 2] = w4.z; wv[h + 3] = w4.w;
                     }
                     tmem_wait_ld();
-                    uint8_t *dsc = dsb + c * 128;
-                    uint32_t m16 = 0;
+                    uint32_t m16 = 0, pk[8];
 #pragma unroll
-                    for (int h = 0; h < 16; ++h) {
-                        const float sval = sv[h];
-                        const float a0 = it.first ? 0.f : acc[h];
-                        acc[h] = fmaf(dI, fmaxf(sval, 0.f), a0);
-                        const float dsv = sval > 0.f ? dI * wv[h] : 0.f;
-                        if (kRec) m16 |= (sval > 0.f ? 1u : 0u) << h;
-                        *reinterpret_cast<uint16_t *>(dsc + sw128(h, jj)) = to_bits16<T>(dsv);
+                    for (int h = 0; h < 16; h += 2) {
+                        const float s0 = sv[h], s1 = sv[h + 1];
+                        acc[h] = fmaf(dI, fmaxf(s0, 0.f), it.first ? 0.f : acc[h]);
+                        acc[h + 1] = fmaf(dI, fmaxf(s1, 0.f), it.first ? 0.f : acc[h + 1]);
+                        pk[h >> 1] = pack2<T>(s0 > 0.f ? dI * wv[h] : 0.f, s1 > 0.f ? dI * wv[h + 1] : 0.f);
+                        if (kRec) m16 |= (s0 > 0.f ? 1u : 0u) << h | (s1 > 0.f ? 2u : 0u) << h;
                     }
+                    const int c8 = c >> 3;          // 16-byte chunk of heads c .. c + 7
+                    *reinterpret_cast<uint4 *>(dsrow + (((c8 ^ lrow) & 7) << 4)) =
+                        make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    *reinterpret_cast<uint4 *>(dsrow + ((((c8 + 1) ^ lrow) & 7) << 4)) =
+                        make_uint4(pk[4], pk[5], pk[6], pk[7]);
                     if (kRec) smask |= (uint64_t)m16 << c;
                     tmem_st16(dwa + c, acc);
                 }

@@ -15,7 +15,8 @@
 // and two for the key-major dK path:
 //   km_units       one warp per unit (32 query rows of a batch x one 256-key block pair):
 //                  which of the 32 rows name a key of the pair
-//   km_split       one block: cost-balanced contiguous unit ranges, one per worker
+//   km_split       one block: drops the empty units, then cost-balanced contiguous ranges of
+//                  the rest, one per worker
 #include "slikl_common.cuh"
 
 namespace slikl {
@@ -266,9 +267,20 @@ __global__ void km_units(Params P) {
 }
 
 __global__ void km_split(Params P, int workers) {
-    const int64_t n = P.unit_off[P.B];
-    // cost of a unit: a small fixed part plus its token count
-    block_prefix(n, [&](int64_t u) -> int64_t { return 1 + 8 * __popc((uint32_t)P.units[u].w); },
+    const int64_t n_all = P.unit_off[P.B];
+    // keep the units that hold at least one row (their order is kept)
+    block_prefix(n_all, [&](int64_t u) -> int64_t { return P.units[u].w != 0 ? 1 : 0; },
+                 P.unit_prefix);
+    __threadfence_block();
+    for (int64_t u = threadIdx.x; u < n_all; u += blockDim.x) {
+        const int4 x = P.units[u];
+        if (x.w != 0) P.units_c[P.unit_prefix[u]] = x;
+    }
+    const int64_t n = P.unit_prefix[n_all];
+    __syncthreads();
+    __threadfence_block();
+    // cost of a unit: a small fixed part plus its row count
+    block_prefix(n, [&](int64_t u) -> int64_t { return 1 + 8 * __popc((uint32_t)P.units_c[u].w); },
                  P.unit_prefix);
     __threadfence_block();
     const int64_t C = P.unit_prefix[n];

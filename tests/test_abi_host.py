@@ -144,3 +144,52 @@ def test_metadata_size_and_strings(lib):
     n = ctypes.c_size_t(0)
     assert lib.slikl_grad_metadata_workspace_size(ctypes.byref(pr), ctypes.byref(n)) == 0
     assert 0 < n.value < 4096 * 128 * 4 + 4096 * 64
+
+
+def dk_path(lib, pr, path=None):
+    v = ctypes.c_int32(-1)
+    opt = sli.make_options(path) if path is not None else None
+    rc = lib.slikl_grad_dk_path(ctypes.byref(pr), ctypes.byref(opt) if opt is not None else None,
+                                ctypes.byref(v))
+    return rc, v.value
+
+
+def ws_ex(lib, pr, path):
+    n = ctypes.c_size_t(0)
+    opt = sli.make_options(path)
+    rc = lib.slikl_grad_workspace_size_ex(ctypes.byref(pr), ctypes.byref(opt), ctypes.byref(n))
+    return rc, n.value
+
+
+def test_dk_path_choice(lib):
+    # key range (4096) within 16x topk: key-major on auto
+    assert dk_path(lib, base_problem()) == (sli.SLIKL_OK, sli.SLIKL_DK_KEYMAJOR)
+    assert dk_path(lib, base_problem(), "scatter") == (sli.SLIKL_OK, sli.SLIKL_DK_SCATTER)
+    # deterministic mode, long key ranges, N1 > 64: scatter on auto, key-major refused
+    for kw in (dict(deterministic=1), dict(S2=131072), dict(N1=128), dict(S2=20000, topk=4096)):
+        assert dk_path(lib, base_problem(**kw)) == (sli.SLIKL_OK, sli.SLIKL_DK_SCATTER), kw
+        assert dk_path(lib, base_problem(**kw), "keymajor")[0] == sli.SLIKL_ERR_PARAM_INVALID, kw
+    # key range above 16x topk: scatter on auto, key-major still possible on request
+    sparse = base_problem(S2=8192, topk=256)
+    assert dk_path(lib, sparse) == (sli.SLIKL_OK, sli.SLIKL_DK_SCATTER)
+    assert dk_path(lib, sparse, "keymajor") == (sli.SLIKL_OK, sli.SLIKL_DK_KEYMAJOR)
+    # TND keys: key-major only with a key-range bound in S2
+    tnd = dict(layout_q=sli.SLIKL_TND, layout_k=sli.SLIKL_TND, B=8, T1=35000, T2=35000, N1=32)
+    assert dk_path(lib, base_problem(S2=0, **tnd)) == (sli.SLIKL_OK, sli.SLIKL_DK_SCATTER)
+    assert dk_path(lib, base_problem(S2=8192, **tnd)) == (sli.SLIKL_OK, sli.SLIKL_DK_KEYMAJOR)
+    # unknown path value, NULL output
+    assert dk_path(lib, base_problem(), 7)[0] == sli.SLIKL_ERR_PARAM_INVALID
+    assert lib.slikl_grad_dk_path(ctypes.byref(base_problem()), None, None) == sli.SLIKL_ERR_INNER_NULLPTR
+
+
+def test_keymajor_workspace_holds_the_records(lib):
+    pr = base_problem()                        # T1 = 4096, S2 = 4096, N1 = 64: 16-byte records
+    rc_s, n_s = ws_ex(lib, pr, "scatter")
+    rc_k, n_k = ws_ex(lib, pr, "keymajor")
+    assert rc_s == rc_k == sli.SLIKL_OK
+    assert n_k - n_s >= 4096 * 4096 * 16
+    pr32 = base_problem(N1=32, S2=1000)        # 8-byte records, rows rounded up to 1024 keys
+    rc, n32 = ws_ex(lib, pr32, "keymajor")
+    assert rc == sli.SLIKL_OK and n32 - ws_ex(lib, pr32, "scatter")[1] >= 4096 * 1024 * 8
+    # the plain size call is the auto path
+    assert ws_rc(lib, pr)[1] == n_k
