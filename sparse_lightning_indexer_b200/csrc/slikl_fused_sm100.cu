@@ -7,29 +7,32 @@
 //   after the last pass-A tile: max and sum combined over the token.
 //   pass B  K rows gathered again; S^T recomputed; y = e^(I-m)/Z -> softmax_out, dI = y - p,
 //           dW_h += dI ReLU(S_h) (fp32), dS = dI * w * 1[S > 0] -> bf16/fp16 smem tile;
-//           dq^T[D x N1] += K^T . dS^T and dK^T[D x 128 keys] = q^T . dS (tcgen05);
-//           dK^T scattered into the fp32 key rows with red.global.add.f32, 32 consecutive d
-//           per warp instruction (one 128-byte line), or stored per slot (deterministic mode).
+//           dq^T[D x heads] += K^T . dS^T (tcgen05), and then one of
+//           - scatter mode: dK^T[D x 128 keys] = q^T . dS (tcgen05), scattered into the fp32
+//             key rows with red.global.add.f32, 32 consecutive d per warp instruction (one
+//             128-byte line), or stored per slot (deterministic mode);
+//           - record mode: a record per named (token, key) - the heads with S > 0 and dI -
+//             for the key-major dK kernel, after zero-filling the token's named 256-key block
+//             pairs during pass A.
 //   after the last pass-B tile: dW reduced in a fixed order, dq^T read back from TMEM.
 //
-// Schedule. The L2 fp32 reduction rate bounds this kernel, so the scatter must never
-// idle: all roles walk one deterministic item sequence in which pass A of the CTA's next
+// Schedule. All roles walk one deterministic item sequence in which pass A of the CTA's next
 // token alternates with pass B of the current one (phase k = B(t_{k-1}) interleaved with
 // A(t_k)). Every item gathers one K tile and computes one S tile.
 //
-// Warp roles (384 threads, 168 registers each):
-//   warps 0-2   producers: each warp gathers a third of the rows of every tile with cp.async
+// Warp roles (384 threads):
+//   warps 0-2   producers: each gathers its share of the rows of every tile with cp.async
 //               (16-byte chunks of the 256-byte key rows, zero-fill for invalid slots);
-//               warp 0 also loads q.
+//               warp 0 also loads q by TMA. In record mode warps 4-7 are producers too.
 //   warp 3      MMA issuer (one thread) and TMEM owner; the S product runs one item ahead.
-//   warps 4-7   scatter group: dK^T tiles from TMEM to the fp32 key rows.
-//   warps 8-11  softmax group: pass-A and pass-B epilogues, dW, dq readback.
-// The two 4-warp groups each cover the four TMEM lane quadrants (warp id % 4).
+//   warps 4-7   scatter group (scatter mode): dK^T tiles from TMEM to the fp32 key rows.
+//   warps 8-11  softmax group: pass-A and pass-B epilogues, records, dW, dq readback.
+// The 4-warp groups each cover the four TMEM lane quadrants (warp id % 4).
 //
-// Shared-memory tiles use the 128-byte swizzle in 8-row atoms, so one K tile serves as the
-// K-major A operand of the S product and as the MN-major A operand of the dq product; the q
-// tile is K-major B for S and MN-major A for dK; the dS tile [heads x keys] is K-major B for
-// dq and MN-major B for dK.
+// Shared-memory tiles use the 128-byte swizzle in 8-row atoms: the K tile is the K-major A
+// operand of the S product and the MN-major A operand of the dq product; the q tile is
+// K-major B for S and MN-major A for dK; the dS tile [keys x heads] is MN-major B for dq and
+// K-major B for dK.
 //
 // Every wait on an mbarrier is bounded (about one second of SM clock); on expiry the CTA
 // sets SLIKL_DEV_WAIT_TIMEOUT, every role stops, in-flight copies and MMAs are drained, TMEM
