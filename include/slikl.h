@@ -167,6 +167,10 @@ typedef struct {
                             fused kernel (key-major kernel and cast, the cast alone, or the
                             deterministic reduction), or NULL */
     void *dk_end;        /* optional cudaEvent_t recorded after that stage, or NULL */
+    float *loss;         /* optional DEVICE output, fp32 [T1] (4-byte aligned), or NULL: the KL
+                            loss per query row, L_t = sum over valid slots with p > 0 of
+                            p log(p / y) (section "计算公式"), from the softmax_out of this
+                            call; 0 for a row without a valid slot */
 } slikl_options;
 
 /*

@@ -68,18 +68,20 @@ class slikl_tensors(ctypes.Structure):
 class slikl_options(ctypes.Structure):
     _fields_ = [("dk_path", ctypes.c_int32), ("fused_begin", ctypes.c_void_p),
                 ("fused_end", ctypes.c_void_p), ("dk_begin", ctypes.c_void_p),
-                ("dk_end", ctypes.c_void_p)]
+                ("dk_end", ctypes.c_void_p), ("loss", ctypes.c_void_p)]
 
 
 def make_options(dk_path="auto", fused_begin: int = 0, fused_end: int = 0, dk_begin: int = 0,
-                 dk_end: int = 0) -> slikl_options:
-    """Options of slikl_grad_ex; the event arguments are cudaEvent_t handles (ints) or 0."""
+                 dk_end: int = 0, loss: int = 0) -> slikl_options:
+    """Options of slikl_grad_ex; the event arguments are cudaEvent_t handles (ints) or 0;
+    `loss` is the device address of an fp32 [T1] output for the per-row KL loss, or 0."""
     o = slikl_options()
     o.dk_path = _DK_PATHS[dk_path] if isinstance(dk_path, str) else int(dk_path)
     o.fused_begin = fused_begin or None
     o.fused_end = fused_end or None
     o.dk_begin = dk_begin or None
     o.dk_end = dk_end or None
+    o.loss = loss or None
     return o
 
 
@@ -276,11 +278,12 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
 
 def grad(q, k, w, attn_softmax_l1norm, sparse_indices, layout_q="BSND", layout_k="BSND",
          cu_seqlens_q=None, cu_seqlens_k=None, deterministic=False, stream=None, out=None,
-         workspace=None, dk_path="auto", key_range_bound=0):
+         workspace=None, dk_path="auto", key_range_bound=0, loss=False):
     """Run slikl_grad_ex on CUDA tensors. Returns dict(dq, dk, dw, softmax_out, workspace).
 
     `out` may supply preallocated dq/dk/dw/softmax_out, `workspace` a uint8 CUDA buffer;
-    `dk_path` is "auto", "scatter" or "keymajor"; `key_range_bound` as in make_problem.
+    `dk_path` is "auto", "scatter" or "keymajor"; `key_range_bound` as in make_problem;
+    `loss=True` also returns the per-row KL loss (fp32 [T1]) as res["loss"].
     """
     B = None
     if layout_q == "TND":
@@ -289,7 +292,8 @@ def grad(q, k, w, attn_softmax_l1norm, sparse_indices, layout_q="BSND", layout_k
         B = cu_seqlens_k.numel() - 1
     pr = make_problem(q, k, sparse_indices, layout_q, layout_k, deterministic, B,
                       key_range_bound)
-    opt = make_options(dk_path)
+    loss_t = torch.empty(pr.T1, dtype=torch.float32, device=q.device) if loss else None
+    opt = make_options(dk_path, loss=loss_t.data_ptr() if loss_t is not None else 0)
     nbytes = slikl_grad_workspace_size_ex(pr, opt)
     if workspace is None or workspace.numel() < nbytes:
         workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device)
@@ -308,6 +312,8 @@ def grad(q, k, w, attn_softmax_l1norm, sparse_indices, layout_q="BSND", layout_k
     slikl_grad_ex(pr, tn, workspace.data_ptr(), workspace.numel(), s.cuda_stream, opt)
     res = dict(out)
     res["workspace"] = workspace
+    if loss_t is not None:
+        res["loss"] = loss_t
     return res
 
 
@@ -319,7 +325,8 @@ def key_range_bound_of(wl) -> int:
     return max((c[i + 1] - c[i] for i in range(len(c) - 1)), default=0)
 
 
-def grad_workload(wl, device="cuda", deterministic=False, stream=None, dk_path="auto"):
+def grad_workload(wl, device="cuda", deterministic=False, stream=None, dk_path="auto",
+                  loss=False):
     """Move a slikl_inputs.Workload to the device and run grad()."""
     dev = torch.device(device)
     t = {n: getattr(wl, n).to(dev) for n in ("q", "k", "w", "p", "idx")}
@@ -327,4 +334,4 @@ def grad_workload(wl, device="cuda", deterministic=False, stream=None, dk_path="
     cuk = wl.cu_seqlens_k.to(dev) if wl.cu_seqlens_k is not None else None
     return grad(t["q"], t["k"], t["w"], t["p"], t["idx"], wl.layout, wl.layout, cuq, cuk,
                 deterministic=deterministic, stream=stream, dk_path=dk_path,
-                key_range_bound=key_range_bound_of(wl))
+                key_range_bound=key_range_bound_of(wl), loss=loss)

@@ -10,6 +10,9 @@
 
 namespace slikl {
 
+// per-row KL loss output (slikl_loss.cu)
+cudaError_t launch_kl_loss(const Params &P, float *loss, cudaStream_t s);
+
 namespace {
 
 struct Derived {
@@ -235,6 +238,8 @@ slikl_status slikl_grad_ex(const slikl_problem *problem, const slikl_tensors *te
     if (st != SLIKL_OK) return st;
     st = check_tensors(problem, tensors, true);
     if (st != SLIKL_OK) return st;
+    if (options && options->loss && (reinterpret_cast<uintptr_t>(options->loss) & 3))
+        return SLIKL_ERR_PARAM_INVALID;
     if (!workspace) return SLIKL_ERR_PARAM_NULLPTR;
     if (reinterpret_cast<uintptr_t>(workspace) & 255) return SLIKL_ERR_PARAM_INVALID;
     WsLayout L = make_layout(dv.T1, dv.T2, problem->topk, problem->D, problem->deterministic,
@@ -264,6 +269,8 @@ slikl_status slikl_grad_ex(const slikl_problem *problem, const slikl_tensors *te
         if (P.km && !handled) return SLIKL_ERR_CUDA;   // key-major records need the sm100 kernel
     }
     if (fused_end && cudaEventRecord(static_cast<cudaEvent_t>(fused_end), s) != cudaSuccess)
+        return SLIKL_ERR_CUDA;
+    if (options && options->loss && launch_kl_loss(P, options->loss, s) != cudaSuccess)
         return SLIKL_ERR_CUDA;
     void *dk_begin = options ? options->dk_begin : nullptr;
     void *dk_end = options ? options->dk_end : nullptr;

@@ -336,3 +336,33 @@ def test_metadata_golden_sample_shapes():
                       D=128, K=4)
         m = metadata_gpu(wl, case["cores"], 0)
         assert list(m[:6]) == case["header"]
+
+
+@pytest.mark.parametrize("case", [SMALL[0], SMALL[1], SMALL[7], SMALL[8], SMALL[9], SMALL[10]],
+                         ids=lambda c: f"s{c['seed']}")
+@pytest.mark.parametrize("path", ["scatter", "keymajor"])
+def test_kl_loss_output(case, path):
+    """The optional per-row KL loss output against the oracle's L_t (rel-L2 <= 1e-5, rows
+    without a valid slot exactly 0), on the dK paths that can run the case."""
+    if path == "keymajor" and not keymajor_possible(case):
+        pytest.skip("key-major dK path needs N1 <= 64")
+    wl = si.small(**case)
+    ref = oracle.grad(wl)
+    res = sli.grad_workload(wl, dk_path=path, loss=True)
+    torch.cuda.synchronize()
+    got = res["loss"].double().cpu().numpy()
+    assert got.shape == ref["loss"].shape
+    assert np.all(np.isfinite(got))
+    e = rel_l2(got, ref["loss"])
+    assert e <= 1e-5, f"loss rel-L2 {e:.3e}"
+    idx = wl.idx.numpy().reshape(wl.T1, wl.K)
+    empty = ~(idx >= 0).any(axis=1)
+    assert np.all(got[empty] == 0.0)
+
+
+def test_kl_loss_output_config0():
+    wl = si.config(0)
+    ref = oracle.grad(wl)
+    res = sli.grad_workload(wl, loss=True)
+    torch.cuda.synchronize()
+    assert rel_l2(res["loss"].double().cpu().numpy(), ref["loss"]) <= 1e-5
