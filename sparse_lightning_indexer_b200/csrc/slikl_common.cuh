@@ -133,12 +133,6 @@ __device__ __forceinline__ void red_add_f32(float *addr, float v) {
     asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
 }
 
-__device__ __forceinline__ void red_add_v4_f32(float *addr, float a, float b, float c, float d) {
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
-                 "f"(c), "f"(d)
-                 : "memory");
-}
-
 // Key row of slot value v for a token whose batch keys are [kbase, kbase + klen), or -1.
 // Values outside [-1, klen) break the index contract: they are flagged and treated as invalid.
 __device__ __forceinline__ int32_t slot_row(int32_t v, int32_t kbase, int32_t klen,

@@ -51,9 +51,6 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32
                  "r"(src_bytes)
                  : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() {
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
@@ -135,15 +132,7 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                  ::"r"(smem_u32(bar)), "r"(bytes)
                  : "memory");
 }
-// Tiled TMA load of a box at (x, y[, z]) into shared memory, completing on `bar` (no multicast).
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
-                                            uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
-        "[%0], [%1, {%2, %3}], [%4];"
-        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-        : "memory");
-}
+// Tiled TMA load of a box at (x, y, z) into shared memory, completing on `bar` (no multicast).
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int x, int y,
                                             int z, uint64_t *bar) {
     asm volatile(
@@ -188,16 +177,6 @@ __device__ __forceinline__ bool group_sync(uint64_t *bar, uint32_t &phase, volat
     return ok;
 }
 
-template <typename T>
-__device__ __forceinline__ uint16_t to_bits16(float v);
-template <>
-__device__ __forceinline__ uint16_t to_bits16<__nv_bfloat16>(float v) {
-    return __bfloat16_as_ushort(__float2bfloat16_rn(v));
-}
-template <>
-__device__ __forceinline__ uint16_t to_bits16<__half>(float v) {
-    return __half_as_ushort(__float2half_rn(v));
-}
 
 
 // Two floats rounded to the 16-bit type, packed low / high.

@@ -193,3 +193,48 @@ def test_keymajor_workspace_holds_the_records(lib):
     assert rc == sli.SLIKL_OK and n32 - ws_ex(lib, pr32, "scatter")[1] >= 4096 * 1024 * 8
     # the plain size call is the auto path
     assert ws_rc(lib, pr)[1] == n_k
+
+
+def grad_ex_rc(lib, pr, tn, ws, nbytes, opt):
+    return lib.slikl_grad_ex(ctypes.byref(pr), ctypes.byref(tn), ctypes.c_void_p(ws), nbytes, None,
+                             ctypes.byref(opt) if opt is not None else None)
+
+
+def test_grad_ex_host_validation(lib):
+    """slikl_grad_ex checks everything the host can see before any CUDA call."""
+    pr = base_problem()
+    tn = fake_tensors()
+    _, need_auto = ws_ex(lib, pr, "auto")
+    _, need_scatter = ws_ex(lib, pr, "scatter")
+    assert need_auto > need_scatter                   # auto is key-major here: records
+    # the workspace must be sized for the path the options select
+    assert grad_ex_rc(lib, pr, tn, 1 << 20, need_scatter, sli.make_options("auto")) == \
+        sli.SLIKL_ERR_WORKSPACE_TOO_SMALL
+    assert grad_ex_rc(lib, pr, tn, 1 << 20, need_auto - 1, None) == sli.SLIKL_ERR_WORKSPACE_TOO_SMALL
+    # unknown path, key-major on a problem it cannot run
+    assert grad_ex_rc(lib, pr, tn, 1 << 20, need_auto, sli.make_options(5)) == \
+        sli.SLIKL_ERR_PARAM_INVALID
+    assert grad_ex_rc(lib, base_problem(N1=128), tn, 1 << 20, 1 << 40,
+                      sli.make_options("keymajor")) == sli.SLIKL_ERR_PARAM_INVALID
+    # loss output must be 4-byte aligned
+    assert grad_ex_rc(lib, pr, tn, 1 << 20, need_auto, sli.make_options(loss=0x1002)) == \
+        sli.SLIKL_ERR_PARAM_INVALID
+    # NULL tensors / workspace
+    assert lib.slikl_grad_ex(ctypes.byref(pr), None, None, 0, None, None) == sli.SLIKL_ERR_PARAM_NULLPTR
+    assert grad_ex_rc(lib, pr, tn, 0, need_auto, None) == sli.SLIKL_ERR_PARAM_NULLPTR
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device error path")
+def test_grad_ex_no_device_is_an_error(lib):
+    pr = base_problem()
+    tn = fake_tensors()
+    for path in ("auto", "scatter", "keymajor"):
+        _, need = ws_ex(lib, pr, path)
+        assert grad_ex_rc(lib, pr, tn, 1 << 20, need, sli.make_options(path)) == sli.SLIKL_ERR_CUDA
+
+
+def test_options_struct_layout():
+    """The ctypes mirror of slikl_options matches the header's field order and pointer sizes."""
+    names = [n for n, _ in sli.slikl_options._fields_]
+    assert names == ["dk_path", "fused_begin", "fused_end", "dk_begin", "dk_end", "loss"]
+    assert ctypes.sizeof(sli.slikl_options) == 8 + 5 * ctypes.sizeof(ctypes.c_void_p)
