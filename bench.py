@@ -147,11 +147,10 @@ def raw_elapsed_ms(a, b):
 
 # DRAM bytes (read + write) of one fused-kernel launch on the headline workload, from the ncu
 # capture summarised in profiles/fused_sm100_causal4096_n64_k2048.md, valid only while the
-# kernel's sources stay as they are (hash of the three files below; the capture was taken before
-# unused helpers were removed from the two headers, which does not change the kernel);
-# otherwise the traffic is reported as unknown.
-FUSED_TRAFFIC = {"sources_sha256_16": "046399581925f681", "workload_config": 1,
-                 "dk_path": "keymajor", "bytes": 120.863232e6 + 195.345664e6}
+# kernel's sources stay as they are (hash of the three files below); otherwise the traffic is
+# reported as unknown.
+FUSED_TRAFFIC = {"sources_sha256_16": "ad35ef942028f8db", "workload_config": 1,
+                 "dk_path": "keymajor", "bytes": 120.872448e6 + 193.860096e6}
 
 
 def fused_sources_hash():

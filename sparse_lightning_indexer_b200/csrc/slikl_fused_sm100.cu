@@ -86,7 +86,7 @@ __host__ __device__ inline SmemPlan plan_smem(int stages) {
     s.ds = take(2 * 128 * 128, 1024);                // two buffers [128 keys x 64 heads]
     s.w = take(2 * N1P * 4, 16);                     // w of two tokens
     s.rows = take(2 * kRowsStride * 4, 16);          // key rows of two dS tiles
-    s.red = take(4 * 64 * 4, 16);
+    s.red = take(2 * 4 * 64 * 4, 16);               // dW partials of two tokens
     s.ring = take(7 * 4 * kRingSlot * 4, 16);       // up to 7 producer warps
     s.bar = take(sizeof(Barriers) + 16, 8);
     s.total = off + 1024;                            // slack for aligning the dynamic base
@@ -516,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int et = threadIdx.x - 256;        // 0..127
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
         float *wsm = reinterpret_cast<float *>(smem + SP.w);      // [2][N1P]
-        float *red = reinterpret_cast<float *>(smem + SP.red);    // [4][64]
+        float *red = reinterpret_cast<float *>(smem + SP.red);    // [2][4][64]
         uint8_t *ds_tiles = smem + SP.ds;
         uint32_t gk = 0, gd = 0, nb = 0, ph = 0;
         bool ok = true;
@@ -762,12 +762,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                         span >>= 1;
                         if (lane & o) base += span;
                     }
+                    // dW partials in buffer ord % 2: a warp may reach the next token's write
+                    // before the others have read this one (nothing in between waits on them);
+                    // it writes this buffer again two tokens on, after the next token's group
+                    // sync, which every warp reaches only after its reads below
+                    float *rd = red + (it.ord & 1) * 256;
 #pragma unroll
-                    for (int h = 0; h < kV / 32; ++h) red[ew * 64 + base + h] = vv[h];
+                    for (int h = 0; h < kV / 32; ++h) rd[ew * 64 + base + h] = vv[h];
                     if (!group_sync(&bars->sm_sync, ph, &ctl.abort, P.status)) { ok = false; break; }
                     for (int h = et; h < P.N1; h += 128) {
                         float a = 0.f;
-                        for (int i = 0; i < 4; ++i) a += red[i * 64 + h];
+                        for (int i = 0; i < 4; ++i) a += rd[i * 64 + h];
                         P.dw[(int64_t)it.t * P.N1 + h] = a;
                     }
                     // dq^T readback (lane = d): columns = heads
@@ -791,7 +796,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bars->dq_empty);
                     ++nb;
-                    // red is rewritten only after the next token's group syncs
                 }
             }
             ++gk;
