@@ -171,6 +171,19 @@ typedef struct {
                             loss per query row, L_t = sum over valid slots with p > 0 of
                             p log(p / y) (section "计算公式"), from the softmax_out of this
                             call; 0 for a row without a valid slot */
+    const int32_t *seq_used_q;  /* optional DEVICE input, int32 [B] (4-byte aligned), or NULL:
+                            the query rows of batch b in use (seqUsedQOptional of
+                            aclnnSparseLightningIndexerKLLossGrad; the page fixes only its
+                            type). Rows of batch b at local position >= seq_used_q[b] are
+                            padding: their indices are not read, softmax_out / dq / dw are 0
+                            there and they add nothing to dk. NULL = every row in use. */
+    const int32_t *seq_used_k;  /* optional DEVICE input, int32 [B] (4-byte aligned), or NULL:
+                            the key rows of batch b in use (seqUsedKOptional). A slot naming a
+                            key at local position >= seq_used_k[b] (and < the batch's key
+                            count) is invalid, like -1, without a status flag; dk rows of
+                            unused keys stay 0. NULL = every key in use.
+                            A value outside [0, the batch's row count] sets
+                            SLIKL_DEV_BAD_SEQ_USED and is clamped into that range. */
 } slikl_options;
 
 /*
@@ -207,7 +220,8 @@ SLIKL_API slikl_status slikl_grad_with_events(const slikl_problem *problem,
                                               void *fused_begin, void *fused_end);
 
 /* Device status bits (see slikl_read_device_status). */
-#define SLIKL_DEV_INDEX_OUT_OF_RANGE  0x1u  /* some valid-looking index was >= len_k(b) or < -1 */
+#define SLIKL_DEV_INDEX_OUT_OF_RANGE  0x1u  /* an index of a row in use was >= len_k(b) or < -1
+                                               (len_k(b): the batch's key count, used or not) */
 #define SLIKL_DEV_BAD_CU_SEQLENS_Q    0x2u  /* cu_seqlens_q not 0..T1 non-decreasing           */
 #define SLIKL_DEV_BAD_CU_SEQLENS_K    0x4u  /* cu_seqlens_k not 0..T2 non-decreasing; the key
                                                ranges of the batches were emptied            */
@@ -215,6 +229,8 @@ SLIKL_API slikl_status slikl_grad_with_events(const slikl_problem *problem,
 #define SLIKL_DEV_KEY_RANGE_ABOVE_S2  0x10u /* key-major dK path: a batch holds more key rows
                                                than problem->S2 promised (TND); the rows of
                                                that batch are left out, outputs invalid    */
+#define SLIKL_DEV_BAD_SEQ_USED        0x20u /* a seq_used_q / seq_used_k entry was outside
+                                               [0, the batch's row count]; it was clamped  */
 
 /*
  * Copies the status word of the last slikl_grad call that used `workspace` (device) into

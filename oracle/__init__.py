@@ -50,7 +50,9 @@ class _Problem(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int64), ("T1", ctypes.c_int64), ("T2", ctypes.c_int64),
                 ("N1", ctypes.c_int64), ("D", ctypes.c_int64), ("K", ctypes.c_int64),
                 ("q_start", ctypes.POINTER(ctypes.c_int64)),
-                ("k_start", ctypes.POINTER(ctypes.c_int64))]
+                ("k_start", ctypes.POINTER(ctypes.c_int64)),
+                ("q_used", ctypes.POINTER(ctypes.c_int64)),
+                ("k_used", ctypes.POINTER(ctypes.c_int64))]
 
 
 def _load():
@@ -98,10 +100,13 @@ def row_starts(layout_q: str, layout_k: str, B: int, S1: int, S2: int,
 
 def grad_arrays(q: np.ndarray, k: np.ndarray, w: np.ndarray, p: np.ndarray, idx: np.ndarray,
                 q_start: np.ndarray, k_start: np.ndarray, tokens: Optional[np.ndarray] = None,
-                nthreads: int = 0) -> dict:
+                nthreads: int = 0, q_used: Optional[Sequence[int]] = None,
+                k_used: Optional[Sequence[int]] = None) -> dict:
     """Oracle on flat fp64 arrays.
 
-    q [T1,N1,D], k [T2,D], w [T1,N1], p [T1,K], idx [T1,K] int32, q_start/k_start [B+1].
+    q [T1,N1,D], k [T2,D], w [T1,N1], p [T1,K], idx [T1,K] int32, q_start/k_start [B+1];
+    q_used / k_used: optional [B] rows of each batch in use (seqUsedQ / seqUsedK reading:
+    query rows past q_used[b] are padding, keys past k_used[b] are invalid slots).
     Returns fp64 y [T1,K], dw [T1,N1], dq [T1,N1,D], dk [T2,D], loss [T1].
     """
     q = np.ascontiguousarray(q, dtype=np.float64)
@@ -117,7 +122,12 @@ def grad_arrays(q: np.ndarray, k: np.ndarray, w: np.ndarray, p: np.ndarray, idx:
     qs = np.ascontiguousarray(q_start, dtype=np.int64)
     ks = np.ascontiguousarray(k_start, dtype=np.int64)
     B = qs.size - 1
-    prob = _Problem(B, T1, T2, N1, D, K, _ptr(qs, ctypes.c_int64), _ptr(ks, ctypes.c_int64))
+    qu = None if q_used is None else np.ascontiguousarray(q_used, dtype=np.int64)
+    ku = None if k_used is None else np.ascontiguousarray(k_used, dtype=np.int64)
+    if (qu is not None and qu.shape != (B,)) or (ku is not None and ku.shape != (B,)):
+        raise ValueError("q_used / k_used must have B entries")
+    prob = _Problem(B, T1, T2, N1, D, K, _ptr(qs, ctypes.c_int64), _ptr(ks, ctypes.c_int64),
+                    _ptr(qu, ctypes.c_int64), _ptr(ku, ctypes.c_int64))
     y = np.zeros((T1, K))
     dw = np.zeros((T1, N1))
     dq = np.zeros((T1, N1, D))
@@ -132,13 +142,16 @@ def grad_arrays(q: np.ndarray, k: np.ndarray, w: np.ndarray, p: np.ndarray, idx:
                              _ptr(dq, ctypes.c_double), _ptr(dk, ctypes.c_double),
                              _ptr(loss, ctypes.c_double))
     if rc != 0:
-        raise ValueError({1: "bad shape", 2: "index outside its batch's key range",
+        raise ValueError({1: "bad shape or used length", 2: "index outside its batch's key range",
                           3: "out of memory"}.get(rc, f"oracle error {rc}"))
     return {"y": y, "dw": dw, "dq": dq, "dk": dk, "loss": loss}
 
 
-def grad(wl, tokens: Optional[np.ndarray] = None, nthreads: int = 0) -> dict:
-    """Oracle on a slikl_inputs.Workload (inputs converted exactly from their dtypes)."""
+def grad(wl, tokens: Optional[np.ndarray] = None, nthreads: int = 0,
+         seq_used_q: Optional[Sequence[int]] = None,
+         seq_used_k: Optional[Sequence[int]] = None) -> dict:
+    """Oracle on a slikl_inputs.Workload (inputs converted exactly from their dtypes);
+    seq_used_q / seq_used_k as q_used / k_used of grad_arrays."""
     T1, T2, N1, D, K = wl.T1, wl.T2, wl.N1, wl.D, wl.K
     q = wl.q.double().numpy().reshape(T1, N1, D)
     k = wl.k.double().numpy().reshape(T2, D)
@@ -148,7 +161,8 @@ def grad(wl, tokens: Optional[np.ndarray] = None, nthreads: int = 0) -> dict:
     cuq = None if wl.cu_seqlens_q is None else wl.cu_seqlens_q.numpy()
     cuk = None if wl.cu_seqlens_k is None else wl.cu_seqlens_k.numpy()
     qs, ks = row_starts(wl.layout, wl.layout, wl.B, wl.S1, wl.S2, cuq, cuk)
-    return grad_arrays(q, k, w, p, idx, qs, ks, tokens=tokens, nthreads=nthreads)
+    return grad_arrays(q, k, w, p, idx, qs, ks, tokens=tokens, nthreads=nthreads,
+                       q_used=seq_used_q, k_used=seq_used_k)
 
 
 def split_equal(total: int, cores: int, max_seq_k: int):

@@ -26,6 +26,12 @@
  * The KL loss of the same section, L_t = sum_{valid j} p_j log(p_j / y_j) (with
  * 0 log 0 = 0), is returned per token for finite-difference checks.
  *
+ * Used lengths (seqUsedQOptional / seqUsedKOptional of the same page, which fixes only
+ * their type; read here as the rows of each batch in use): when given, query rows of
+ * batch b at local position >= q_used[b] are padding (their indices are not read, all
+ * their outputs are 0, they add nothing to dk) and a slot naming a key at local position
+ * >= k_used[b] is invalid like -1.
+ *
  * Everything is fp64. Tokens are independent and run in parallel (OpenMP); dk is
  * accumulated key row by key row, each row summing its references in ascending
  * (token, slot) order, so the result does not depend on the thread count.
@@ -44,6 +50,8 @@ typedef struct {
     int64_t N1, D, K;         /* query heads, head dim, top-k */
     const int64_t *q_start;   /* [B+1] first query row of each batch (q_start[B] = T1) */
     const int64_t *k_start;   /* [B+1] first key row of each batch (k_start[B] = T2) */
+    const int64_t *q_used;    /* [B] query rows of each batch in use, or NULL (all) */
+    const int64_t *k_used;    /* [B] key rows of each batch in use, or NULL (all) */
 } oracle_problem;
 
 enum { ORACLE_OK = 0, ORACLE_BAD_SHAPE = 1, ORACLE_BAD_INDEX = 2, ORACLE_NO_MEMORY = 3 };
@@ -55,16 +63,28 @@ static int64_t batch_of(const oracle_problem *pr, int64_t t) {
     return pr->B - 1;
 }
 
-/* Key row of slot j of query row t, or -1 when the slot is invalid. */
-static int64_t key_row(const oracle_problem *pr, const int32_t *idx, int64_t t, int64_t j) {
-    int32_t v = idx[t * pr->K + j];
-    if (v < 0) return -1;
-    return pr->k_start[batch_of(pr, t)] + v;
+/* Is query row t in use (not a padding row past q_used of its batch)? */
+static int row_in_use(const oracle_problem *pr, int64_t t) {
+    if (!pr->q_used) return 1;
+    int64_t b = batch_of(pr, t);
+    return t - pr->q_start[b] < pr->q_used[b];
 }
 
-/* Check the index contract: -1 or inside the batch's key range. */
+/* Key row of slot j of query row t, or -1 when the slot is invalid (index -1, a key past
+ * k_used of the batch, or any slot of a padding row). */
+static int64_t key_row(const oracle_problem *pr, const int32_t *idx, int64_t t, int64_t j) {
+    if (!row_in_use(pr, t)) return -1;
+    int32_t v = idx[t * pr->K + j];
+    if (v < 0) return -1;
+    int64_t b = batch_of(pr, t);
+    if (pr->k_used && v >= pr->k_used[b]) return -1;
+    return pr->k_start[b] + v;
+}
+
+/* Check the index contract on the rows in use: -1 or inside the batch's key range. */
 int oracle_check_indices(const oracle_problem *pr, const int32_t *idx) {
     for (int64_t t = 0; t < pr->T1; ++t) {
+        if (!row_in_use(pr, t)) continue;
         int64_t b = batch_of(pr, t);
         int64_t klen = pr->k_start[b + 1] - pr->k_start[b];
         for (int64_t j = 0; j < pr->K; ++j) {
@@ -125,10 +145,10 @@ static void token_forward_backward(const oracle_problem *pr, const double *q, co
     /* y = Softmax(I) over the valid slots (max subtracted; identical in exact arithmetic) */
     double Z = 0.0;
     for (int64_t j = 0; j < K; ++j)
-        if (idx[t * K + j] >= 0) Z += exp(I[j] - m);
+        if (key_row(pr, idx, t, j) >= 0) Z += exp(I[j] - m);
     double L = 0.0;
     for (int64_t j = 0; j < K; ++j) {
-        if (idx[t * K + j] < 0) { yt[j] = 0.0; dIt[j] = 0.0; continue; }
+        if (key_row(pr, idx, t, j) < 0) { yt[j] = 0.0; dIt[j] = 0.0; continue; }
         yt[j] = exp(I[j] - m) / Z;
         dIt[j] = yt[j] - pt[j];                         /* dI = Softmax(I) - p */
         if (pt[j] > 0.0) L += pt[j] * log(pt[j] / yt[j]);
@@ -166,6 +186,14 @@ int oracle_grad(const oracle_problem *pr, const double *q, const double *k, cons
     if (pr->q_start[0] != 0 || pr->k_start[0] != 0 || pr->q_start[pr->B] != T1 ||
         pr->k_start[pr->B] != T2)
         return ORACLE_BAD_SHAPE;
+    for (int64_t b = 0; b < pr->B; ++b) {
+        if (pr->q_used && (pr->q_used[b] < 0 ||
+                           pr->q_used[b] > pr->q_start[b + 1] - pr->q_start[b]))
+            return ORACLE_BAD_SHAPE;
+        if (pr->k_used && (pr->k_used[b] < 0 ||
+                           pr->k_used[b] > pr->k_start[b + 1] - pr->k_start[b]))
+            return ORACLE_BAD_SHAPE;
+    }
     int rc = oracle_check_indices(pr, idx);
     if (rc != ORACLE_OK) return rc;
 

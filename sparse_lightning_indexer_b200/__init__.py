@@ -36,6 +36,7 @@ SLIKL_DEV_BAD_CU_SEQLENS_Q = 0x2
 SLIKL_DEV_BAD_CU_SEQLENS_K = 0x4
 SLIKL_DEV_WAIT_TIMEOUT = 0x8
 SLIKL_DEV_KEY_RANGE_ABOVE_S2 = 0x10
+SLIKL_DEV_BAD_SEQ_USED = 0x20
 
 SLIKL_DK_AUTO = 0
 SLIKL_DK_SCATTER = 1
@@ -68,13 +69,16 @@ class slikl_tensors(ctypes.Structure):
 class slikl_options(ctypes.Structure):
     _fields_ = [("dk_path", ctypes.c_int32), ("fused_begin", ctypes.c_void_p),
                 ("fused_end", ctypes.c_void_p), ("dk_begin", ctypes.c_void_p),
-                ("dk_end", ctypes.c_void_p), ("loss", ctypes.c_void_p)]
+                ("dk_end", ctypes.c_void_p), ("loss", ctypes.c_void_p),
+                ("seq_used_q", ctypes.c_void_p), ("seq_used_k", ctypes.c_void_p)]
 
 
 def make_options(dk_path="auto", fused_begin: int = 0, fused_end: int = 0, dk_begin: int = 0,
-                 dk_end: int = 0, loss: int = 0) -> slikl_options:
+                 dk_end: int = 0, loss: int = 0, seq_used_q: int = 0,
+                 seq_used_k: int = 0) -> slikl_options:
     """Options of slikl_grad_ex; the event arguments are cudaEvent_t handles (ints) or 0;
-    `loss` is the device address of an fp32 [T1] output for the per-row KL loss, or 0."""
+    `loss` is the device address of an fp32 [T1] output for the per-row KL loss, or 0;
+    `seq_used_q` / `seq_used_k` are device addresses of int32 [B] used lengths, or 0."""
     o = slikl_options()
     o.dk_path = _DK_PATHS[dk_path] if isinstance(dk_path, str) else int(dk_path)
     o.fused_begin = fused_begin or None
@@ -82,6 +86,8 @@ def make_options(dk_path="auto", fused_begin: int = 0, fused_end: int = 0, dk_be
     o.dk_begin = dk_begin or None
     o.dk_end = dk_end or None
     o.loss = loss or None
+    o.seq_used_q = seq_used_q or None
+    o.seq_used_k = seq_used_k or None
     return o
 
 
@@ -278,12 +284,15 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
 
 def grad(q, k, w, attn_softmax_l1norm, sparse_indices, layout_q="BSND", layout_k="BSND",
          cu_seqlens_q=None, cu_seqlens_k=None, deterministic=False, stream=None, out=None,
-         workspace=None, dk_path="auto", key_range_bound=0, loss=False):
+         workspace=None, dk_path="auto", key_range_bound=0, loss=False, seq_used_q=None,
+         seq_used_k=None):
     """Run slikl_grad_ex on CUDA tensors. Returns dict(dq, dk, dw, softmax_out, workspace).
 
     `out` may supply preallocated dq/dk/dw/softmax_out, `workspace` a uint8 CUDA buffer;
     `dk_path` is "auto", "scatter" or "keymajor"; `key_range_bound` as in make_problem;
-    `loss=True` also returns the per-row KL loss (fp32 [T1]) as res["loss"].
+    `loss=True` also returns the per-row KL loss (fp32 [T1]) as res["loss"];
+    `seq_used_q` / `seq_used_k` are optional int32 [B] CUDA tensors of the query / key rows of
+    each batch in use (rows past them are padding).
     """
     B = None
     if layout_q == "TND":
@@ -293,7 +302,12 @@ def grad(q, k, w, attn_softmax_l1norm, sparse_indices, layout_q="BSND", layout_k
     pr = make_problem(q, k, sparse_indices, layout_q, layout_k, deterministic, B,
                       key_range_bound)
     loss_t = torch.empty(pr.T1, dtype=torch.float32, device=q.device) if loss else None
-    opt = make_options(dk_path, loss=loss_t.data_ptr() if loss_t is not None else 0)
+    for name, u in (("seq_used_q", seq_used_q), ("seq_used_k", seq_used_k)):
+        if u is not None and (u.dtype != torch.int32 or not u.is_cuda or not u.is_contiguous()
+                              or u.numel() != pr.B):
+            raise ValueError(f"{name} must be a contiguous int32 CUDA tensor of B entries")
+    opt = make_options(dk_path, loss=loss_t.data_ptr() if loss_t is not None else 0,
+                       seq_used_q=_ptr(seq_used_q) or 0, seq_used_k=_ptr(seq_used_k) or 0)
     nbytes = slikl_grad_workspace_size_ex(pr, opt)
     if workspace is None or workspace.numel() < nbytes:
         workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device)
@@ -326,12 +340,16 @@ def key_range_bound_of(wl) -> int:
 
 
 def grad_workload(wl, device="cuda", deterministic=False, stream=None, dk_path="auto",
-                  loss=False):
-    """Move a slikl_inputs.Workload to the device and run grad()."""
+                  loss=False, seq_used_q=None, seq_used_k=None):
+    """Move a slikl_inputs.Workload to the device and run grad() (seq_used_q / seq_used_k:
+    optional host int sequences of B used lengths)."""
     dev = torch.device(device)
     t = {n: getattr(wl, n).to(dev) for n in ("q", "k", "w", "p", "idx")}
     cuq = wl.cu_seqlens_q.to(dev) if wl.cu_seqlens_q is not None else None
     cuk = wl.cu_seqlens_k.to(dev) if wl.cu_seqlens_k is not None else None
+    uq = None if seq_used_q is None else torch.tensor(list(seq_used_q), dtype=torch.int32, device=dev)
+    uk = None if seq_used_k is None else torch.tensor(list(seq_used_k), dtype=torch.int32, device=dev)
     return grad(t["q"], t["k"], t["w"], t["p"], t["idx"], wl.layout, wl.layout, cuq, cuk,
                 deterministic=deterministic, stream=stream, dk_path=dk_path,
-                key_range_bound=key_range_bound_of(wl), loss=loss)
+                key_range_bound=key_range_bound_of(wl), loss=loss, seq_used_q=uq,
+                seq_used_k=uk)

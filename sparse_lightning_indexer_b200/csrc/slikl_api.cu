@@ -238,7 +238,9 @@ slikl_status slikl_grad_ex(const slikl_problem *problem, const slikl_tensors *te
     if (st != SLIKL_OK) return st;
     st = check_tensors(problem, tensors, true);
     if (st != SLIKL_OK) return st;
-    if (options && options->loss && (reinterpret_cast<uintptr_t>(options->loss) & 3))
+    if (options && ((reinterpret_cast<uintptr_t>(options->loss) & 3) ||
+                    (reinterpret_cast<uintptr_t>(options->seq_used_q) & 3) ||
+                    (reinterpret_cast<uintptr_t>(options->seq_used_k) & 3)))
         return SLIKL_ERR_PARAM_INVALID;
     if (!workspace) return SLIKL_ERR_PARAM_NULLPTR;
     if (reinterpret_cast<uintptr_t>(workspace) & 255) return SLIKL_ERR_PARAM_INVALID;
@@ -250,6 +252,10 @@ slikl_status slikl_grad_ex(const slikl_problem *problem, const slikl_tensors *te
     if (!ok) return SLIKL_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     Params P = make_params(problem, dv, tensors, workspace);
+    if (options) {
+        P.used_q = options->seq_used_q;
+        P.used_k = options->seq_used_k;
+    }
     void *fused_begin = options ? options->fused_begin : nullptr;
     void *fused_end = options ? options->fused_end : nullptr;
 

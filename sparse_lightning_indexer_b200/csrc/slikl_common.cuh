@@ -26,15 +26,17 @@ struct Params {
     const void *q, *k;
     const float *w, *p;
     const int32_t *idx, *cu_q, *cu_k;
+    const int32_t *used_q, *used_k;   // [B] rows of each batch in use, or null (all in use)
     void *dq, *dk;
     float *dw, *y;
     // workspace regions
     uint32_t *status;     // device status word(s)
     int32_t *meta;        // [kMetaHeader + 2*workers]
     int32_t *tok_kbase;   // [T1] first key row of the token's batch
-    int32_t *tok_klen;    // [T1] key count of the token's batch
+    int32_t *tok_klen;    // [T1] keys of the token's batch in use (0 for a padding row); a
+                          // slot is valid when 0 <= index < tok_klen
     int32_t *tok_cost;    // [T1] work estimate per token
-    uint64_t *tok_tiles;  // [T1] bit i set when slot tile i holds an index >= 0
+    uint64_t *tok_tiles;  // [T1] bit i set when slot tile i holds a valid index
     int64_t *cost_prefix; // [T1 + 1]
     float *dk_acc;        // [T2*D] fp32 accumulator (atomic mode)
     float *partials;      // [T1*K*D] per-slot dK rows (deterministic mode)
@@ -133,13 +135,11 @@ __device__ __forceinline__ void red_add_f32(float *addr, float v) {
     asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
 }
 
-// Key row of slot value v for a token whose batch keys are [kbase, kbase + klen), or -1.
-// Values outside [-1, klen) break the index contract: they are flagged and treated as invalid.
-__device__ __forceinline__ int32_t slot_row(int32_t v, int32_t kbase, int32_t klen,
-                                            uint32_t *status) {
-    if (v >= 0 && v < klen) return kbase + v;
-    if (v != -1) set_status(status, SLIKL_DEV_INDEX_OUT_OF_RANGE);
-    return -1;
+// Key row of slot value v for a token whose keys in use are [kbase, kbase + klen), or -1.
+// (Values that break the index contract were flagged by the metadata pass; here they are
+// simply invalid.)
+__device__ __forceinline__ int32_t slot_row(int32_t v, int32_t kbase, int32_t klen) {
+    return v >= 0 && v < klen ? kbase + v : -1;
 }
 
 // kernels (defined in the .cu files)

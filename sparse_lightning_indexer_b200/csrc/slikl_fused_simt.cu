@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_simt(Params P) {
         for (int c0 = 0; c0 < K; c0 += kChunk) {
             if (tid < kChunk) {
                 int j = c0 + tid;
-                rows[tid] = j < K ? slot_row(irow[j], kbase, klen, P.status) : -1;
+                rows[tid] = j < K ? slot_row(irow[j], kbase, klen) : -1;
             }
             __syncthreads();
             int any = __syncthreads_or(tid < kChunk && rows[tid] >= 0);
@@ -143,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_simt(Params P) {
         for (int c0 = 0; c0 < K; c0 += kChunk) {
             if (tid < kChunk) {
                 int j = c0 + tid;
-                rows[tid] = j < K ? slot_row(irow[j], kbase, klen, P.status) : -1;
+                rows[tid] = j < K ? slot_row(irow[j], kbase, klen) : -1;
             }
             __syncthreads();
             int any = __syncthreads_or(tid < kChunk && rows[tid] >= 0);

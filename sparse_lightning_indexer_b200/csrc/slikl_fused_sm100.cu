@@ -590,8 +590,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     z_a = 0.f;
                 }
                 const int32_t v = cur.v;
-                const bool valid = v >= 0 && v < kl;
-                if (v != -1 && !valid) set_status(P.status, SLIKL_DEV_INDEX_OUT_OF_RANGE);
+                const bool valid = v >= 0 && v < kl;   // (the metadata pass checked the index)
                 if (!wait_bar(&bars->s_full[sb], (gk >> 1) & 1, &ctl.abort, P.status)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t sa = tm_s + sb * N1P + lane_addr;

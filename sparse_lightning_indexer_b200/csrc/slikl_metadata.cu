@@ -9,8 +9,9 @@
 // Three kernels:
 //   meta_validate  one block: checks cu_seqlens_q/k, longest key range -> header[5]; for the
 //                  key-major dK path also the first unit of every batch
-//   meta_tokens    one warp per query row: batch, key range, cost, non-empty slot tiles and
-//                  (key-major path) the 256-key block pairs the row names
+//   meta_tokens    one warp per query row: batch, key range in use, index-contract check,
+//                  cost, non-empty slot tiles and (key-major path) the 256-key block pairs
+//                  the row names
 //   meta_split     one block: header fields, prefix sum of costs, per-worker ranges
 // and two for the key-major dK path:
 //   km_units       one warp per unit (32 query rows of a batch x one 256-key block pair):
@@ -134,21 +135,41 @@ __global__ void meta_tokens(Params P) {
     const int lane = threadIdx.x & 31;
     const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     if (t >= P.T1) return;
-    int64_t b = batch_of_row(P, t);
-    int32_t kbase, klen;
-    if (P.status[1]) { kbase = 0; klen = 0; }
-    else if (P.layout_k == SLIKL_BSND) { kbase = (int32_t)(b * P.S2); klen = (int32_t)P.S2; }
-    else { kbase = P.cu_k[b]; klen = P.cu_k[b + 1] - kbase; }
-    // cost = 1 + number of 128-slot tiles holding an index >= 0; lane l reads slots
-    // 4l..4l+3 of each tile (one 16-byte load when the row is 16-byte aligned)
+    const int64_t b = batch_of_row(P, t);
+    int64_t q0, q1, k0, kfull;
+    batch_ranges(P, b, q0, q1, k0, kfull);
+    // rows and keys of the batch in use (seqUsedQ / seqUsedK), clamped into its ranges
+    bool in_use = true;
+    int64_t kuse = kfull;
+    if (P.used_q) {
+        const int64_t u = P.used_q[b], n = q1 - q0 > 0 ? q1 - q0 : 0;
+        const int64_t c = u < 0 ? 0 : (u > n ? n : u);
+        if (c != u && lane == 0) set_status(P.status, SLIKL_DEV_BAD_SEQ_USED);
+        in_use = t - q0 < c;
+    }
+    if (P.used_k) {
+        const int64_t u = P.used_k[b];
+        const int64_t c = u < 0 ? 0 : (u > kfull ? kfull : u);
+        if (c != u && lane == 0) set_status(P.status, SLIKL_DEV_BAD_SEQ_USED);
+        kuse = c;
+    }
+    const int32_t kbase = (int32_t)k0;
+    const int32_t klen = in_use ? (int32_t)kuse : 0;   // a slot is valid when 0 <= v < klen
+    // cost = 1 + number of 128-slot tiles holding a valid index; lane l reads slots
+    // 4l..4l+3 of each tile (one 16-byte load when the row is 16-byte aligned). Every index
+    // of a row in use is checked against the batch's whole key range (a padding row's
+    // indices are not read).
     const int32_t *row = P.idx + t * (int64_t)P.K;
     const bool vec = (P.K & 3) == 0;
+    const bool check = !P.status[1];
     const int32_t klim = P.km ? (klen < P.S2m ? klen : P.S2m) : 0;
     int tiles = 0;
     uint64_t mask = 0;
     uint32_t pw0 = 0, pw1 = 0;           // 256-key block pairs named (key-major path, <= 64)
+    bool bad = false;
+    const int ntiles = in_use ? (P.K + kSlotTile - 1) / kSlotTile : 0;
 #pragma unroll 4
-    for (int i = 0; i < (P.K + kSlotTile - 1) / kSlotTile; ++i) {
+    for (int i = 0; i < ntiles; ++i) {
         const int j = i * kSlotTile + 4 * lane;
         int v[4] = {-1, -1, -1, -1};
         if (vec) {
@@ -163,7 +184,8 @@ __global__ void meta_tokens(Params P) {
         bool any = false;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-            any |= v[u] >= 0;
+            bad |= check && (v[u] < -1 || v[u] >= kfull);
+            any |= v[u] >= 0 && v[u] < klen;
             if (v[u] >= 0 && v[u] < klim) {
                 const int kp = v[u] >> 8;
                 const uint32_t bit = 1u << (kp & 31);
@@ -175,6 +197,7 @@ __global__ void meta_tokens(Params P) {
             mask |= uint64_t(1) << i;
         }
     }
+    if (bad) set_status(P.status, SLIKL_DEV_INDEX_OUT_OF_RANGE);
     if (P.km) {
         pw0 = __reduce_or_sync(0xffffffffu, pw0);
         pw1 = __reduce_or_sync(0xffffffffu, pw1);

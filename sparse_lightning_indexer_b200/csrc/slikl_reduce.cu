@@ -37,7 +37,7 @@ __global__ void sort_init(Params P, int64_t n) {
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
          i += (int64_t)gridDim.x * blockDim.x) {
         int64_t t = i / P.K;
-        int32_t r = slot_row(P.idx[i], P.tok_kbase[t], P.tok_klen[t], P.status);
+        int32_t r = slot_row(P.idx[i], P.tok_kbase[t], P.tok_klen[t]);
         P.keys0[i] = r >= 0 ? r : (int32_t)P.T2;
         P.vals0[i] = (int32_t)i;
     }

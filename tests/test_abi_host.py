@@ -216,8 +216,12 @@ def test_grad_ex_host_validation(lib):
         sli.SLIKL_ERR_PARAM_INVALID
     assert grad_ex_rc(lib, base_problem(N1=128), tn, 1 << 20, 1 << 40,
                       sli.make_options("keymajor")) == sli.SLIKL_ERR_PARAM_INVALID
-    # loss output must be 4-byte aligned
+    # loss output and used-length inputs must be 4-byte aligned
     assert grad_ex_rc(lib, pr, tn, 1 << 20, need_auto, sli.make_options(loss=0x1002)) == \
+        sli.SLIKL_ERR_PARAM_INVALID
+    assert grad_ex_rc(lib, pr, tn, 1 << 20, need_auto, sli.make_options(seq_used_q=0x1001)) == \
+        sli.SLIKL_ERR_PARAM_INVALID
+    assert grad_ex_rc(lib, pr, tn, 1 << 20, need_auto, sli.make_options(seq_used_k=0x1003)) == \
         sli.SLIKL_ERR_PARAM_INVALID
     # NULL tensors / workspace
     assert lib.slikl_grad_ex(ctypes.byref(pr), None, None, 0, None, None) == sli.SLIKL_ERR_PARAM_NULLPTR
@@ -233,8 +237,19 @@ def test_grad_ex_no_device_is_an_error(lib):
         assert grad_ex_rc(lib, pr, tn, 1 << 20, need, sli.make_options(path)) == sli.SLIKL_ERR_CUDA
 
 
+def header_struct_fields(struct_name):
+    """Field names of a typedef'd struct in include/slikl.h, in declaration order."""
+    text = open(os.path.join(ROOT, "include", "slikl.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    body = re.search(r"typedef struct \{([^}]*)\}\s*" + struct_name + ";", text).group(1)
+    return [re.search(r"(\w+)\s*(\[[^\]]*\])?\s*$", d.strip()).group(1)
+            for d in body.split(";") if d.strip()]
+
+
 def test_options_struct_layout():
     """The ctypes mirror of slikl_options matches the header's field order and pointer sizes."""
     names = [n for n, _ in sli.slikl_options._fields_]
-    assert names == ["dk_path", "fused_begin", "fused_end", "dk_begin", "dk_end", "loss"]
-    assert ctypes.sizeof(sli.slikl_options) == 8 + 5 * ctypes.sizeof(ctypes.c_void_p)
+    assert names == header_struct_fields("slikl_options")
+    assert names == ["dk_path", "fused_begin", "fused_end", "dk_begin", "dk_end", "loss",
+                     "seq_used_q", "seq_used_k"]
+    assert ctypes.sizeof(sli.slikl_options) == 8 + 7 * ctypes.sizeof(ctypes.c_void_p)

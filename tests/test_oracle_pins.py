@@ -9,7 +9,9 @@
   reduces to the softmax cross-entropy gradient;
 * invariants: sum y = 1 over valid slots, y = 0 off them, untouched dk rows exactly 0,
   unreferenced key rows and p at invalid slots have no influence, and the identities
-  w_h dW_h = <q_h, dq_h> and sum_t,h w dW = sum_r <k_r, dk_r>.
+  w_h dW_h = <q_h, dq_h> and sum_t,h w dW = sum_r <k_r, dk_r>;
+* used lengths (seqUsedQ / seqUsedK): equal to the excluded slots rewritten to -1,
+  padding rows never read, finite differences of the loss over the slots in use.
 """
 
 import json
@@ -373,3 +375,91 @@ def test_split_weighted_brute_force():
             t = ranges[c, 0]
             assert P[t] * cores >= target
             assert t == 0 or P[t - 1] * cores < target
+
+
+# ---------------------------------------------------------------------------
+# used lengths (seqUsedQOptional / seqUsedKOptional: the page fixes only their type; the
+# reading is "rows of each batch in use": query rows past q_used[b] are padding, slots
+# naming a key past k_used[b] are invalid)
+# ---------------------------------------------------------------------------
+
+def used_valid(pr, q_used, k_used):
+    """Valid-slot mask under used lengths, written from the reading alone."""
+    idx, qs = pr["idx"], pr["q_start"]
+    valid = np.zeros(idx.shape, dtype=bool)
+    for b in range(qs.size - 1):
+        for t in range(qs[b], qs[b + 1]):
+            if t - qs[b] < q_used[b]:
+                valid[t] = (idx[t] >= 0) & (idx[t] < k_used[b])
+    return valid
+
+
+def test_seq_used_equals_masked_indices():
+    """Used lengths act exactly as rewriting the slots they exclude to -1."""
+    pr = tiny_problem(10, lens_q=(3, 2), lens_k=(4, 3))
+    qu, ku = [2, 1], [3, 1]
+    valid = used_valid(pr, qu, ku)
+    assert valid.any() and (~valid & (pr["idx"] >= 0)).any()
+    g = run(pr, q_used=qu, k_used=ku)
+    pm = dict(pr, idx=np.where(valid, pr["idx"], -1).astype(np.int32))
+    gm = run(pm)
+    for name in ("y", "dw", "dq", "dk", "loss"):
+        assert np.array_equal(g[name], gm[name]), name
+    # padding rows (local position >= q_used) are all zero
+    for t in (2, 4):
+        assert np.all(g["y"][t] == 0) and np.all(g["dw"][t] == 0) and np.all(g["dq"][t] == 0)
+    # key rows past k_used are never named, so their dk rows are exactly zero
+    assert np.all(g["dk"][[3, 5, 6]] == 0)
+
+
+def test_seq_used_padding_rows_not_read():
+    pr = tiny_problem(12, lens_q=(3, 2), lens_k=(4, 3))
+    qu, ku = [1, 2], [4, 3]
+    g = run(pr, q_used=qu, k_used=ku)
+    bad = dict(pr, idx=pr["idx"].copy())
+    bad["idx"][1] = 99            # padding rows of batch 0: out of range, never read
+    bad["idx"][2] = -5
+    g2 = run(bad, q_used=qu, k_used=ku)
+    for name in ("y", "dw", "dq", "dk", "loss"):
+        assert np.array_equal(g[name], g2[name]), name
+    with pytest.raises(ValueError):
+        run(bad)                   # without used lengths those rows break the contract
+
+
+def test_seq_used_finite_differences():
+    """The gradients under used lengths are those of the KL loss over the slots in use (p
+    normalised over them)."""
+    pr = tiny_problem(11, lens_q=(3, 2), lens_k=(4, 3))
+    qu, ku = [3, 1], [2, 3]
+    valid = used_valid(pr, qu, ku)
+    e = np.where(valid, pr["p"] + 0.1, 0.0)
+    pr["p"] = e / np.maximum(e.sum(1, keepdims=True), 1e-300)
+    g = run(pr, q_used=qu, k_used=ku)
+    h = 1e-6
+
+    def loss():
+        return run(pr, q_used=qu, k_used=ku)["loss"].sum()
+
+    for name, grad in (("q", g["dq"]), ("k", g["dk"]), ("w", g["dw"])):
+        x = pr[name]
+        fd = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            i = it.multi_index
+            old = x[i]
+            x[i] = old + h
+            lp = loss()
+            x[i] = old - h
+            lm = loss()
+            x[i] = old
+            fd[i] = (lp - lm) / (2 * h)
+        scale = np.abs(grad).max()
+        assert scale > 1e-3
+        assert np.abs(fd - grad).max() / scale < 1e-6, name
+
+
+def test_seq_used_out_of_range_rejected():
+    pr = tiny_problem(13, lens_q=(3, 2), lens_k=(4, 3))
+    for qu, ku in (([4, 1], None), ([-1, 1], None), (None, [5, 3]), (None, [1, -2])):
+        with pytest.raises(ValueError):
+            run(pr, q_used=qu, k_used=ku)

@@ -49,8 +49,8 @@ def assert_close(name, got, ref):
         assert a <= mtol * m, f"{name}: max-abs {a:.3e} > {mtol} * {m:.3e}"
 
 
-def run_gpu(wl, deterministic=False, dk_path="auto"):
-    res = sli.grad_workload(wl, deterministic=deterministic, dk_path=dk_path)
+def run_gpu(wl, deterministic=False, dk_path="auto", **kw):
+    res = sli.grad_workload(wl, deterministic=deterministic, dk_path=dk_path, **kw)
     torch.cuda.synchronize()
     flags = sli.slikl_read_device_status(res["workspace"].data_ptr())
     T1, T2, N1, D, K = wl.T1, wl.T2, wl.N1, wl.D, wl.K
@@ -58,7 +58,8 @@ def run_gpu(wl, deterministic=False, dk_path="auto"):
                 dw=res["dw"].double().cpu().numpy().reshape(T1, N1),
                 dq=res["dq"].double().cpu().numpy().reshape(T1, N1, D),
                 dk=res["dk"].double().cpu().numpy().reshape(T2, D),
-                dk_raw=res["dk"].cpu(), flags=flags)
+                dk_raw=res["dk"].cpu(), flags=flags,
+                loss=res["loss"].double().cpu().numpy() if "loss" in res else None)
 
 
 def referenced_rows(wl):
@@ -366,3 +367,111 @@ def test_kl_loss_output_config0():
     res = sli.grad_workload(wl, loss=True)
     torch.cuda.synchronize()
     assert rel_l2(res["loss"].double().cpu().numpy(), ref["loss"]) <= 1e-5
+
+
+# ---------------------------------------------------------------------------
+# used lengths (seq_used_q / seq_used_k): query rows past seq_used_q[b] are padding, slots
+# naming a key past seq_used_k[b] are invalid
+# ---------------------------------------------------------------------------
+
+def batch_starts(wl):
+    return oracle.row_starts(wl.layout, wl.layout, wl.B, wl.S1, wl.S2,
+                             None if wl.cu_seqlens_q is None else wl.cu_seqlens_q.numpy(),
+                             None if wl.cu_seqlens_k is None else wl.cu_seqlens_k.numpy())
+
+
+def used_masked(wl, qu, ku):
+    """Same workload with every slot the used lengths exclude set to -1."""
+    qs, _ = batch_starts(wl)
+    idx = wl.idx.clone().reshape(wl.T1, wl.K)
+    for b in range(wl.B):
+        for t in range(int(qs[b]), int(qs[b + 1])):
+            if t - qs[b] >= qu[b]:
+                idx[t] = -1
+            else:
+                idx[t][idx[t] >= ku[b]] = -1
+    out = si.Workload(**{f: getattr(wl, f) for f in wl.__dataclass_fields__})
+    out.idx = idx.reshape(wl.idx.shape).contiguous()
+    return out
+
+
+def with_garbage_in_padding(wl, qu):
+    """Padding rows get indices that break the contract: they must not be read."""
+    qs, _ = batch_starts(wl)
+    idx = wl.idx.clone().reshape(wl.T1, wl.K)
+    for b in range(wl.B):
+        for t in range(int(qs[b] + qu[b]), int(qs[b + 1])):
+            idx[t, 0::2] = 1 << 30
+            idx[t, 1::2] = -9
+    out = si.Workload(**{f: getattr(wl, f) for f in wl.__dataclass_fields__})
+    out.idx = idx.reshape(wl.idx.shape).contiguous()
+    return out
+
+
+def lengths(wl):
+    qs, ks = batch_starts(wl)
+    return [int(qs[b + 1] - qs[b]) for b in range(wl.B)], [int(ks[b + 1] - ks[b]) for b in range(wl.B)]
+
+
+SEQ_USED = [
+    dict(case=dict(seed=31, layout="BSND", B=3, S1=40, S2=300, N1=16, D=128, K=200),
+         used=lambda lq, lk: ([lq[0], 17, 0], [lk[0], 150, 7])),
+    dict(case=dict(seed=32, layout="TND", B=3, S1=50, S2=400, N1=32, D=128, K=300,
+                   dtype=torch.float16, pattern="causal"),
+         used=lambda lq, lk: ([lq[0] // 2, lq[1], 1], [lk[0] // 3 + 1, lk[1], lk[2]])),
+    dict(case=dict(seed=33, layout="BSND", B=2, S1=24, S2=3000, N1=64, D=128, K=2048,
+                   qk_scale=0.1, w_var=1 / 64),
+         used=lambda lq, lk: ([20, 24], [1000, 2999])),
+    dict(case=dict(seed=34, layout="TND", B=2, S1=20, S2=600, N1=128, D=128, K=257),
+         used=lambda lq, lk: ([lq[0], lq[1] // 2], [lk[0] // 2, lk[1]])),
+]
+
+
+@pytest.mark.parametrize("sc", SEQ_USED, ids=lambda c: f"s{c['case']['seed']}")
+@pytest.mark.parametrize("mode", MODES, ids=MODE_IDS)
+def test_seq_used_parity(sc, mode):
+    det, path = mode
+    case = sc["case"]
+    if path == "keymajor" and not keymajor_possible(case):
+        pytest.skip("the key-major path needs N1 <= 64")
+    wl = si.small(**case)
+    lq, lk = lengths(wl)
+    qu, ku = sc["used"](lq, lk)
+    wm = used_masked(wl, qu, ku)
+    idx = wl.idx.reshape(wl.T1, wl.K)
+    assert (wm.idx.reshape(wl.T1, wl.K) != idx).any()     # the lengths exclude something
+    ref = oracle.grad(wl, seq_used_q=qu, seq_used_k=ku)
+    got = run_gpu(with_garbage_in_padding(wl, qu), deterministic=det, dk_path=path,
+                  seq_used_q=qu, seq_used_k=ku, loss=True)
+    assert got["flags"] == 0
+    check_against(wm, got, ref)
+    check_exact(wm, got)
+    assert rel_l2(got["loss"], ref["loss"]) <= 1e-5
+    assert np.all(got["loss"][ref["loss"] == 0] == 0)      # padding rows: exactly 0
+
+
+def test_seq_used_out_of_range_is_flagged_and_clamped():
+    wl = si.small(seed=35, layout="BSND", B=2, S1=30, S2=200, N1=16, D=128, K=150)
+    got = run_gpu(wl, seq_used_q=[wl.S1 + 5, -3], seq_used_k=[wl.S2 + 1, 60])
+    assert got["flags"] & sli.SLIKL_DEV_BAD_SEQ_USED
+    assert not got["flags"] & sli.SLIKL_DEV_INDEX_OUT_OF_RANGE
+    qu, ku = [wl.S1, 0], [wl.S2, 60]
+    ref = oracle.grad(wl, seq_used_q=qu, seq_used_k=ku)
+    wm = used_masked(wl, qu, ku)
+    check_against(wm, got, ref)
+    check_exact(wm, got)
+
+
+def test_seq_used_keeps_the_index_contract_check():
+    """An index at or past the batch's whole key range is still flagged in a row in use;
+    one inside the range but past seq_used_k is not."""
+    wl = si.small(seed=36, layout="BSND", B=1, S1=12, S2=100, N1=16, D=128, K=40)
+    idx = wl.idx.clone().reshape(wl.T1, wl.K)
+    idx[0, 0] = 99                       # inside the key range, past the used keys: invalid
+    fine = si.Workload(**{f: getattr(wl, f) for f in wl.__dataclass_fields__})
+    fine.idx = idx.reshape(wl.idx.shape).contiguous()
+    assert run_gpu(fine, seq_used_k=[50])["flags"] == 0
+    idx[3, 1] = 100                      # past the batch's key range
+    bad = si.Workload(**{f: getattr(wl, f) for f in wl.__dataclass_fields__})
+    bad.idx = idx.reshape(wl.idx.shape).contiguous()
+    assert run_gpu(bad, seq_used_k=[50])["flags"] & sli.SLIKL_DEV_INDEX_OUT_OF_RANGE
