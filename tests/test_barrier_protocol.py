@@ -1,0 +1,359 @@
+"""A discrete model of the mbarrier protocol of the fused per-token kernel
+(sparse_lightning_indexer_b200/csrc/slikl_fused_sm100.cu), checked on the CPU.
+
+Every warp role is a generator over the barriers it waits on and arrives at, walking the same
+item schedule as the kernel (pass A of the next token alternating with pass B of the current
+one). An mbarrier is modelled by its count of completed phases: a wait on parity P passes once
+the phase of parity P has completed, i.e. while the completed-phase count has the other parity
+(so a fresh barrier passes a wait on parity 1 at once, as in hardware). Asynchronous
+completions (cp.async and TMA arrivals, tcgen05.commit) are taken as immediate: they depend on
+nothing else, so delaying them cannot create a dependency cycle.
+
+The roles run in random interleavings over random token tile masks. Each run must finish (no
+deadlock), and explicit safety checks fail a run in which a buffer is overwritten before its
+previous contents were consumed: K stages, S buffers in TMEM and dS tiles. The checks are what
+catches parity aliasing, where a waiter that skips phases passes a barrier two phases early.
+A negative test keeps the model honest: the producer variant in which each warp waits on a
+stage only at the items it owns is caught.
+"""
+
+import itertools
+import random
+
+import pytest
+
+N_TILE_BITS = 16
+
+
+class Bar:
+    def __init__(self, count):
+        self.count = count
+        self.arrivals = 0
+        self.phases = 0                      # completed phases
+
+    def ready(self, parity):
+        return (self.phases & 1) != parity
+
+    def arrive(self):
+        self.arrivals += 1
+        assert self.arrivals <= self.count
+        if self.arrivals == self.count:
+            self.phases += 1
+            self.arrivals = 0
+
+
+class Violation(AssertionError):
+    pass
+
+
+def schedule(masks):
+    """The kernel's item order: phase 0 = A(t0); phase k = B(t_{k-1}) and A(t_k) alternated,
+    B first, then whichever remains; tiles of a token in index order. Tokens without an
+    active tile are skipped."""
+    toks = [t for t, m in enumerate(masks) if m]
+    items = []
+    nxt = 0
+
+    def take_token():
+        nonlocal nxt
+        if nxt == len(toks):
+            return None
+        t = toks[nxt]
+        tiles = [i for i in range(N_TILE_BITS) if masks[t] >> i & 1]
+        tok = dict(t=t, ord=nxt, tiles=tiles)
+        nxt += 1
+        return tok
+
+    a = take_token()
+    b = None
+    while a is not None or b is not None:
+        ra = list(a["tiles"]) if a else []
+        rb = list(b["tiles"]) if b else []
+        fa, fb, turn_b = True, True, True
+        while ra or rb:
+            if rb and (not ra or turn_b):
+                tile = rb.pop(0)
+                items.append(dict(kind=1, t=b["t"], ord=b["ord"], tile=tile, first=fb, last=not rb))
+                fb = False
+            else:
+                tile = ra.pop(0)
+                items.append(dict(kind=0, t=a["t"], ord=a["ord"], tile=tile, first=fa, last=not ra))
+                fa = False
+            turn_b = not turn_b
+        b = a
+        a = take_token()
+    return items
+
+
+def build(items, rec, stages=4, owner_producers=False):
+    """Roles of one CTA. rec: record mode (key-major dK; no scatter group, the MMA releases the
+    dS tile after the dq product). owner_producers: the known-bad variant."""
+    nprod = 7 if rec else 3
+    bars = {}
+
+    def bar(name, count):
+        bars[name] = Bar(count)
+
+    for s in range(stages):
+        bar(f"kv_full{s}", nprod)
+        bar(f"kv_empty{s}", 1)
+    for b in range(2):
+        bar(f"q_full{b}", 1)
+        bar(f"q_empty{b}", 1)
+        bar(f"s_full{b}", 1)
+        bar(f"s_empty{b}", 4)
+        bar(f"ds_full{b}", 4)
+        bar(f"rows_full{b}", 4)
+        bar(f"dk_full{b}", 1)
+        bar(f"dk_empty{b}", 1 if rec else 4)
+    bar("dq_full", 1)
+    bar("dq_empty", 4)
+    bar("sm_sync", 4)
+
+    # safety bookkeeping: how many times each buffer was filled, and released by each of the
+    # warps that read it (a buffer is free again only when every reader is done with it)
+    st = dict(stage_free=[0] * stages, s_fill=[0, 0], s_free=[[0, 0] for _ in range(4)],
+              ds_fill=[[0, 0] for _ in range(4)], ds_free=[[0, 0] for _ in range(4)])
+
+    def freed(key, b):
+        return min(w[b] for w in st[key])
+
+    serial = itertools.count()
+
+    def wait(name, parity):
+        # each wait carries its own serial number, so a role blocked again on the same
+        # barrier (e.g. back-to-back group syncs) does not read as one that never moved
+        token = next(serial)
+        while not bars[name].ready(parity):
+            yield ("wait", name, token)
+
+    def producer(w):
+        for g, it in enumerate(items):
+            if owner_producers and g % nprod != w:
+                continue
+            if w == 0 and it["kind"] == 0 and it["first"]:
+                qb = it["ord"] & 1
+                yield from wait(f"q_empty{qb}", ((it["ord"] >> 1) & 1) ^ 1)
+                bars[f"q_full{qb}"].arrive()
+            s = g % stages
+            yield from wait(f"kv_empty{s}", ((g // stages) & 1) ^ 1)
+            # this warp writes its rows of item g into stage s: every earlier item of the stage
+            # must have been released by the MMA
+            if st["stage_free"][s] < g // stages:
+                raise Violation(f"producer {w} overwrote stage {s} (item {g}) still in use")
+            if owner_producers:
+                for _ in range(nprod):
+                    bars[f"kv_full{s}"].arrive()
+            else:
+                bars[f"kv_full{s}"].arrive()
+            yield ("step",)
+
+    def mma():
+        gk = gd = nb = 0
+
+        def issue_s(it):
+            nonlocal gk
+            s, b = gk % stages, gk & 1
+            if it["kind"] == 0 and it["first"]:
+                yield from wait(f"q_full{it['ord'] & 1}", (it["ord"] >> 1) & 1)
+            yield from wait(f"kv_full{s}", (gk // stages) & 1)
+            yield from wait(f"s_empty{b}", ((gk >> 1) & 1) ^ 1)
+            if freed("s_free", b) < gk >> 1:
+                raise Violation(f"S buffer {b} overwritten (item {gk}) before it was read")
+            st["s_fill"][b] += 1
+            bars[f"s_full{b}"].arrive()
+            if it["kind"] == 0:
+                st["stage_free"][s] += 1
+                bars[f"kv_empty{s}"].arrive()
+            gk += 1
+            return s
+
+        if not items:
+            return
+        i = 0
+        stage_cur = yield from issue_s(items[0])
+        while i < len(items):
+            cur = items[i]
+            stage_nxt = None
+            if i + 1 < len(items):
+                stage_nxt = yield from issue_s(items[i + 1])
+            if cur["kind"] == 1:
+                b = gd & 1
+                if cur["first"]:
+                    yield from wait("dq_empty", (nb & 1) ^ 1)
+                yield from wait(f"ds_full{b}", (gd >> 1) & 1)
+                if not rec:
+                    yield from wait(f"dk_empty{b}", ((gd >> 1) & 1) ^ 1)
+                if min(w[b] for w in st["ds_fill"]) != (gd >> 1) + 1:
+                    raise Violation(f"dq product read dS buffer {b} not holding item {gd}")
+                st["stage_free"][stage_cur] += 1
+                bars[f"kv_empty{stage_cur}"].arrive()
+                if rec:
+                    for w in st["ds_free"]:
+                        w[b] += 1
+                    bars[f"dk_empty{b}"].arrive()
+                else:
+                    bars[f"dk_full{b}"].arrive()
+                if cur["last"]:
+                    bars["dq_full"].arrive()
+                    bars[f"q_empty{cur['ord'] & 1}"].arrive()
+                    nb += 1
+                gd += 1
+            stage_cur = stage_nxt
+            i += 1
+            yield ("step",)
+
+    def scatter(wq):
+        gd = 0
+        for it in items:
+            if it["kind"] != 1:
+                continue
+            b = gd & 1
+            yield from wait(f"rows_full{b}", (gd >> 1) & 1)
+            yield from wait(f"dk_full{b}", (gd >> 1) & 1)
+            st["ds_free"][wq][b] += 1
+            bars[f"dk_empty{b}"].arrive()
+            gd += 1
+            yield ("step",)
+
+    phase = [0] * 4
+
+    def group_sync(wq):
+        bars["sm_sync"].arrive()
+        yield from wait("sm_sync", phase[wq] & 1)
+        phase[wq] += 1
+
+    def softmax(wq):
+        gk = gd = nb = 0
+        for it in items:
+            sb = gk & 1
+            if it["kind"] == 0:
+                if it["first"]:
+                    yield from group_sync(wq)
+                yield from wait(f"s_full{sb}", (gk >> 1) & 1)
+                if st["s_fill"][sb] != (gk >> 1) + 1:
+                    raise Violation(f"pass A read S buffer {sb} not holding item {gk}")
+                st["s_free"][wq][sb] += 1
+                bars[f"s_empty{sb}"].arrive()
+                if it["last"]:
+                    yield from group_sync(wq)
+                    yield from group_sync(wq)
+            else:
+                b = gd & 1
+                yield from wait(f"dk_empty{b}", ((gd >> 1) & 1) ^ 1)
+                if freed("ds_free", b) < gd >> 1:
+                    raise Violation(f"dS buffer {b} overwritten (item {gd}) before it was read")
+                yield from wait(f"s_full{sb}", (gk >> 1) & 1)
+                if st["s_fill"][sb] != (gk >> 1) + 1:
+                    raise Violation(f"pass B read S buffer {sb} not holding item {gk}")
+                st["s_free"][wq][sb] += 1
+                st["ds_fill"][wq][b] += 1
+                bars[f"s_empty{sb}"].arrive()
+                bars[f"ds_full{b}"].arrive()
+                if not rec:
+                    bars[f"rows_full{b}"].arrive()
+                gd += 1
+                if it["last"]:
+                    yield from group_sync(wq)
+                    yield from wait("dq_full", nb & 1)
+                    bars["dq_empty"].arrive()
+                    nb += 1
+            gk += 1
+            yield ("step",)
+
+    roles = {f"producer{w}": producer(w) for w in range(nprod)}
+    roles["mma"] = mma()
+    for q in range(4):
+        roles[f"softmax{q}"] = softmax(q)
+        if not rec:
+            roles[f"scatter{q}"] = scatter(q)
+    return roles
+
+
+def run(masks, rec, seed, **kw):
+    """Random interleaving until every role ends. Returns None, or the names of the roles
+    left waiting (deadlock). Raises Violation on a buffer overwritten too early."""
+    rnd = random.Random(seed)
+    roles = build(schedule(masks), rec, **kw)
+    blocked = {}
+    while roles:
+        progressed = False
+        for name in rnd.sample(list(roles), len(roles)):
+            gen = roles[name]
+            for _ in range(rnd.randint(1, 6)):
+                try:
+                    ev = next(gen)
+                except StopIteration:
+                    del roles[name]
+                    blocked.pop(name, None)
+                    progressed = True
+                    break
+                if ev[0] == "wait":
+                    if blocked.get(name) != ev:
+                        blocked[name] = ev
+                        progressed = True
+                    break
+                blocked.pop(name, None)
+                progressed = True
+        if not progressed:
+            return sorted(roles)
+    return None
+
+
+def random_masks(rnd):
+    n = rnd.randint(1, 6)
+    out = []
+    for _ in range(n):
+        kind = rnd.random()
+        if kind < 0.15:
+            out.append(0)                                   # token without an active tile
+        elif kind < 0.4:
+            out.append((1 << rnd.randint(1, N_TILE_BITS)) - 1)   # causal-like prefix
+        else:
+            out.append(rnd.getrandbits(N_TILE_BITS))
+    return out
+
+
+EDGE_MASKS = [[1], [1, 1], [0b11, 1], [1, 0xFFFF], [0xFFFF, 1, 0xFFFF], [0, 0, 1], [0], [],
+              [1, 0, 1, 0, 1], [0b1010, 0b0101, 0b1111]]
+
+
+@pytest.mark.parametrize("rec", [False, True], ids=["scatter", "record"])
+def test_protocol_finishes_and_is_safe(rec):
+    rnd = random.Random(20261202 + rec)
+    cases = EDGE_MASKS + [random_masks(rnd) for _ in range(250)]
+    for i, masks in enumerate(cases):
+        for seed in range(3):
+            stuck = run(masks, rec, seed=1000 * i + seed)
+            assert stuck is None, f"deadlock with masks {masks}: {stuck}"
+
+
+def test_schedule_order():
+    """Phase k interleaves B(t_{k-1}) and A(t_k), B first; every tile is visited once per
+    pass; first / last flags mark each token's pass boundaries."""
+    items = schedule([0b11, 0, 0b111])
+    got = [(it["kind"], it["t"], it["tile"]) for it in items]
+    assert got == [(0, 0, 0), (0, 0, 1),
+                   (1, 0, 0), (0, 2, 0), (1, 0, 1), (0, 2, 1), (0, 2, 2),
+                   (1, 2, 0), (1, 2, 1), (1, 2, 2)]
+    for kind in (0, 1):
+        for t in (0, 2):
+            mine = [it for it in items if it["kind"] == kind and it["t"] == t]
+            assert mine[0]["first"] and mine[-1]["last"]
+            assert sum(it["first"] for it in mine) == 1 and sum(it["last"] for it in mine) == 1
+
+
+def test_owner_only_producers_are_caught():
+    """Producers that wait on a stage only at the items they own can pass its empty barrier
+    two phases early (a fresh barrier reads as 'previous phase complete'); the model must
+    catch that as an overwritten stage or a deadlock."""
+    rnd = random.Random(7)
+    caught = 0
+    for i in range(60):
+        masks = random_masks(rnd) + [0xFFFF]
+        try:
+            if run(masks, rec=True, seed=i, owner_producers=True) is not None:
+                caught += 1
+        except Violation:
+            caught += 1
+    assert caught > 0
