@@ -15,6 +15,11 @@ previous contents were consumed: K stages, S buffers in TMEM and dS tiles. The c
 catches parity aliasing, where a waiter that skips phases passes a barrier two phases early.
 A negative test keeps the model honest: the producer variant in which each warp waits on a
 stage only at the items it owns is caught.
+
+The key-major dK kernel (sparse_lightning_indexer_b200/csrc/slikl_dk_keymajor.cu) is modelled
+the same way: its producer, 16 dS-builder warps, MMA issuer and 4 flush warps over runs of work
+units, with checks on stage reuse (q, w, records and the dS tile) and on the two TMEM dK
+buffers (a run accumulates only into its own buffer, which is not reused before its flush).
 """
 
 import itertools
@@ -353,6 +358,154 @@ def test_owner_only_producers_are_caught():
         masks = random_masks(rnd) + [0xFFFF]
         try:
             if run(masks, rec=True, seed=i, owner_producers=True) is not None:
+                caught += 1
+        except Violation:
+            caught += 1
+    assert caught > 0
+
+
+# ---------------------------------------------------------------------------
+# key-major dK kernel (sparse_lightning_indexer_b200/csrc/slikl_dk_keymajor.cu)
+# ---------------------------------------------------------------------------
+
+def km_items(runs):
+    """Items of one CTA: one per (query row, work unit); consecutive units on the same key
+    block pair form a run (first / last mark its ends). runs = list of run lengths."""
+    items = []
+    for r, n in enumerate(runs):
+        for k in range(n):
+            items.append(dict(run=r, first=k == 0, last=k == n - 1))
+    return items
+
+
+def km_build(items, stages=4, builders=16, flushers=4, wait_empty=True):
+    """Roles of the key-major kernel. wait_empty=False is a planted mistake (the producer
+    fills a stage without waiting for the MMA to release it)."""
+    bars = {}
+    for s in range(stages):
+        bars[f"full{s}"] = Bar(1)
+        bars[f"dsr{s}"] = Bar(builders)
+        bars[f"empty{s}"] = Bar(1)
+    for b in range(2):
+        bars[f"accf{b}"] = Bar(1)
+        bars[f"acce{b}"] = Bar(flushers)
+    serial = itertools.count()
+    st = dict(stage_free=[0] * stages, ds_fill=[[0] * stages for _ in range(builders)],
+              acc_run=[None, None], acc_flushed=[[0, 0] for _ in range(flushers)])
+
+    def wait(name, parity):
+        token = next(serial)
+        while not bars[name].ready(parity):
+            yield ("wait", name, token)
+
+    def producer():
+        for i, _ in enumerate(items):
+            s = i % stages
+            if wait_empty:
+                yield from wait(f"empty{s}", ((i // stages) & 1) ^ 1)
+            # q, w and records of item i land in stage s
+            if st["stage_free"][s] < i // stages:
+                raise Violation(f"producer overwrote stage {s} (item {i}) still in use")
+            bars[f"full{s}"].arrive()
+            yield ("step",)
+
+    def builder(wb):
+        for i, _ in enumerate(items):
+            s = i % stages
+            yield from wait(f"full{s}", (i // stages) & 1)
+            # the dS tile of stage s is rewritten: the MMA must be done with item i - stages
+            if st["stage_free"][s] < i // stages:
+                raise Violation(f"builder {wb} overwrote dS of stage {s} (item {i}) still in use")
+            st["ds_fill"][wb][s] += 1
+            bars[f"dsr{s}"].arrive()
+            yield ("step",)
+
+    def mma():
+        nrun = 0
+        for i, it in enumerate(items):
+            s, ab = i % stages, nrun & 1
+            yield from wait(f"dsr{s}", (i // stages) & 1)
+            if min(w[s] for w in st["ds_fill"]) != i // stages + 1:
+                raise Violation(f"MMA read dS of stage {s} not holding item {i}")
+            if it["first"]:
+                yield from wait(f"acce{ab}", ((nrun >> 1) & 1) ^ 1)
+                if min(w[ab] for w in st["acc_flushed"]) < nrun >> 1:
+                    raise Violation(f"dK buffer {ab} reused (run {nrun}) before its flush")
+                st["acc_run"][ab] = it["run"]
+            elif st["acc_run"][ab] != it["run"]:
+                raise Violation(f"run {it['run']} accumulates into buffer {ab} of another run")
+            st["stage_free"][s] += 1
+            bars[f"empty{s}"].arrive()
+            if it["last"]:
+                bars[f"accf{ab}"].arrive()
+                nrun += 1
+            yield ("step",)
+
+    def flush(wf):
+        nrun = 0
+        for it in items:
+            if not it["last"]:
+                continue
+            ab = nrun & 1
+            yield from wait(f"accf{ab}", (nrun >> 1) & 1)
+            if st["acc_run"][ab] != it["run"]:
+                raise Violation(f"flush of run {it['run']} found buffer {ab} holding another run")
+            st["acc_flushed"][wf][ab] += 1
+            bars[f"acce{ab}"].arrive()
+            nrun += 1
+            yield ("step",)
+
+    roles = {"producer": producer(), "mma": mma()}
+    for w in range(builders):
+        roles[f"builder{w}"] = builder(w)
+    for w in range(flushers):
+        roles[f"flush{w}"] = flush(w)
+    return roles
+
+
+def km_run(runs, seed, **kw):
+    rnd = random.Random(seed)
+    roles = km_build(km_items(runs), **kw)
+    blocked = {}
+    while roles:
+        progressed = False
+        for name in rnd.sample(list(roles), len(roles)):
+            gen = roles[name]
+            for _ in range(rnd.randint(1, 6)):
+                try:
+                    ev = next(gen)
+                except StopIteration:
+                    del roles[name]
+                    progressed = True
+                    break
+                if ev[0] == "wait":
+                    if blocked.get(name) != ev:
+                        blocked[name] = ev
+                        progressed = True
+                    break
+                blocked.pop(name, None)
+                progressed = True
+        if not progressed:
+            return sorted(roles)
+    return None
+
+
+def test_keymajor_protocol_finishes_and_is_safe():
+    rnd = random.Random(20261203)
+    cases = [[1], [1, 1, 1], [32], [1, 32, 1], [5, 5, 5, 5, 5]]
+    cases += [[rnd.randint(1, 12) for _ in range(rnd.randint(1, 8))] for _ in range(150)]
+    for i, runs in enumerate(cases):
+        for seed in range(3):
+            assert km_run(runs, seed=1000 * i + seed) is None, f"deadlock with runs {runs}"
+
+
+def test_keymajor_planted_mistake_is_caught():
+    rnd = random.Random(11)
+    caught = 0
+    for i in range(40):
+        runs = [rnd.randint(1, 12) for _ in range(rnd.randint(2, 8))]
+        try:
+            if km_run(runs, seed=i, wait_empty=False) is not None:
                 caught += 1
         except Violation:
             caught += 1
