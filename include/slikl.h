@@ -100,7 +100,9 @@ typedef struct {
 } slikl_problem;
 
 /* Tensors of one call. All DEVICE pointers, caller-owned, contiguous; q, k, dq, dk 16-byte
- * aligned, the others 4-byte aligned (SLIKL_ERR_PARAM_INVALID otherwise). */
+ * aligned, the others 4-byte aligned (SLIKL_ERR_PARAM_INVALID otherwise). A tensor with no
+ * elements may be NULL: with TND queries and T1 = 0, q, w, attn_softmax_l1norm,
+ * sparse_indices, dq, dw and softmax_out; with TND keys and T2 = 0, k and dk. */
 typedef struct {
     const void *q;                      /* dtype  [B,S1,N1,D] / [T1,N1,D]            */
     const void *k;                      /* dtype  [B,S2,1,D]  / [T2,1,D]             */

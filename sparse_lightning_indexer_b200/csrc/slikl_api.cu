@@ -161,12 +161,17 @@ Params make_params(const slikl_problem *pr, const Derived &dv, const slikl_tenso
 
 slikl_status check_tensors(const slikl_problem *pr, const slikl_tensors *tn, bool need_all) {
     if (!tn) return SLIKL_ERR_PARAM_NULLPTR;
-    if (!tn->sparse_indices) return SLIKL_ERR_PARAM_NULLPTR;
+    // a tensor with no elements (TND with T1 = 0 rows of q, or T2 = 0 rows of k) may be NULL:
+    // nothing reads or writes it
+    const bool q_rows = !(pr->layout_q == SLIKL_TND && pr->T1 == 0);
+    const bool k_rows = !(pr->layout_k == SLIKL_TND && pr->T2 == 0);
+    if (q_rows && !tn->sparse_indices) return SLIKL_ERR_PARAM_NULLPTR;
     if (pr->layout_q == SLIKL_TND && !tn->cu_seqlens_q) return SLIKL_ERR_PARAM_NULLPTR;
     if (pr->layout_k == SLIKL_TND && !tn->cu_seqlens_k) return SLIKL_ERR_PARAM_NULLPTR;
-    if (need_all && (!tn->q || !tn->k || !tn->w || !tn->attn_softmax_l1norm || !tn->dq ||
-                     !tn->dk || !tn->dw || !tn->softmax_out))
+    if (need_all && q_rows && (!tn->q || !tn->w || !tn->attn_softmax_l1norm || !tn->dq ||
+                               !tn->dw || !tn->softmax_out))
         return SLIKL_ERR_PARAM_NULLPTR;
+    if (need_all && k_rows && (!tn->k || !tn->dk)) return SLIKL_ERR_PARAM_NULLPTR;
     // 16-byte vector loads/stores of q, k, dq, dk rows; 4-byte elements elsewhere
     auto mis = [](const void *p, uintptr_t a) { return p && (reinterpret_cast<uintptr_t>(p) & (a - 1)); };
     if (mis(tn->q, 16) || mis(tn->k, 16) || mis(tn->dq, 16) || mis(tn->dk, 16) ||

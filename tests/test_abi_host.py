@@ -253,3 +253,30 @@ def test_options_struct_layout():
     assert names == ["dk_path", "fused_begin", "fused_end", "dk_begin", "dk_end", "loss",
                      "seq_used_q", "seq_used_k"]
     assert ctypes.sizeof(sli.slikl_options) == 8 + 7 * ctypes.sizeof(ctypes.c_void_p)
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks host validation up to the first CUDA call")
+def test_empty_tensors_may_be_null(lib):
+    """With TND and no query rows (T1 = 0) the query-side tensors may be NULL, with no key rows
+    (T2 = 0) k and dk may be; validation then passes and the call reaches the device (which is
+    absent here: SLIKL_ERR_CUDA). Non-empty tensors stay required."""
+    q_side = ("q", "w", "attn_softmax_l1norm", "sparse_indices", "dq", "dw", "softmax_out")
+    pr = base_problem(layout_q=sli.SLIKL_TND, layout_k=sli.SLIKL_TND, B=2, T1=0, T2=50, S2=30)
+    need = ws_ex(lib, pr, "auto")[1]
+    tn = fake_tensors(tnd_q=True, tnd_k=True)
+    for name in q_side:
+        setattr(tn, name, None)
+    assert grad_ex_rc(lib, pr, tn, 1 << 20, need, None) == sli.SLIKL_ERR_CUDA
+    tn.k = None                                          # T2 > 0: k is required
+    assert grad_ex_rc(lib, pr, tn, 1 << 20, need, None) == sli.SLIKL_ERR_PARAM_NULLPTR
+
+    pr = base_problem(layout_q=sli.SLIKL_TND, layout_k=sli.SLIKL_TND, B=2, T1=40, T2=0, S2=0)
+    need = ws_ex(lib, pr, "auto")[1]
+    tn = fake_tensors(tnd_q=True, tnd_k=True)
+    tn.k = tn.dk = None
+    assert grad_ex_rc(lib, pr, tn, 1 << 20, need, None) == sli.SLIKL_ERR_CUDA
+    for name in q_side:                                  # T1 > 0: each query-side tensor required
+        tn2 = fake_tensors(tnd_q=True, tnd_k=True)
+        tn2.k = tn2.dk = None
+        setattr(tn2, name, None)
+        assert grad_ex_rc(lib, pr, tn2, 1 << 20, need, None) == sli.SLIKL_ERR_PARAM_NULLPTR, name

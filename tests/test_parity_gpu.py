@@ -475,3 +475,36 @@ def test_seq_used_keeps_the_index_contract_check():
     bad = si.Workload(**{f: getattr(wl, f) for f in wl.__dataclass_fields__})
     bad.idx = idx.reshape(wl.idx.shape).contiguous()
     assert run_gpu(bad, seq_used_k=[50])["flags"] & sli.SLIKL_DEV_INDEX_OUT_OF_RANGE
+
+
+# ---------------------------------------------------------------------------
+# empty problems (TND): no query rows, or no key rows
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("mode", MODES, ids=MODE_IDS)
+def test_no_query_rows(mode):
+    """Every query batch empty (T1 = 0; the query-side tensors have no elements and go in as
+    NULL): nothing is computed and dk is exactly +0."""
+    det, path = mode
+    wl = si.small(seed=41, layout="TND", B=2, lens_q=[0, 0], lens_k=[5, 7], N1=16, D=128, K=8)
+    assert wl.T1 == 0 and wl.T2 == 12
+    got = run_gpu(wl, deterministic=det, dk_path=path)
+    assert got["flags"] == 0
+    assert got["y"].shape == (0, wl.K) and got["dq"].shape == (0, wl.N1, wl.D)
+    assert torch.all(got["dk_raw"].view(torch.int16) == 0)
+
+
+@pytest.mark.parametrize("det", [False, True], ids=["scatter", "det"])
+def test_no_key_rows(det):
+    """Every key batch empty (T2 = 0; k and dk go in as NULL): no slot can be valid, so
+    softmax_out, dq and dw are exactly 0."""
+    wl = si.small(seed=42, layout="TND", B=2, lens_q=[3, 2], lens_k=[0, 0], N1=16, D=128, K=8,
+                  pattern="none")
+    assert wl.T1 == 5 and wl.T2 == 0
+    got = run_gpu(wl, deterministic=det)
+    assert got["flags"] == 0
+    for name in ("y", "dw", "dq"):
+        assert np.all(got[name] == 0.0), name
+    ref = oracle.grad(wl)
+    for name in ("y", "dw", "dq"):
+        assert np.array_equal(got[name], ref[name]), name
