@@ -280,3 +280,22 @@ def test_empty_tensors_may_be_null(lib):
         tn2.k = tn2.dk = None
         setattr(tn2, name, None)
         assert grad_ex_rc(lib, pr, tn2, 1 << 20, need, None) == sli.SLIKL_ERR_PARAM_NULLPTR, name
+
+
+def test_binding_rejects_bad_used_lengths():
+    """grad() checks the used-length tensors before any CUDA call: int32, on the device,
+    contiguous, B entries."""
+    q = torch.zeros(6, 16, 128, dtype=torch.bfloat16)
+    k = torch.zeros(10, 1, 128, dtype=torch.bfloat16)
+    w = torch.zeros(6, 16)
+    p = torch.zeros(6, 1, 8)
+    idx = torch.full((6, 1, 8), -1, dtype=torch.int32)
+    cuq = torch.tensor([0, 2, 6], dtype=torch.int32)
+    cuk = torch.tensor([0, 4, 10], dtype=torch.int32)
+    bad = [torch.tensor([1, 2], dtype=torch.int64),          # wrong dtype
+           torch.tensor([1, 2, 3], dtype=torch.int32),       # wrong length
+           torch.tensor([1, 2], dtype=torch.int32)]          # host tensor
+    for u in bad:
+        for name in ("seq_used_q", "seq_used_k"):
+            with pytest.raises(ValueError, match=name):
+                sli.grad(q, k, w, p, idx, "TND", "TND", cuq, cuk, **{name: u})
