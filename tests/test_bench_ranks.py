@@ -62,3 +62,26 @@ def test_fused_flop_count():
         N1, D, K, T1 = 64, 128, 2048, 4096
     assert bench.fused_algorithmic_flop(W, "keymajor") == 4.0 * 64 * 128 * 2048 * 4096
     assert bench.fused_algorithmic_flop(W, "scatter") == 6.0 * 64 * 128 * 2048 * 4096
+
+
+def test_reference_arm_prints_the_contract_line():
+    """`bench.py --impl reference` (the fp64 oracle on the host cores) prints one JSON line
+    with the contract's keys; it needs no GPU."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference",
+                          "--config", "0", "--steps", "1", "--warmup", "3"],
+                         check=True, capture_output=True, text=True, timeout=600).stdout
+    lines = [ln for ln in out.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    j = json.loads(lines[0])
+    assert j["impl"] == "reference" and j["value"] > 0 and j["unit"] == "query-tokens/s"
+    for key in ("metric", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in j, key
+    assert j["steps"] == 1 and j["warmup"] == 3 and j["higher_is_better"] is True
+    assert j["cpu_baseline"]["kind"] == "oracle" and j["cpu_baseline"]["value"] == j["value"]
+    assert j["e2e"] == {"value": j["value"], "unit": j["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
