@@ -145,10 +145,10 @@ def raw_elapsed_ms(a, b):
     return ms
 
 
-# DRAM bytes (read + write) of one fused-kernel launch on the headline workload, from the ncu
-# capture summarised in profiles/fused_sm100_causal4096_n64_k2048.md, valid only while the
-# kernel's sources stay as they are (hash of the three files below); otherwise the traffic is
-# reported as unknown.
+# DRAM bytes (read + write) of one fused-kernel launch on the headline workload, read from an
+# ncu capture of that launch (dram__bytes_read.sum + dram__bytes_write.sum). The figure holds
+# only while the kernel's sources are the ones captured (hash of the three files below);
+# otherwise the traffic is reported as unknown (null).
 FUSED_TRAFFIC = {"sources_sha256_16": "c4172c992f118d38", "workload_config": 1,
                  "dk_path": "keymajor", "bytes": 120.852736e6 + 193.821952e6}
 
@@ -174,12 +174,16 @@ def combine_over_ranks(local, world, device):
     return t.tolist()
 
 
-def fused_algorithmic_flop(wl, dk_path):
-    """Algorithmic FLOPs of one fused-kernel launch at the nominal slot count: the S and dq
-    products (2 N1 D each per slot), plus the dK product (2 N1 D) when the fused kernel forms dK
-    itself (scatter path). The second S product of pass B is recomputation, not counted."""
+def fused_algorithmic_flop(wl, dk_path, valid_slots=None):
+    """Algorithmic FLOPs of one fused-kernel launch: the S and dq products (2 N1 D each per
+    slot), plus the dK product (2 N1 D) when the fused kernel forms dK itself (scatter path).
+    With valid_slots the count is over the slots that hold an index (the work the kernel
+    does: tiles without a valid slot are skipped); without it, over all T1 * topk slots
+    (nominal). The second S product of the softmax's second pass is recomputation, not
+    counted."""
     per_slot = 4.0 if dk_path == "keymajor" else 6.0
-    return per_slot * wl.N1 * wl.D * wl.K * wl.T1
+    slots = wl.K * wl.T1 if valid_slots is None else valid_slots
+    return per_slot * wl.N1 * wl.D * slots
 
 
 def oracle_rate(wl, ntok, seed=0, min_seconds=0.0):
@@ -227,6 +231,117 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+NOMINAL_BF16_TFLOPS = 2250.0   # B200 dense bf16 at the boost clock (context beside the measured peak)
+
+
+class Runner:
+    """One workload resident on the device, called through slikl_grad_ex on `stream`."""
+
+    def __init__(self, sli, wl, dev, stream, deterministic, dk_path):
+        import torch
+        self.sli, self.wl, self.dev, self.stream = sli, wl, dev, stream
+        self.q, self.k, self.w, self.p, self.idx = (getattr(wl, n).to(dev)
+                                                   for n in ("q", "k", "w", "p", "idx"))
+        self.cuq = wl.cu_seqlens_q.to(dev) if wl.cu_seqlens_q is not None else None
+        self.cuk = wl.cu_seqlens_k.to(dev) if wl.cu_seqlens_k is not None else None
+        B = wl.B if wl.layout == "TND" else None
+        self.pr = sli.make_problem(self.q, self.k, self.idx, wl.layout, wl.layout,
+                                   deterministic, B, sli.key_range_bound_of(wl))
+        self.dk_path_arg = dk_path
+        self.opt = sli.make_options(dk_path)
+        self.dk_path = ("keymajor" if sli.slikl_grad_dk_path(self.pr, self.opt)
+                        == sli.SLIKL_DK_KEYMAJOR else "scatter")
+        self.nbytes = sli.slikl_grad_workspace_size_ex(self.pr, self.opt)
+        self.ws = torch.empty(self.nbytes, dtype=torch.uint8, device=dev)
+        self.out = dict(dq=torch.empty_like(self.q), dk=torch.empty_like(self.k),
+                        dw=torch.empty_like(self.w), softmax_out=torch.empty_like(self.p))
+        self.tn = self.tensors(self.q, self.k, self.w, self.p, self.idx)
+
+    def tensors(self, qq, kk, ww, pp, ii):
+        tn = self.sli.slikl_tensors()
+        tn.q, tn.k, tn.w, tn.attn_softmax_l1norm, tn.sparse_indices = (
+            qq.data_ptr(), kk.data_ptr(), ww.data_ptr(), pp.data_ptr(), ii.data_ptr())
+        tn.cu_seqlens_q = self.cuq.data_ptr() if self.cuq is not None else None
+        tn.cu_seqlens_k = self.cuk.data_ptr() if self.cuk is not None else None
+        o = self.out
+        tn.dq, tn.dk, tn.dw, tn.softmax_out = (o["dq"].data_ptr(), o["dk"].data_ptr(),
+                                               o["dw"].data_ptr(), o["softmax_out"].data_ptr())
+        return tn
+
+    def step(self, evs=None, tn=None):
+        opt = self.opt if evs is None else self.sli.make_options(self.dk_path_arg,
+                                                                 *(int(e) for e in evs))
+        self.sli.slikl_grad_ex(self.pr, tn or self.tn, self.ws.data_ptr(), self.nbytes,
+                               self.stream.cuda_stream, opt)
+
+    def timed(self, steps, warmup, flush, barrier=None):
+        """W untimed calls, then `steps` calls each after an L2 flush (outside the events);
+        returns per-step lists (ms) of the whole call, the fused kernel and the dK stage."""
+        import torch
+        for _ in range(warmup):
+            flush.fill_(1)
+            self.step()
+        torch.cuda.synchronize(self.dev)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        kev = [tuple(raw_event() for _ in range(4)) for _ in range(steps)]
+        if barrier:
+            barrier()
+        for i in range(steps):
+            flush.fill_(1)
+            ev[i][0].record(self.stream)
+            self.step(kev[i])
+            ev[i][1].record(self.stream)
+        torch.cuda.synchronize(self.dev)
+        if barrier:
+            barrier()
+        return ([a.elapsed_time(b) for a, b in ev], [raw_elapsed_ms(e[0], e[1]) for e in kev],
+                [raw_elapsed_ms(e[2], e[3]) for e in kev])
+
+    def status(self):
+        return self.sli.slikl_read_device_status(self.ws.data_ptr(), self.stream.cuda_stream)
+
+
+def step_roofline_ms(stats, peaks, peak_tf):
+    return 1e3 * max(stats["flop_nom"] / (peak_tf * 1e12), stats["bytes"] / (peaks["hbm_gbs"] * 1e9))
+
+
+def per_config_lines(sli, dev, stream, flush, peaks, steps, warmup):
+    """The other full-size workloads, timed the same way as the headline (device time, L2
+    flushed before every step): configs 2, 3 and 4 on the auto dK path, and the
+    deterministic reduction on configs 4 and 1."""
+    import torch
+    out = []
+    for cid, det in ((2, False), (3, False), (4, False), (4, True), (1, True)):
+        wl = si.config(cid)
+        stats = workload_stats(wl)
+        r = Runner(sli, wl, dev, stream, det, "auto")
+        with torch.cuda.stream(stream):
+            step_ms, kern_ms, dk_ms = r.timed(steps, warmup, flush)
+        st = statistics.mean(step_ms)
+        roof_meas = step_roofline_ms(stats, peaks, peaks["bf16_tflops"])
+        roof_nom = step_roofline_ms(stats, peaks, NOMINAL_BF16_TFLOPS)
+        kf = statistics.mean(kern_ms)
+        kflop = fused_algorithmic_flop(wl, r.dk_path, stats["valid"])
+        out.append({
+            "config": cid, "workload": wl.name, "deterministic": det, "dk_path": r.dk_path,
+            "T1": wl.T1, "steps": steps, "warmup": warmup,
+            "ms_per_step": st, "query_tokens_per_s": wl.T1 / (st / 1e3),
+            "tflops_nominal": stats["flop_nom"] / st / 1e9,
+            "tflops_valid": stats["flop_valid"] / st / 1e9,
+            "step_roofline_ms": roof_meas, "step_roofline_frac": roof_meas / st,
+            "step_roofline_frac_nominal_peak": roof_nom / st,
+            "stages_ms": {"fused": kf, "dk": statistics.mean(dk_ms),
+                          "memset_and_work_split": st - kf - statistics.mean(dk_ms)},
+            "fused_valid_slot_tflops": kflop / kf / 1e9,
+            "fused_valid_slot_frac": kflop / kf / 1e9 / peaks["bf16_tflops"],
+            "device_status": r.status(),
+        })
+        del r
+        torch.cuda.empty_cache()
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -239,6 +354,9 @@ def main():
     ap.add_argument("--cpu-baseline-tokens", type=int, default=12000)
     ap.add_argument("--dk-path", default="auto", choices=["auto", "scatter", "keymajor"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the per-config block (the other workloads and deterministic mode)")
+    ap.add_argument("--per-config-steps", type=int, default=10)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -258,77 +376,32 @@ def main():
                                 timeout=__import__("datetime").timedelta(seconds=300))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
+    barrier = dist.barrier if world > 1 else None
 
     wl = si.config(args.config)
     stats = workload_stats(wl)
     stream = torch.cuda.Stream(device=dev)
-    # device-resident inputs
-    q, k, w, p, idx = (getattr(wl, n).to(dev) for n in ("q", "k", "w", "p", "idx"))
-    cuq = wl.cu_seqlens_q.to(dev) if wl.cu_seqlens_q is not None else None
-    cuk = wl.cu_seqlens_k.to(dev) if wl.cu_seqlens_k is not None else None
-    B = wl.B if wl.layout == "TND" else None
-    pr = sli.make_problem(q, k, idx, wl.layout, wl.layout, args.deterministic, B,
-                          sli.key_range_bound_of(wl))
-    base_opt = sli.make_options(args.dk_path)
-    dk_path = "keymajor" if sli.slikl_grad_dk_path(pr, base_opt) == sli.SLIKL_DK_KEYMAJOR else "scatter"
-    nbytes = sli.slikl_grad_workspace_size_ex(pr, base_opt)
-    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
-    out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dw=torch.empty_like(w),
-               softmax_out=torch.empty_like(p))
-
-    def tensors(qq, kk, ww, pp, ii, o):
-        tn = sli.slikl_tensors()
-        tn.q, tn.k, tn.w, tn.attn_softmax_l1norm, tn.sparse_indices = (
-            qq.data_ptr(), kk.data_ptr(), ww.data_ptr(), pp.data_ptr(), ii.data_ptr())
-        tn.cu_seqlens_q = cuq.data_ptr() if cuq is not None else None
-        tn.cu_seqlens_k = cuk.data_ptr() if cuk is not None else None
-        tn.dq, tn.dk, tn.dw, tn.softmax_out = (o["dq"].data_ptr(), o["dk"].data_ptr(),
-                                               o["dw"].data_ptr(), o["softmax_out"].data_ptr())
-        return tn
-
-    tn = tensors(q, k, w, p, idx, out)
+    r = Runner(sli, wl, dev, stream, args.deterministic, args.dk_path)
+    dk_path = r.dk_path
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    sid = stream.cuda_stream
 
-    def step(evs=None):
-        opt = base_opt if evs is None else sli.make_options(args.dk_path, *(int(e) for e in evs))
-        sli.slikl_grad_ex(pr, tn, ws.data_ptr(), nbytes, sid, opt)
-
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    clocks = ClockSampler(vis.split(",")[local] if vis else str(local))
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             flush.fill_(1)
-            step()
+            r.step()
         torch.cuda.synchronize(dev)
-        if world > 1:
-            dist.barrier()
-        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
-        clocks = ClockSampler(vis.split(",")[local] if vis else str(local))
         clocks.start()
         time.sleep(0.3)
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)]
-        kev = [tuple(raw_event() for _ in range(4)) for _ in range(args.steps)]
-        torch.cuda.synchronize(dev)
-        if world > 1:
-            dist.barrier()
-        for i in range(args.steps):
-            flush.fill_(1)
-            ev[i][0].record(stream)
-            step(kev[i])
-            ev[i][1].record(stream)
-        torch.cuda.synchronize(dev)
-        if world > 1:
-            dist.barrier()
-        step_ms = [a.elapsed_time(b) for a, b in ev]
-        kern_ms = [raw_elapsed_ms(e[0], e[1]) for e in kev]
-        dk_ms = [raw_elapsed_ms(e[2], e[3]) for e in kev]
-        flags = sli.slikl_read_device_status(ws.data_ptr(), sid)
+        step_ms, kern_ms, dk_ms = r.timed(args.steps, 0, flush, barrier)
+        flags = r.status()
 
         # end to end through the public API with pinned host buffers
-        hq, hk, hw, hp, hi = (t.cpu().pin_memory() for t in (q, k, w, p, idx))
-        hout = {n: torch.empty(t.shape, dtype=t.dtype).pin_memory() for n, t in out.items()}
-        q2, k2, w2, p2, i2 = (torch.empty_like(t) for t in (q, k, w, p, idx))
-        tn2 = tensors(q2, k2, w2, p2, i2, out)
+        hq, hk, hw, hp, hi = (t.cpu().pin_memory() for t in (r.q, r.k, r.w, r.p, r.idx))
+        hout = {n: torch.empty(t.shape, dtype=t.dtype).pin_memory() for n, t in r.out.items()}
+        q2, k2, w2, p2, i2 = (torch.empty_like(t) for t in (r.q, r.k, r.w, r.p, r.idx))
+        tn2 = r.tensors(q2, k2, w2, p2, i2)
         h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hw, hp, hi))
         d2h = sum(t.numel() * t.element_size() for t in hout.values())
         e2e_ms = []
@@ -338,24 +411,32 @@ def main():
             a.record(stream)
             for dst, src in ((q2, hq), (k2, hk), (w2, hw), (p2, hp), (i2, hi)):
                 dst.copy_(src, non_blocking=True)
-            sli.slikl_grad_ex(pr, tn2, ws.data_ptr(), nbytes, sid, base_opt)
-            for n, t in out.items():
+            r.step(tn=tn2)
+            for n, t in r.out.items():
                 hout[n].copy_(t, non_blocking=True)
             b.record(stream)
             b.synchronize()
             if i >= args.warmup:
                 e2e_ms.append(a.elapsed_time(b))
-        clk = clocks.stop()
+        del hq, hk, hw, hp, hi, hout, q2, k2, w2, p2, i2
+    peaks, peak_src = load_peaks()
+    per_config = None
+    if world == 1 and not args.no_per_config and args.config == 1 and not args.deterministic:
+        del r
+        torch.cuda.empty_cache()
+        per_config = per_config_lines(sli, dev, stream, flush, peaks, args.per_config_steps,
+                                      args.warmup)
+    clk = clocks.stop()
 
     t_total, t_e2e, t_kern, t_dk = combine_over_ranks(
         [sum(step_ms) / 1e3, sum(e2e_ms) / 1e3, sum(kern_ms) / 1e3, sum(dk_ms) / 1e3], world, dev)
     tokens = wl.T1 * args.steps * world
     value = tokens / t_total
-    peaks, peak_src = load_peaks()
     k_avg = t_kern / args.steps
     dk_avg = t_dk / args.steps
     flop = stats["flop_nom"]
-    kflop = fused_algorithmic_flop(wl, dk_path)
+    kflop = fused_algorithmic_flop(wl, dk_path, stats["valid"])
+    kflop_nom = fused_algorithmic_flop(wl, dk_path)
     achieved_tf = kflop / k_avg / 1e12
     peak_tf = peaks["bf16_tflops"]
     traffic = None
@@ -363,7 +444,8 @@ def main():
             and not args.deterministic and fused_sources_hash() == FUSED_TRAFFIC["sources_sha256_16"]):
         traffic = FUSED_TRAFFIC["bytes"]
     step_avg = t_total / args.steps
-    t_roof = max(flop / (peak_tf * 1e12), stats["bytes"] / (peaks["hbm_gbs"] * 1e9))
+    t_roof = step_roofline_ms(stats, peaks, peak_tf) / 1e3
+    t_roof_nom = step_roofline_ms(stats, peaks, NOMINAL_BF16_TFLOPS) / 1e3
     # our kernels per call: 3 work-split + fused + (cast | sort init, 3 per radix pass,
     # row pointers, segmented reduce); the key-major path adds 2 metadata kernels and its dK kernel
     launches_per_step = 5 + (3 if dk_path == "keymajor" else 0)
@@ -391,12 +473,20 @@ def main():
             "tflops_nominal": flop / step_avg / 1e12,
             "tflops_valid": stats["flop_valid"] / step_avg / 1e12,
             "roofline_step": {"t_roof_ms": 1e3 * t_roof, "frac": t_roof / step_avg,
+                              "t_roof_ms_nominal_peak": 1e3 * t_roof_nom,
+                              "frac_nominal_peak": t_roof_nom / step_avg,
                               "flop_nominal": flop, "compulsory_bytes": stats["bytes"],
-                              "peaks": peak_src},
+                              "peaks": f"bf16 {peak_tf} TFLOP/s ({peak_src}); "
+                                       f"nominal {NOMINAL_BF16_TFLOPS} TFLOP/s; "
+                                       f"hbm {peaks['hbm_gbs']} GB/s ({peak_src})"},
             "roofline": {"bound": "tensor", "achieved": achieved_tf, "peak": peak_tf,
                          "unit": "TFLOP/s", "frac": achieved_tf / peak_tf, "traffic": traffic,
                          "kernel": "fused_sm100 (fused per-token kernel)",
                          "algorithmic_flop_per_launch": kflop,
+                         "flop_basis": "valid slots (tiles without a valid slot are skipped)",
+                         "achieved_nominal_slots": kflop_nom / k_avg / 1e12,
+                         "frac_nominal_slots": kflop_nom / k_avg / 1e12 / peak_tf,
+                         "frac_of_nominal_peak": achieved_tf / NOMINAL_BF16_TFLOPS,
                          "peak_source": f"bf16_tflops, burst ({peak_src})"},
             "stages_ms": {"fused": 1e3 * k_avg, "dk": 1e3 * dk_avg,
                           "memset_and_work_split": 1e3 * (step_avg - k_avg - dk_avg)},
@@ -405,6 +495,7 @@ def main():
             "gpu_launches": launches_per_step * args.steps,
             "device_status": flags,
             "clocks": clk,
+            "per_config": per_config,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)

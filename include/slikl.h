@@ -13,7 +13,7 @@
  *   dq_t  = dS_t . K_topk(t)           -> dq
  *   dK_topk(t) = dS_t^T . q_t          scatter-added into the key rows -> dk
  *
- * Invalid top-k slots hold -1 and take no part ("无效top-k位置不参与计算"):
+ * Invalid top-k slots hold -1 and take no part in any of these sums (same section):
  * softmax_out is exactly 0 there and nothing is added for them. A token with no valid
  * slot gets softmax_out = 0 and zero dq/dw. Key rows that no valid slot names get dk = +0.
  *
@@ -286,7 +286,8 @@ SLIKL_API slikl_status slikl_grad_metadata(const slikl_problem *problem, const s
  * (make that first call outside any stream capture). All calls share the array: calls whose
  * GPU work overlaps (unordered streams) race and give wrong results.
  * Errors: as slikl_grad; SLIKL_ERR_WORKSPACE_TOO_SMALL if the problem needs more scratch than
- * SLIKL_NOALLOC_SCRATCH_BYTES (slikl_grad_workspace_size tells how much);
+ * SLIKL_NOALLOC_SCRATCH_BYTES; slikl_grad_workspace_size_ex with options.dk_path =
+ * SLIKL_DK_SCATTER (the path this call takes) tells how much it needs;
  * SLIKL_ERR_PARAM_INVALID for deterministic = 1, whose per-slot scratch does not fit.
  */
 #define SLIKL_NOALLOC_SCRATCH_BYTES (32u << 20)

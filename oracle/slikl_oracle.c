@@ -18,7 +18,7 @@
  * dS is not printed on the page; it follows from I = W . ReLU(S) by the chain rule:
  *   dS[h][j] = dI[j] * w[t,h] * (S[h][j] > 0 ? 1 : 0).
  *
- * Invalid top-k slots (index -1) take no part (same section: "无效top-k位置不参与计算"):
+ * Invalid top-k slots (index -1) take no part in any sum (same section):
  * the softmax runs over the valid slots only, y = 0 and dI = 0 at invalid slots.
  * Valid indices are local to the query's batch (section "公共约束"): key row =
  * k_start[b] + index. A token with no valid slot gets y = 0 and zero gradients.

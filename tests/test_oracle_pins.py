@@ -377,6 +377,25 @@ def test_split_weighted_brute_force():
             assert t == 0 or P[t - 1] * cores < target
 
 
+def golden_split_rows(fx):
+    """Index rows of the hand-worked split fixture: the listed slots valid, the rest -1."""
+    idx = np.full((len(fx["rows_valid_slots"]), fx["topk"]), -1, dtype=np.int32)
+    for t, slots in enumerate(fx["rows_valid_slots"]):
+        for j in slots:
+            idx[t, j] = j % 7
+    return idx
+
+
+def test_split_weighted_hand_worked():
+    """The cost-weighted split against ranges worked out by hand (tests/golden)."""
+    with open(os.path.join(GOLDEN, "split_weighted_hand.json")) as f:
+        fx = json.load(f)
+    idx = golden_split_rows(fx)
+    for case in fx["cases"]:
+        ranges = oracle.split_weighted(idx, case["cores"])
+        assert ranges.tolist() == case["ranges"], case["cores"]
+
+
 # ---------------------------------------------------------------------------
 # used lengths (seqUsedQOptional / seqUsedKOptional: the page fixes only their type; the
 # reading is "rows of each batch in use": query rows past q_used[b] are padding, slots

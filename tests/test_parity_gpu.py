@@ -6,10 +6,9 @@ rel-L2 <= 5e-3 and max-abs <= 2e-2 * max|ref|. Bit-exact: softmax_out = 0 at inv
 slots, dk = 0 on key rows no valid slot names, the work split, and deterministic-mode
 repeats.
 
-Full-size workloads: softmax_out, dw and dq are compared on a sample of tokens (the oracle
-computes any token on its own); dk is compared in full on the same launch shape with every
-token outside the sample masked to -1, which leaves each sampled token's outputs unchanged
-(a pinned invariant of the oracle) and makes the full dk computable by the oracle.
+Full-size workloads (configs 1-4): every token's softmax_out, dw and dq and the full dk are
+compared with one full oracle run of the same workload, on the auto and scatter dK paths and
+(configs 1 and 4) the deterministic reduction.
 """
 
 import json
@@ -160,24 +159,6 @@ def test_keymajor_key_range_bound_too_small_flagged():
     assert flags & sli.SLIKL_DEV_KEY_RANGE_ABOVE_S2
 
 
-def masked(wl, tokens):
-    """Same workload with every token outside `tokens` made all-invalid."""
-    idx = wl.idx.clone().reshape(wl.T1, wl.K)
-    keep = torch.zeros(wl.T1, dtype=torch.bool)
-    keep[torch.from_numpy(np.asarray(tokens))] = True
-    idx[~keep] = -1
-    out = si.Workload(**{f: getattr(wl, f) for f in wl.__dataclass_fields__})
-    out.idx = idx.reshape(wl.idx.shape).contiguous()
-    return out
-
-
-def sample_tokens(wl, n, seed):
-    rng = np.random.default_rng(seed)
-    pick = rng.choice(wl.T1, size=min(n, wl.T1), replace=False)
-    pick = np.union1d(pick, [0, wl.T1 - 1])           # first and last rows always
-    return np.sort(pick)
-
-
 _CFG_CACHE = {}
 
 
@@ -187,25 +168,30 @@ def cfg(cid):
     return _CFG_CACHE[cid]
 
 
-@pytest.mark.parametrize("cid,path", [(1, "auto"), (2, "auto"), (3, "auto"), (4, "auto"),
-                                      (1, "scatter"), (4, "scatter")])
-def test_full_size_sampled_parity(cid, path):
+# dK modes compared in full at each full-size workload: the auto path (key-major where the
+# key range allows it), the scatter path, and the deterministic reduction on configs 1 and 4
+FULL_MODES = {
+    1: [(False, "auto"), (False, "scatter"), (True, "auto")],
+    2: [(False, "auto"), (False, "scatter")],
+    3: [(False, "auto")],
+    4: [(False, "auto"), (False, "scatter"), (True, "auto")],
+}
+
+
+@pytest.mark.parametrize("cid", [1, 2, 3, 4])
+def test_full_size_parity(cid):
+    """Every output of the full-size workload against one full oracle run: softmax_out, dw and
+    dq of every token and the full dk (unmasked: every hot key with all its adds), element by
+    element, on each dK mode; plus the bit-exact zeros."""
     wl = cfg(cid)
-    toks = sample_tokens(wl, 48, seed=cid)
-    ref = oracle.grad(wl, tokens=toks)
-    got = run_gpu(wl, dk_path=path)
-    assert got["flags"] == 0
-    check_exact(wl, got)
-    for name in ("y", "dw", "dq"):
-        assert_close(name, got[name][toks], ref[name][toks])
-    # full dk on the masked problem of the same shape
-    wm = masked(wl, toks)
-    gm = run_gpu(wm, dk_path=path)
-    assert gm["flags"] == 0
-    check_exact(wm, gm)
-    assert_close("dk", gm["dk"], ref["dk"])
-    for name in ("y", "dw", "dq"):
-        assert_close(name, gm[name][toks], ref[name][toks])
+    ref = oracle.grad(wl)
+    for det, path in FULL_MODES[cid]:
+        got = run_gpu(wl, deterministic=det, dk_path=path)
+        assert got["flags"] == 0, (det, path)
+        check_exact(wl, got)
+        check_against(wl, got, ref)
+        del got
+    _CFG_CACHE.pop(cid, None)
 
 
 @pytest.mark.parametrize("cid", [1, 3])
@@ -213,7 +199,7 @@ def test_full_size_identities(cid):
     """Properties that hold at any size, checked on the full GPU outputs:
     sum_d q_hd dq_hd = w_h dW_h per token and head, and
     sum_r <k_r, dk_r> = sum_t,h w_th dW_th."""
-    wl = cfg(cid)
+    wl = si.config(cid)
     got = run_gpu(wl)
     q = wl.q.double().numpy().reshape(wl.T1, wl.N1, wl.D)
     k = wl.k.double().numpy().reshape(wl.T2, wl.D)
@@ -225,8 +211,14 @@ def test_full_size_identities(cid):
     assert abs(total - rhs.sum()) <= 1e-2 * np.abs(rhs).sum()
 
 
-def test_deterministic_bitwise_repeat_config4():
-    wl = cfg(4)
+def bits(t):
+    return t.view(torch.int16) if t.element_size() == 2 else t.view(torch.int32)
+
+
+@pytest.mark.parametrize("cid", [1, 4])
+def test_deterministic_bitwise_repeat(cid):
+    """Deterministic mode: ten calls on the same inputs give bit-identical outputs."""
+    wl = si.config(cid)
     dev = torch.device("cuda")
     t = {n: getattr(wl, n).to(dev) for n in ("q", "k", "w", "p", "idx")}
     first = None
@@ -235,28 +227,12 @@ def test_deterministic_bitwise_repeat_config4():
         res = sli.grad(t["q"], t["k"], t["w"], t["p"], t["idx"], deterministic=True,
                        workspace=ws)
         ws = res["workspace"]
-        cur = [res[n].clone() for n in ("dq", "dk", "dw", "softmax_out")]
+        cur = [bits(res[n]).clone() for n in ("dq", "dk", "dw", "softmax_out")]
         if first is None:
             first = cur
         else:
             for a, b in zip(first, cur):
-                assert torch.equal(a.view(torch.uint8) if a.dtype != torch.float32 else a.view(torch.int32),
-                                   b.view(torch.uint8) if b.dtype != torch.float32 else b.view(torch.int32))
-
-
-def test_deterministic_parity_config4():
-    wl = cfg(4)
-    toks = sample_tokens(wl, 48, seed=44)
-    ref = oracle.grad(wl, tokens=toks)
-    wm = masked(wl, toks)
-    gm = run_gpu(wm, deterministic=True)
-    assert gm["flags"] == 0
-    check_exact(wm, gm)
-    assert_close("dk", gm["dk"], ref["dk"])
-    got = run_gpu(wl, deterministic=True)
-    for name in ("y", "dw", "dq"):
-        assert_close(name, got[name][toks], ref[name][toks])
-    check_exact(wl, got)
+                assert torch.equal(a, b)
 
 
 def test_out_of_range_index_flagged_and_ignored():
@@ -337,6 +313,23 @@ def test_metadata_golden_sample_shapes():
                       D=128, K=4)
         m = metadata_gpu(wl, case["cores"], 0)
         assert list(m[:6]) == case["header"]
+
+
+def test_metadata_weighted_hand_worked():
+    """The device's cost-weighted split (mode 1) on the hand-worked fixture of tests/golden."""
+    with open(os.path.join(GOLDEN, "split_weighted_hand.json")) as f:
+        fx = json.load(f)
+    rows = fx["rows_valid_slots"]
+    wl = si.small(seed=0, layout="BSND", B=1, S1=len(rows), S2=300, N1=8, D=128,
+                  K=fx["topk"], pattern="none")
+    idx = torch.full((len(rows), fx["topk"]), -1, dtype=torch.int32)
+    for t, slots in enumerate(rows):
+        for j in slots:
+            idx[t, j] = j % 7
+    wl.idx = idx.reshape(wl.idx.shape).contiguous()
+    for case in fx["cases"]:
+        m = metadata_gpu(wl, case["cores"], 1)
+        assert m[8:].reshape(case["cores"], 2).tolist() == case["ranges"], case["cores"]
 
 
 @pytest.mark.parametrize("case", [SMALL[0], SMALL[1], SMALL[7], SMALL[8], SMALL[9], SMALL[10]],
