@@ -188,9 +188,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __shared__ Ctl ctl;
     constexpr int kFmt = std::is_same<T, __nv_bfloat16>::value ? 1 : 0;
     constexpr uint32_t kIdescS = idesc_f16(kFmt, 128, N1P, 0, 0);
-    // dq^T [D x 64 heads]: dS^T read MN-major from the [keys x heads] tile (heads past N1P
-    // are zero columns); dK^T [D x 128 keys]: the same tile read K-major
-    constexpr uint32_t kIdescDq = idesc_f16(kFmt, 128, 64, 1, 1);
+    // dq^T [D x N1P heads]: dS^T read MN-major from the [keys x heads] tile; dK^T [D x 128
+    // keys]: the same tile read K-major
+    constexpr uint32_t kIdescDq = idesc_f16(kFmt, 128, N1P, 1, 1);
     constexpr uint32_t kIdescDk = idesc_f16(kFmt, 128, 128, 1, 0);
     constexpr int kDChunks = D / 8;          // 16-byte chunks per key row
     constexpr int kC = N1P < 32 ? N1P : 32;  // S columns per TMEM load
@@ -225,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&bars->sm_sync, 4);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    // zero the dS tiles once: heads past N1P stay 0 (the dq product reads 64 heads)
+    // zero the dS tiles once: heads past N1P stay 0
     for (uint32_t i = threadIdx.x; i < 2 * 16384 / 16; i += kThreads)
         reinterpret_cast<uint4 *>(smem + SP.ds)[i] = make_uint4(0, 0, 0, 0);
     // zero the q buffers once: padded heads and, for D = 64, the upper column block stay 0;
