@@ -182,3 +182,92 @@ def split_weighted(idx: np.ndarray, cores: int) -> np.ndarray:
     _load().oracle_split_weighted(_ptr(idx, ctypes.c_int32), T1, K, cores,
                                   _ptr(ranges, ctypes.c_int64))
     return ranges.reshape(cores, 2)
+
+
+# ---------------------------------------------------------------------------------------------
+# Dense variant (DenseLightningIndexerKLLossGrad)
+#
+# The article on DenseLightningIndexerKLLossGradMetadata (lmnt.cn) names the dense operator and
+# its interface (sections 功能定位, 第一段接口参数说明, 特殊约束): one key head, headDim 128, layouts
+# BSND / TND, maskMode 0 (no mask) or 3 (rightDownCausal: the lower triangle aligned to the
+# bottom-right corner), cmpRatio 1 for uncompressed keys. It prints no formula of its own. The
+# reading taken here: the formulas of aclnnSparseLightningIndexerKLLossGrad (计算公式) with the
+# top-k slots of a query replaced by every key of its batch that the mask leaves visible, slot j
+# being key j of the batch; attn_softmax_l1norm and softmax_out are [T1, Ld] rows with Ld at
+# least the longest key range.
+# ---------------------------------------------------------------------------------------------
+
+def dense_visible(mask_mode: int, s: int, qlen: int, klen: int) -> int:
+    """Keys of a batch visible to its query at local position s: all klen of them with no
+    mask; with the right-down causal mask, keys 0 .. s + (klen - qlen), i.e. the diagonal runs
+    through the last query and the last key (none when that bound is negative)."""
+    if mask_mode == 0:
+        return klen
+    if mask_mode == 3:
+        return min(klen, max(0, s + klen - qlen + 1))
+    raise ValueError("mask_mode must be 0 or 3")
+
+
+def dense_grad_arrays(q: np.ndarray, k: np.ndarray, w: np.ndarray, p: np.ndarray,
+                      q_start: np.ndarray, k_start: np.ndarray, mask_mode: int,
+                      q_used: Optional[Sequence[int]] = None,
+                      k_used: Optional[Sequence[int]] = None) -> dict:
+    """Dense oracle on flat fp64 arrays: q [T1,N1,D], k [T2,D], w [T1,N1], p [T1,Ld];
+    q_start / k_start [B+1]; optional used lengths [B] (rows past them are padding, keys past
+    them are not visible). Plain fp64 per query row: S = q_t K^T over the visible keys, then the
+    sparse operator's formulas. Returns y [T1,Ld], dw, dq, dk [T2,D], loss [T1]."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    p = np.asarray(p, dtype=np.float64)
+    T1, N1, D = q.shape
+    T2 = k.shape[0]
+    Ld = p.shape[1]
+    B = len(q_start) - 1
+    y = np.zeros((T1, Ld))
+    dw = np.zeros((T1, N1))
+    dq = np.zeros((T1, N1, D))
+    dk = np.zeros((T2, D))
+    loss = np.zeros(T1)
+    for b in range(B):
+        q0, q1 = int(q_start[b]), int(q_start[b + 1])
+        k0, k1 = int(k_start[b]), int(k_start[b + 1])
+        qlen = q1 - q0 if q_used is None else int(q_used[b])
+        klen = k1 - k0 if k_used is None else int(k_used[b])
+        for s in range(qlen):
+            t = q0 + s
+            L = dense_visible(mask_mode, s, qlen, klen)
+            if L == 0:
+                continue
+            if L > Ld:
+                raise ValueError("row length below the visible key count")
+            Kv = k[k0:k0 + L]                               # [L, D]
+            S = q[t] @ Kv.T                                 # [N1, L]
+            R = np.maximum(S, 0.0)
+            I = w[t] @ R                                    # [L]
+            e = np.exp(I - I.max())
+            yv = e / e.sum()
+            pv = p[t, :L]
+            dI = yv - pv                                    # dI = Softmax(I) - p
+            y[t, :L] = yv
+            dw[t] = R @ dI                                  # dW = dI . ReLU(S)^T
+            dS = dI[None, :] * w[t][:, None] * (S > 0.0)    # chain rule on I = W . ReLU(S)
+            dq[t] = dS @ Kv                                 # dq = dS . K
+            dk[k0:k0 + L] += dS.T @ q[t]                    # dK = dS^T . q
+            pos = pv > 0.0
+            loss[t] = float(np.sum(pv[pos] * np.log(pv[pos] / yv[pos])))
+    return {"y": y, "dw": dw, "dq": dq, "dk": dk, "loss": loss}
+
+
+def dense_grad(wl, seq_used_q: Optional[Sequence[int]] = None,
+               seq_used_k: Optional[Sequence[int]] = None) -> dict:
+    """Dense oracle on a slikl_inputs.DenseWorkload."""
+    T1, T2, N1, D = wl.T1, wl.T2, wl.N1, wl.D
+    q = wl.q.double().numpy().reshape(T1, N1, D)
+    k = wl.k.double().numpy().reshape(T2, D)
+    w = wl.w.double().numpy().reshape(T1, N1)
+    p = wl.p.double().numpy().reshape(T1, wl.Ld)
+    cuq = None if wl.cu_seqlens_q is None else wl.cu_seqlens_q.numpy()
+    cuk = None if wl.cu_seqlens_k is None else wl.cu_seqlens_k.numpy()
+    qs, ks = row_starts(wl.layout, wl.layout, wl.B, wl.S1, wl.S2, cuq, cuk)
+    return dense_grad_arrays(q, k, w, p, qs, ks, wl.mask_mode, seq_used_q, seq_used_k)

@@ -286,3 +286,98 @@ def small(seed: int, layout: str = "BSND", B: int = 2, S1: int = 40, S2: int = 3
     return _finish(f"small-{layout}-{pattern}", layout, dtype, B, max(lens_q), max(lens_k),
                    [int(x) for x in lens_q], [int(x) for x in lens_k], N1, D, K, qk_scale,
                    w_var, rows, rng)
+
+
+# ----------------------------------------------------------------------------
+# Dense variant inputs (every visible key of the batch is a slot)
+# ----------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class DenseWorkload:
+    """One synthetic dense problem. attn_softmax_l1norm p is [.., 1, Ld]: slot j of a row is
+    key j of its batch; Ld >= the longest key range."""
+
+    name: str
+    layout: str
+    dtype: torch.dtype
+    mask_mode: int              # 0 = no mask, 3 = right-down causal
+    B: int
+    S1: int
+    S2: int
+    T1: int
+    T2: int
+    N1: int
+    D: int
+    Ld: int
+    q: torch.Tensor
+    k: torch.Tensor
+    w: torch.Tensor
+    p: torch.Tensor
+    cu_seqlens_q: Optional[torch.Tensor] = None
+    cu_seqlens_k: Optional[torch.Tensor] = None
+
+
+def _visible_count(mask_mode: int, s: int, qlen: int, klen: int) -> int:
+    # the input's structure (which slots carry target mass): every key with no mask; with the
+    # right-down causal mask the keys up to the diagonal through the last query and key
+    if mask_mode == 0:
+        return klen
+    return min(klen, max(0, s + klen - qlen + 1))
+
+
+def dense_small(seed: int, layout: str = "BSND", B: int = 2, S1: int = 40, S2: int = 300,
+                N1: int = 16, D: int = 128, mask_mode: int = 3,
+                dtype: torch.dtype = torch.bfloat16, qk_scale: float = 0.3,
+                w_var: float = 1.0 / 16, lens_q=None, lens_k=None, Ld: Optional[int] = None,
+                used_q=None, used_k=None) -> DenseWorkload:
+    """A dense problem; p = exp(N(0,1)) normalised over each row's visible keys (the used
+    lengths, when given, decide the visible set), 0 elsewhere."""
+    rng = np.random.default_rng(seed)
+    if layout == "TND":
+        if lens_q is None:
+            lens_q = list(rng.integers(1, S1 + 1, size=B))
+        if lens_k is None:
+            lens_k = list(rng.integers(1, S2 + 1, size=B))
+    else:
+        lens_q = [S1] * B
+        lens_k = [S2] * B
+    lens_q = [int(x) for x in lens_q]
+    lens_k = [int(x) for x in lens_k]
+    T1, T2 = sum(lens_q), sum(lens_k)
+    if Ld is None:
+        Ld = max(lens_k) if lens_k else 1
+    q = rng.standard_normal((T1, N1, D)) * qk_scale
+    k = rng.standard_normal((T2, D)) * qk_scale
+    w = rng.standard_normal((T1, N1)) * np.sqrt(w_var)
+    e = np.exp(rng.standard_normal((T1, Ld)))
+    mask = np.zeros((T1, Ld), dtype=bool)
+    t = 0
+    for b in range(B):
+        qlen = lens_q[b] if used_q is None else int(used_q[b])
+        klen = lens_k[b] if used_k is None else int(used_k[b])
+        for s in range(lens_q[b]):
+            if s < qlen:
+                mask[t, : _visible_count(mask_mode, s, qlen, klen)] = True
+            t += 1
+    e = np.where(mask, e, 0.0)
+    tot = e.sum(axis=-1, keepdims=True)
+    p = (e / np.where(tot > 0, tot, 1.0)).astype(np.float32)
+    qt, kt = _round(q, dtype), _round(k, dtype)
+    wt, pt = torch.from_numpy(w.astype(np.float32)), torch.from_numpy(p)
+    if layout == "BSND":
+        qt = qt.reshape(B, S1, N1, D)
+        kt = kt.reshape(B, S2, 1, D)
+        wt = wt.reshape(B, S1, N1)
+        pt = pt.reshape(B, S1, 1, Ld)
+        cuq = cuk = None
+    else:
+        qt = qt.reshape(T1, N1, D)
+        kt = kt.reshape(T2, 1, D)
+        pt = pt.reshape(T1, 1, Ld)
+        cuq = torch.tensor(np.concatenate([[0], np.cumsum(lens_q)]), dtype=torch.int32)
+        cuk = torch.tensor(np.concatenate([[0], np.cumsum(lens_k)]), dtype=torch.int32)
+    return DenseWorkload(name=f"dense-{layout}-mask{mask_mode}", layout=layout, dtype=dtype,
+                         mask_mode=mask_mode, B=B, S1=max(lens_q) if lens_q else 0,
+                         S2=max(lens_k) if lens_k else 0, T1=T1, T2=T2, N1=N1, D=D, Ld=Ld,
+                         q=qt.contiguous(), k=kt.contiguous(), w=wt.contiguous(),
+                         p=pt.contiguous(), cu_seqlens_q=cuq, cu_seqlens_k=cuk)
