@@ -149,8 +149,8 @@ def raw_elapsed_ms(a, b):
 # ncu capture of that launch (dram__bytes_read.sum + dram__bytes_write.sum). The figure holds
 # only while the kernel's sources are the ones captured (hash of the three files below);
 # otherwise the traffic is reported as unknown (null).
-FUSED_TRAFFIC = {"sources_sha256_16": "c4172c992f118d38", "workload_config": 1,
-                 "dk_path": "keymajor", "bytes": 120.852736e6 + 193.821952e6}
+FUSED_TRAFFIC = {"sources_sha256_16": "585d0d6c2ddf69bf", "workload_config": 1,
+                 "dk_path": "keymajor", "bytes": 121.169152e6 + 193.834496e6}
 
 
 def fused_sources_hash():
@@ -302,20 +302,78 @@ class Runner:
         return self.sli.slikl_read_device_status(self.ws.data_ptr(), self.stream.cuda_stream)
 
 
+class DenseRunner(Runner):
+    """The dense variant's workload resident on the device, called through slikl_dense_grad
+    on `stream` (timing, flush and status as Runner)."""
+
+    def __init__(self, sli, wl, dev, stream, deterministic, dk_path):
+        import torch
+        self.sli, self.wl, self.dev, self.stream = sli, wl, dev, stream
+        self.q, self.k, self.w, self.p = (getattr(wl, n).to(dev) for n in ("q", "k", "w", "p"))
+        self.cuq = wl.cu_seqlens_q.to(dev) if wl.cu_seqlens_q is not None else None
+        self.cuk = wl.cu_seqlens_k.to(dev) if wl.cu_seqlens_k is not None else None
+        B = wl.B if wl.layout == "TND" else None
+        self.pr = sli.make_dense_problem(self.q, self.k, self.p, wl.layout, wl.layout,
+                                         wl.mask_mode, deterministic, B)
+        self.dk_path_arg = dk_path
+        self.opt = sli.make_options(dk_path)
+        self.dk_path = ("keymajor" if sli.slikl_dense_grad_dk_path(self.pr, self.opt)
+                        == sli.SLIKL_DK_KEYMAJOR else "scatter")
+        self.nbytes = sli.slikl_dense_grad_workspace_size(self.pr, self.opt)
+        self.ws = torch.empty(self.nbytes, dtype=torch.uint8, device=dev)
+        self.out = dict(dq=torch.empty_like(self.q), dk=torch.empty_like(self.k),
+                        dw=torch.empty_like(self.w), softmax_out=torch.empty_like(self.p))
+        tn = sli.slikl_dense_tensors()
+        tn.q, tn.k, tn.w, tn.attn_softmax_l1norm = (self.q.data_ptr(), self.k.data_ptr(),
+                                                    self.w.data_ptr(), self.p.data_ptr())
+        tn.cu_seqlens_q = self.cuq.data_ptr() if self.cuq is not None else None
+        tn.cu_seqlens_k = self.cuk.data_ptr() if self.cuk is not None else None
+        o = self.out
+        tn.dq, tn.dk, tn.dw, tn.softmax_out = (o["dq"].data_ptr(), o["dk"].data_ptr(),
+                                               o["dw"].data_ptr(), o["softmax_out"].data_ptr())
+        self.tn = tn
+
+    def step(self, evs=None, tn=None):
+        opt = self.opt if evs is None else self.sli.make_options(self.dk_path_arg,
+                                                                 *(int(e) for e in evs))
+        self.sli.slikl_dense_grad(self.pr, tn or self.tn, self.ws.data_ptr(), self.nbytes,
+                                  self.stream.cuda_stream, opt)
+
+
+def dense_stats(wl):
+    """workload_stats for a dense problem: the slots are the Ld positions of every query row,
+    the valid ones those the mask leaves visible; the compulsory bytes are every key row once,
+    q, w, p, softmax_out, dw, dq, dk and the fp32 dK workspace (no index rows: a dense caller
+    passes none)."""
+    T1, T2, N1, D, Ld = wl.T1, wl.T2, wl.N1, wl.D, wl.Ld
+    valid = si.dense_visible_slots(wl)
+    el = 2
+    bytes_comp = (T2 * D * el + T1 * N1 * D * el + T1 * N1 * 4 + T1 * Ld * 4
+                  + T1 * Ld * 4 + T1 * N1 * 4 + T1 * N1 * D * el + T2 * D * el + T2 * D * 4)
+    return dict(valid=valid, flop_nom=6.0 * N1 * Ld * D * T1, flop_valid=6.0 * N1 * D * valid,
+                bytes=bytes_comp, uniq_rows=T2)
+
+
 def step_roofline_ms(stats, peaks, peak_tf):
     return 1e3 * max(stats["flop_nom"] / (peak_tf * 1e12), stats["bytes"] / (peaks["hbm_gbs"] * 1e9))
 
 
 def per_config_lines(sli, dev, stream, flush, peaks, steps, warmup):
     """The other full-size workloads, timed the same way as the headline (device time, L2
-    flushed before every step): configs 2, 3 and 4 on the auto dK path, and the
-    deterministic reduction on configs 4 and 1."""
+    flushed before every step): configs 2, 3 and 4 on the auto dK path, the deterministic
+    reduction on configs 4 and 1, and the dense variant's causal workload in both modes."""
     import torch
     out = []
-    for cid, det in ((2, False), (3, False), (4, False), (4, True), (1, True)):
-        wl = si.config(cid)
-        stats = workload_stats(wl)
-        r = Runner(sli, wl, dev, stream, det, "auto")
+    for cid, det in ((2, False), (3, False), (4, False), (4, True), (1, True), ("dense", False),
+                     ("dense", True)):
+        if cid == "dense":
+            wl = si.dense_full()
+            stats = dense_stats(wl)
+            r = DenseRunner(sli, wl, dev, stream, det, "auto")
+        else:
+            wl = si.config(cid)
+            stats = workload_stats(wl)
+            r = Runner(sli, wl, dev, stream, det, "auto")
         with torch.cuda.stream(stream):
             step_ms, kern_ms, dk_ms = r.timed(steps, warmup, flush)
         st = statistics.mean(step_ms)

@@ -294,6 +294,80 @@ SLIKL_API slikl_status slikl_grad_metadata(const slikl_problem *problem, const s
 SLIKL_API slikl_status slikl_grad_noalloc(const slikl_problem *problem,
                                           const slikl_tensors *tensors, void *stream);
 
+/*
+ * Dense variant (DenseLightningIndexerKLLossGrad). The article on that operator's metadata
+ * generator (sections 功能定位, 第一段接口参数说明 and 特殊约束) names the operator and its
+ * interface: one key head, layouts BSND / TND, maskMode 0 (no mask) or 3 (rightDownCausal, the
+ * lower triangle anchored at the bottom-right vertex), cmpRatio 1 for uncompressed keys. The
+ * pages print no formula of its own. This library reads it as the formulas at the top of this
+ * header, with the top-k slots of a query replaced by every key of its batch that the mask
+ * leaves visible; slot j of a row is key j, local to the batch:
+ *   mask_mode 0: all klen keys of the batch;
+ *   mask_mode 3: query s (0-based, of qlen queries) sees keys 0 .. s + (klen - qlen), none when
+ *                that bound is negative.
+ * With options->seq_used_q / seq_used_k the used lengths stand for qlen / klen; rows past a
+ * batch's used queries are padding (outputs 0).
+ *
+ * attn_softmax_l1norm and softmax_out are [B,S1,1,Ld] (BSND) / [T1,1,Ld] (TND) with
+ * Ld = row_len slots per row; slots past a row's visible keys are invalid (p there is ignored,
+ * softmax_out is exactly 0). q, k, w, dq, dk, dw and cu_seqlens are as in slikl_tensors.
+ * The call runs the sparse operator's kernels on index rows 0, 1, .., L_t - 1 (then -1) that a
+ * device kernel writes into the workspace, so every dK path and option of slikl_grad_ex
+ * applies (options->loss included).
+ */
+typedef struct {
+    int32_t dtype;           /* SLIKL_FP16 or SLIKL_BF16 */
+    int32_t layout_q;        /* SLIKL_BSND or SLIKL_TND */
+    int32_t layout_k;        /* SLIKL_BSND or SLIKL_TND */
+    int32_t deterministic;   /* 0 or 1 */
+    int64_t B, S1, S2;       /* as in slikl_problem (TND keys: S2 = 0 or a key-range bound) */
+    int64_t T1, T2;          /* TND total query / key rows */
+    int64_t N1, D;           /* query heads, head dim */
+    int64_t row_len;         /* Ld, slots per row, in [1, 8192]; 0 = S2 (BSND keys only). Must
+                                cover the longest key range in use; keys of a batch past it are
+                                left out and SLIKL_DEV_ROW_LEN_BELOW_KEYS is set */
+    int32_t mask_mode;       /* 0 or 3 */
+    int32_t reserved;        /* must be 0 */
+} slikl_dense_problem;
+
+typedef struct {
+    const void *q;                      /* dtype  [B,S1,N1,D] / [T1,N1,D]             */
+    const void *k;                      /* dtype  [B,S2,1,D]  / [T2,1,D]              */
+    const float *w;                     /* fp32   [B,S1,N1]   / [T1,N1]               */
+    const float *attn_softmax_l1norm;   /* fp32   [.., 1, Ld] target distribution p    */
+    const int32_t *cu_seqlens_q;        /* int32  [B+1], TND query side only, else NULL */
+    const int32_t *cu_seqlens_k;        /* int32  [B+1], TND key side only, else NULL   */
+    void *dq;                           /* out dtype  same shape as q                   */
+    void *dk;                           /* out dtype  same shape as k                   */
+    float *dw;                          /* out fp32   same shape as w                   */
+    float *softmax_out;                 /* out fp32   [.., 1, Ld]                       */
+} slikl_dense_tensors;
+
+#define SLIKL_DEV_ROW_LEN_BELOW_KEYS  0x40u /* dense variant: a batch holds more keys than
+                                               row_len; the keys past it were left out  */
+
+/*
+ * Two-phase dense call, the same contract as slikl_grad_workspace_size_ex / slikl_grad_ex
+ * (options may be NULL). Errors: as those calls; SLIKL_ERR_PARAM_INVALID also for mask_mode
+ * not 0 or 3, reserved != 0, row_len outside [1, 8192] (after 0 -> S2), or row_len < S2 with
+ * BSND keys.
+ */
+SLIKL_API slikl_status slikl_dense_grad_workspace_size(const slikl_dense_problem *problem,
+                                                       const slikl_options *options,
+                                                       size_t *workspace_bytes);
+SLIKL_API slikl_status slikl_dense_grad(const slikl_dense_problem *problem,
+                                        const slikl_dense_tensors *tensors, void *workspace,
+                                        size_t workspace_bytes, void *stream,
+                                        const slikl_options *options);
+
+/*
+ * The dK path slikl_dense_grad would take for `problem` with `options` (NULL = SLIKL_DK_AUTO):
+ * writes SLIKL_DK_SCATTER or SLIKL_DK_KEYMAJOR to *path. Host only, no CUDA call.
+ * Errors: SLIKL_ERR_INNER_NULLPTR (path NULL) and those of slikl_dense_grad_workspace_size.
+ */
+SLIKL_API slikl_status slikl_dense_grad_dk_path(const slikl_dense_problem *problem,
+                                                const slikl_options *options, int32_t *path);
+
 /* Human-readable name of a status code (static string, never NULL). */
 SLIKL_API const char *slikl_status_string(slikl_status status);
 

@@ -329,7 +329,7 @@ def dense_small(seed: int, layout: str = "BSND", B: int = 2, S1: int = 40, S2: i
                 N1: int = 16, D: int = 128, mask_mode: int = 3,
                 dtype: torch.dtype = torch.bfloat16, qk_scale: float = 0.3,
                 w_var: float = 1.0 / 16, lens_q=None, lens_k=None, Ld: Optional[int] = None,
-                used_q=None, used_k=None) -> DenseWorkload:
+                used_q=None, used_k=None, name: Optional[str] = None) -> DenseWorkload:
     """A dense problem; p = exp(N(0,1)) normalised over each row's visible keys (the used
     lengths, when given, decide the visible set), 0 elsewhere."""
     rng = np.random.default_rng(seed)
@@ -376,8 +376,30 @@ def dense_small(seed: int, layout: str = "BSND", B: int = 2, S1: int = 40, S2: i
         pt = pt.reshape(T1, 1, Ld)
         cuq = torch.tensor(np.concatenate([[0], np.cumsum(lens_q)]), dtype=torch.int32)
         cuk = torch.tensor(np.concatenate([[0], np.cumsum(lens_k)]), dtype=torch.int32)
-    return DenseWorkload(name=f"dense-{layout}-mask{mask_mode}", layout=layout, dtype=dtype,
+    return DenseWorkload(name=name or f"dense-{layout}-mask{mask_mode}", layout=layout, dtype=dtype,
                          mask_mode=mask_mode, B=B, S1=max(lens_q) if lens_q else 0,
                          S2=max(lens_k) if lens_k else 0, T1=T1, T2=T2, N1=N1, D=D, Ld=Ld,
                          q=qt.contiguous(), k=kt.contiguous(), w=wt.contiguous(),
                          p=pt.contiguous(), cu_seqlens_q=cuq, cu_seqlens_k=cuk)
+
+
+DENSE_FULL_NAME = "dense-causal-bsnd B1 S4096 N1=64 D128 mask3 bf16"
+
+
+def dense_full(seed: int = SEED_BASE + 100) -> DenseWorkload:
+    """The full-size dense problem: one batch of 4096 queries over 4096 keys under the
+    right-down causal mask (query s sees keys 0..s), N1 = 64, D = 128, bf16, row length 4096;
+    values drawn like the causal sparse workload's (q, k scaled by 0.1, w of variance 1/64)."""
+    return dense_small(seed, "BSND", 1, 4096, 4096, 64, 128, 3, torch.bfloat16, 0.1, 1.0 / 64,
+                       name=DENSE_FULL_NAME)
+
+
+def dense_visible_slots(wl: DenseWorkload) -> int:
+    """Number of (query row, key) pairs that the mask leaves visible (the slots in use)."""
+    if wl.layout == "TND":
+        lq = np.diff(wl.cu_seqlens_q.numpy())
+        lk = np.diff(wl.cu_seqlens_k.numpy())
+    else:
+        lq, lk = [wl.S1] * wl.B, [wl.S2] * wl.B
+    return int(sum(min(_visible_count(wl.mask_mode, s, int(a), int(b)), wl.Ld)
+                   for a, b in zip(lq, lk) for s in range(int(a))))

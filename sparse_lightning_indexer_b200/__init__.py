@@ -37,6 +37,7 @@ SLIKL_DEV_BAD_CU_SEQLENS_K = 0x4
 SLIKL_DEV_WAIT_TIMEOUT = 0x8
 SLIKL_DEV_KEY_RANGE_ABOVE_S2 = 0x10
 SLIKL_DEV_BAD_SEQ_USED = 0x20
+SLIKL_DEV_ROW_LEN_BELOW_KEYS = 0x40
 
 SLIKL_DK_AUTO = 0
 SLIKL_DK_SCATTER = 1
@@ -47,7 +48,8 @@ EXPORTED = ("slikl_grad_workspace_size", "slikl_grad", "slikl_grad_with_events",
             "slikl_grad_workspace_size_ex", "slikl_grad_ex", "slikl_grad_dk_path",
             "slikl_read_device_status",
             "slikl_grad_metadata_size", "slikl_grad_metadata_workspace_size",
-            "slikl_grad_metadata", "slikl_status_string", "slikl_grad_noalloc")
+            "slikl_grad_metadata", "slikl_status_string", "slikl_grad_noalloc",
+            "slikl_dense_grad_workspace_size", "slikl_dense_grad", "slikl_dense_grad_dk_path")
 
 SLIKL_NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -64,6 +66,21 @@ class slikl_tensors(ctypes.Structure):
     _fields_ = [(name, ctypes.c_void_p) for name in
                 ("q", "k", "w", "attn_softmax_l1norm", "sparse_indices", "cu_seqlens_q",
                  "cu_seqlens_k", "dq", "dk", "dw", "softmax_out")]
+
+
+class slikl_dense_problem(ctypes.Structure):
+    _fields_ = [("dtype", ctypes.c_int32), ("layout_q", ctypes.c_int32),
+                ("layout_k", ctypes.c_int32), ("deterministic", ctypes.c_int32),
+                ("B", ctypes.c_int64), ("S1", ctypes.c_int64), ("S2", ctypes.c_int64),
+                ("T1", ctypes.c_int64), ("T2", ctypes.c_int64), ("N1", ctypes.c_int64),
+                ("D", ctypes.c_int64), ("row_len", ctypes.c_int64), ("mask_mode", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
+class slikl_dense_tensors(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_void_p) for name in
+                ("q", "k", "w", "attn_softmax_l1norm", "cu_seqlens_q", "cu_seqlens_k", "dq",
+                 "dk", "dw", "softmax_out")]
 
 
 class slikl_options(ctypes.Structure):
@@ -126,6 +143,15 @@ def load_library() -> ctypes.CDLL:
                                             ctypes.c_int32, VP, VP, ctypes.c_size_t, VP]
         lib.slikl_grad_noalloc.argtypes = [P(slikl_problem), P(slikl_tensors), VP]
         lib.slikl_grad_noalloc.restype = ctypes.c_int32
+        lib.slikl_dense_grad_workspace_size.argtypes = [P(slikl_dense_problem), P(slikl_options),
+                                                        P(ctypes.c_size_t)]
+        lib.slikl_dense_grad_workspace_size.restype = ctypes.c_int32
+        lib.slikl_dense_grad.argtypes = [P(slikl_dense_problem), P(slikl_dense_tensors), VP,
+                                         ctypes.c_size_t, VP, P(slikl_options)]
+        lib.slikl_dense_grad.restype = ctypes.c_int32
+        lib.slikl_dense_grad_dk_path.argtypes = [P(slikl_dense_problem), P(slikl_options),
+                                                 P(ctypes.c_int32)]
+        lib.slikl_dense_grad_dk_path.restype = ctypes.c_int32
         lib.slikl_status_string.argtypes = [ctypes.c_int32]
         lib.slikl_status_string.restype = ctypes.c_char_p
         for name in ("slikl_grad_workspace_size", "slikl_grad", "slikl_grad_with_events",
@@ -213,6 +239,39 @@ def slikl_grad_noalloc(problem: slikl_problem, tensors: slikl_tensors, stream: i
     rc = load_library().slikl_grad_noalloc(ctypes.byref(problem), ctypes.byref(tensors), stream)
     if rc != SLIKL_OK:
         raise SliklError(rc, "slikl_grad_noalloc")
+
+
+def slikl_dense_grad_workspace_size(problem: slikl_dense_problem,
+                                    options: Optional[slikl_options] = None) -> int:
+    n = ctypes.c_size_t(0)
+    rc = load_library().slikl_dense_grad_workspace_size(
+        ctypes.byref(problem), ctypes.byref(options) if options is not None else None,
+        ctypes.byref(n))
+    if rc != SLIKL_OK:
+        raise SliklError(rc, "slikl_dense_grad_workspace_size")
+    return int(n.value)
+
+
+def slikl_dense_grad_dk_path(problem: slikl_dense_problem,
+                             options: Optional[slikl_options] = None) -> int:
+    """SLIKL_DK_SCATTER or SLIKL_DK_KEYMAJOR: the dK path slikl_dense_grad would take."""
+    v = ctypes.c_int32(0)
+    rc = load_library().slikl_dense_grad_dk_path(
+        ctypes.byref(problem), ctypes.byref(options) if options is not None else None,
+        ctypes.byref(v))
+    if rc != SLIKL_OK:
+        raise SliklError(rc, "slikl_dense_grad_dk_path")
+    return int(v.value)
+
+
+def slikl_dense_grad(problem: slikl_dense_problem, tensors: slikl_dense_tensors, workspace: int,
+                     workspace_bytes: int, stream: int = 0,
+                     options: Optional[slikl_options] = None) -> None:
+    rc = load_library().slikl_dense_grad(ctypes.byref(problem), ctypes.byref(tensors), workspace,
+                                         workspace_bytes, stream,
+                                         ctypes.byref(options) if options is not None else None)
+    if rc != SLIKL_OK:
+        raise SliklError(rc, "slikl_dense_grad")
 
 
 def slikl_grad_metadata_size(num_workers: int) -> int:
@@ -353,3 +412,69 @@ def grad_workload(wl, device="cuda", deterministic=False, stream=None, dk_path="
                 deterministic=deterministic, stream=stream, dk_path=dk_path,
                 key_range_bound=key_range_bound_of(wl), loss=loss, seq_used_q=uq,
                 seq_used_k=uk)
+
+
+def make_dense_problem(q: torch.Tensor, k: torch.Tensor, p: torch.Tensor, layout_q: str = "BSND",
+                       layout_k: str = "BSND", mask_mode: int = 3, deterministic: bool = False,
+                       B: Optional[int] = None, key_range_bound: int = 0) -> slikl_dense_problem:
+    """Dense problem struct from tensor shapes; the row length is p's last dimension."""
+    sp = make_problem(q, k, p, layout_q, layout_k, deterministic, B, key_range_bound)
+    pr = slikl_dense_problem()
+    for f in ("dtype", "layout_q", "layout_k", "deterministic", "B", "S1", "S2", "T1", "T2",
+              "N1", "D"):
+        setattr(pr, f, getattr(sp, f))
+    pr.row_len = p.shape[-1]
+    pr.mask_mode = mask_mode
+    pr.reserved = 0
+    return pr
+
+
+def dense_grad(q, k, w, attn_softmax_l1norm, layout_q="BSND", layout_k="BSND", cu_seqlens_q=None,
+               cu_seqlens_k=None, mask_mode=3, deterministic=False, stream=None, out=None,
+               workspace=None, dk_path="auto", loss=False, seq_used_q=None, seq_used_k=None):
+    """Run slikl_dense_grad on CUDA tensors (p and the returned softmax_out are [.., 1, Ld]).
+    Returns dict(dq, dk, dw, softmax_out, workspace[, loss])."""
+    B = None
+    if layout_q == "TND":
+        B = cu_seqlens_q.numel() - 1
+    elif layout_k == "TND":
+        B = cu_seqlens_k.numel() - 1
+    pr = make_dense_problem(q, k, attn_softmax_l1norm, layout_q, layout_k, mask_mode,
+                            deterministic, B)
+    loss_t = torch.empty(pr.T1, dtype=torch.float32, device=q.device) if loss else None
+    opt = make_options(dk_path, loss=loss_t.data_ptr() if loss_t is not None else 0,
+                       seq_used_q=_ptr(seq_used_q) or 0, seq_used_k=_ptr(seq_used_k) or 0)
+    nbytes = slikl_dense_grad_workspace_size(pr, opt)
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dw=torch.empty_like(w),
+                   softmax_out=torch.empty_like(attn_softmax_l1norm))
+    tn = slikl_dense_tensors()
+    tn.q, tn.k, tn.w = _ptr(q), _ptr(k), _ptr(w)
+    tn.attn_softmax_l1norm = _ptr(attn_softmax_l1norm)
+    tn.cu_seqlens_q = _ptr(cu_seqlens_q) if layout_q == "TND" else None
+    tn.cu_seqlens_k = _ptr(cu_seqlens_k) if layout_k == "TND" else None
+    tn.dq, tn.dk, tn.dw = _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dw"])
+    tn.softmax_out = _ptr(out["softmax_out"])
+    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+    slikl_dense_grad(pr, tn, workspace.data_ptr(), workspace.numel(), s.cuda_stream, opt)
+    res = dict(out)
+    res["workspace"] = workspace
+    if loss_t is not None:
+        res["loss"] = loss_t
+    return res
+
+
+def dense_grad_workload(wl, device="cuda", deterministic=False, stream=None, dk_path="auto",
+                        loss=False, seq_used_q=None, seq_used_k=None):
+    """Move a slikl_inputs.DenseWorkload to the device and run dense_grad()."""
+    dev = torch.device(device)
+    t = {n: getattr(wl, n).to(dev) for n in ("q", "k", "w", "p")}
+    cuq = wl.cu_seqlens_q.to(dev) if wl.cu_seqlens_q is not None else None
+    cuk = wl.cu_seqlens_k.to(dev) if wl.cu_seqlens_k is not None else None
+    uq = None if seq_used_q is None else torch.tensor(list(seq_used_q), dtype=torch.int32, device=dev)
+    uk = None if seq_used_k is None else torch.tensor(list(seq_used_k), dtype=torch.int32, device=dev)
+    return dense_grad(t["q"], t["k"], t["w"], t["p"], wl.layout, wl.layout, cuq, cuk,
+                      mask_mode=wl.mask_mode, deterministic=deterministic, stream=stream,
+                      dk_path=dk_path, loss=loss, seq_used_q=uq, seq_used_k=uk)

@@ -182,7 +182,52 @@ slikl_status check_tensors(const slikl_problem *pr, const slikl_tensors *tn, boo
     return SLIKL_OK;
 }
 
+// The sparse problem a dense one runs as (reading in include/slikl.h): topk = the row length,
+// and for TND keys the row length is the key-range bound the key-major path may assume.
+slikl_status dense_to_sparse(const slikl_dense_problem *d, slikl_problem *sp, int64_t *ld_out) {
+    if (!d) return SLIKL_ERR_PARAM_NULLPTR;
+    if ((d->mask_mode != 0 && d->mask_mode != 3) || d->reserved != 0) return SLIKL_ERR_PARAM_INVALID;
+    int64_t ld = d->row_len;
+    if (ld == 0 && d->layout_k == SLIKL_BSND) ld = d->S2;
+    if (ld < 1 || ld > 8192) return SLIKL_ERR_PARAM_INVALID;
+    if (d->layout_k == SLIKL_BSND && ld < d->S2) return SLIKL_ERR_PARAM_INVALID;
+    memset(sp, 0, sizeof(*sp));
+    sp->dtype = d->dtype;
+    sp->layout_q = d->layout_q;
+    sp->layout_k = d->layout_k;
+    sp->deterministic = d->deterministic;
+    sp->B = d->B;
+    sp->S1 = d->S1;
+    sp->S2 = d->layout_k == SLIKL_BSND ? d->S2 : ld;
+    sp->T1 = d->T1;
+    sp->T2 = d->T2;
+    sp->N1 = d->N1;
+    sp->D = d->D;
+    sp->topk = ld;
+    *ld_out = ld;
+    return SLIKL_OK;
+}
+
+// Dense workspace: the sparse call's workspace first (its status word at offset 0), then the
+// index rows [T1][Ld] int32, then one word for the dense kernel's flag.
+struct DenseLayout {
+    size_t sparse, idx, flag, total;
+};
+
 }  // namespace
+
+slikl_status dense_layout(const slikl_problem *sp, const slikl_options *options, int64_t ld,
+                          DenseLayout *L) {
+    size_t sparse = 0;
+    slikl_status st = slikl_grad_workspace_size_ex(sp, options, &sparse);
+    if (st != SLIKL_OK) return st;
+    const int64_t T1 = sp->layout_q == SLIKL_BSND ? sp->B * sp->S1 : sp->T1;
+    L->sparse = sparse;
+    L->idx = align256(sparse);
+    L->flag = align256(L->idx + sizeof(int32_t) * (size_t)T1 * (size_t)ld);
+    L->total = L->flag + 256;
+    return SLIKL_OK;
+}
 }  // namespace slikl
 
 using namespace slikl;
@@ -360,6 +405,83 @@ const char *slikl_status_string(slikl_status status) {
         case SLIKL_ERR_CUDA: return "SLIKL_ERR_CUDA: CUDA runtime error or no sm_100 device";
         default: return "unknown slikl status";
     }
+}
+
+
+slikl_status slikl_dense_grad_workspace_size(const slikl_dense_problem *problem,
+                                             const slikl_options *options,
+                                             size_t *workspace_bytes) {
+    if (!workspace_bytes) return SLIKL_ERR_INNER_NULLPTR;
+    slikl_problem sp;
+    int64_t ld = 0;
+    slikl_status st = dense_to_sparse(problem, &sp, &ld);
+    if (st != SLIKL_OK) return st;
+    DenseLayout L;
+    st = dense_layout(&sp, options, ld, &L);
+    if (st != SLIKL_OK) return st;
+    *workspace_bytes = L.total;
+    return SLIKL_OK;
+}
+
+slikl_status slikl_dense_grad_dk_path(const slikl_dense_problem *problem,
+                                      const slikl_options *options, int32_t *path) {
+    slikl_problem sp;
+    int64_t ld = 0;
+    slikl_status st = dense_to_sparse(problem, &sp, &ld);
+    if (st != SLIKL_OK) return st;
+    return slikl_grad_dk_path(&sp, options, path);
+}
+
+slikl_status slikl_dense_grad(const slikl_dense_problem *problem,
+                              const slikl_dense_tensors *tensors, void *workspace,
+                              size_t workspace_bytes, void *stream,
+                              const slikl_options *options) {
+    slikl_problem sp;
+    int64_t ld = 0;
+    slikl_status st = dense_to_sparse(problem, &sp, &ld);
+    if (st != SLIKL_OK) return st;
+    DenseLayout L;
+    st = dense_layout(&sp, options, ld, &L);
+    if (st != SLIKL_OK) return st;
+    if (!tensors) return SLIKL_ERR_PARAM_NULLPTR;
+    if (!workspace) return SLIKL_ERR_PARAM_NULLPTR;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255) return SLIKL_ERR_PARAM_INVALID;
+    if (workspace_bytes < L.total) return SLIKL_ERR_WORKSPACE_TOO_SMALL;
+    char *ws = static_cast<char *>(workspace);
+    slikl_tensors tn;
+    tn.q = tensors->q;
+    tn.k = tensors->k;
+    tn.w = tensors->w;
+    tn.attn_softmax_l1norm = tensors->attn_softmax_l1norm;
+    tn.sparse_indices = reinterpret_cast<const int32_t *>(ws + L.idx);
+    tn.cu_seqlens_q = tensors->cu_seqlens_q;
+    tn.cu_seqlens_k = tensors->cu_seqlens_k;
+    tn.dq = tensors->dq;
+    tn.dk = tensors->dk;
+    tn.dw = tensors->dw;
+    tn.softmax_out = tensors->softmax_out;
+    // every host-side check of the sparse call first, so that nothing is launched for a call
+    // that the sparse entry point would reject
+    Derived dv;
+    st = validate(&sp, &dv);
+    if (st != SLIKL_OK) return st;
+    st = check_tensors(&sp, &tn, true);
+    if (st != SLIKL_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t *flag = reinterpret_cast<uint32_t *>(ws + L.flag);
+    if (cudaMemsetAsync(flag, 0, 4, s) != cudaSuccess) return SLIKL_ERR_CUDA;
+    if (launch_dense_indices(reinterpret_cast<int32_t *>(ws + L.idx), dv.T1, sp.B,
+                             sp.layout_q == SLIKL_BSND ? sp.S1 : 0,
+                             sp.layout_k == SLIKL_BSND ? sp.S2 : 0, (int)ld, sp.layout_q,
+                             sp.layout_k, problem->mask_mode, tn.cu_seqlens_q, tn.cu_seqlens_k,
+                             options ? options->seq_used_q : nullptr,
+                             options ? options->seq_used_k : nullptr, flag, s) != cudaSuccess)
+        return SLIKL_ERR_CUDA;
+    st = slikl_grad_ex(&sp, &tn, workspace, L.sparse, stream, options);
+    if (st != SLIKL_OK) return st;
+    if (launch_dense_flag_merge(flag, reinterpret_cast<uint32_t *>(ws), s) != cudaSuccess)
+        return SLIKL_ERR_CUDA;
+    return SLIKL_OK;
 }
 
 }  // extern "C"

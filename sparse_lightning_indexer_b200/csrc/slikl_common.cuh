@@ -150,5 +150,10 @@ cudaError_t launch_cast(const Params &P, cudaStream_t s);
 cudaError_t launch_deterministic_reduce(const Params &P, cudaStream_t s);
 cudaError_t launch_km_metadata(const Params &P, int workers, cudaStream_t s);
 cudaError_t launch_dk_keymajor(const Params &P, int workers, cudaStream_t s);
+cudaError_t launch_dense_indices(int32_t *idx, int64_t T1, int64_t B, int64_t S1, int64_t S2,
+                                 int Ld, int layout_q, int layout_k, int mask,
+                                 const int32_t *cu_q, const int32_t *cu_k, const int32_t *used_q,
+                                 const int32_t *used_k, uint32_t *flag, cudaStream_t s);
+cudaError_t launch_dense_flag_merge(const uint32_t *flag, uint32_t *status, cudaStream_t s);
 
 }  // namespace slikl

@@ -31,6 +31,19 @@ static void layouts(void) {
     FIELD(slikl_options, dk_path); FIELD(slikl_options, fused_begin);
     FIELD(slikl_options, fused_end); FIELD(slikl_options, dk_begin); FIELD(slikl_options, dk_end);
     FIELD(slikl_options, loss); FIELD(slikl_options, seq_used_q); FIELD(slikl_options, seq_used_k);
+    printf("size slikl_dense_problem %zu\n", sizeof(slikl_dense_problem));
+    FIELD(slikl_dense_problem, dtype); FIELD(slikl_dense_problem, layout_q);
+    FIELD(slikl_dense_problem, layout_k); FIELD(slikl_dense_problem, deterministic);
+    FIELD(slikl_dense_problem, B); FIELD(slikl_dense_problem, S1); FIELD(slikl_dense_problem, S2);
+    FIELD(slikl_dense_problem, T1); FIELD(slikl_dense_problem, T2); FIELD(slikl_dense_problem, N1);
+    FIELD(slikl_dense_problem, D); FIELD(slikl_dense_problem, row_len);
+    FIELD(slikl_dense_problem, mask_mode); FIELD(slikl_dense_problem, reserved);
+    printf("size slikl_dense_tensors %zu\n", sizeof(slikl_dense_tensors));
+    FIELD(slikl_dense_tensors, q); FIELD(slikl_dense_tensors, k); FIELD(slikl_dense_tensors, w);
+    FIELD(slikl_dense_tensors, attn_softmax_l1norm); FIELD(slikl_dense_tensors, cu_seqlens_q);
+    FIELD(slikl_dense_tensors, cu_seqlens_k); FIELD(slikl_dense_tensors, dq);
+    FIELD(slikl_dense_tensors, dk); FIELD(slikl_dense_tensors, dw);
+    FIELD(slikl_dense_tensors, softmax_out);
 }
 
 int main(int argc, char **argv) {

@@ -299,3 +299,85 @@ def test_binding_rejects_bad_used_lengths():
         for name in ("seq_used_q", "seq_used_k"):
             with pytest.raises(ValueError, match=name):
                 sli.grad(q, k, w, p, idx, "TND", "TND", cuq, cuk, **{name: u})
+
+
+# ---------------------------------------------------------------------------
+# dense variant: host-side validation and workspace size (no CUDA call)
+# ---------------------------------------------------------------------------
+
+def dense_problem(**kw):
+    pr = sli.slikl_dense_problem()
+    pr.dtype, pr.layout_q, pr.layout_k = sli.SLIKL_BF16, sli.SLIKL_BSND, sli.SLIKL_BSND
+    pr.deterministic = 0
+    pr.B, pr.S1, pr.S2, pr.T1, pr.T2, pr.N1, pr.D = 2, 64, 96, 0, 0, 16, 128
+    pr.row_len, pr.mask_mode, pr.reserved = 0, 3, 0
+    for f, v in kw.items():
+        setattr(pr, f, v)
+    return pr
+
+
+def dense_code(pr, opt=None):
+    n = ctypes.c_size_t(0)
+    return sli.load_library().slikl_dense_grad_workspace_size(
+        ctypes.byref(pr), ctypes.byref(opt) if opt is not None else None, ctypes.byref(n)), n.value
+
+
+def test_dense_validation_codes(lib):
+    assert dense_code(dense_problem())[0] == sli.SLIKL_OK
+    assert dense_code(dense_problem(mask_mode=0))[0] == sli.SLIKL_OK
+    for bad in (dict(mask_mode=1), dict(mask_mode=2), dict(reserved=1), dict(row_len=8193),
+                dict(row_len=50), dict(layout_k=sli.SLIKL_TND, row_len=0), dict(N1=129),
+                dict(D=96)):
+        assert dense_code(dense_problem(**bad))[0] == sli.SLIKL_ERR_PARAM_INVALID, bad
+    assert sli.load_library().slikl_dense_grad_workspace_size(None, None, ctypes.byref(ctypes.c_size_t())) \
+        == sli.SLIKL_ERR_PARAM_NULLPTR
+    assert sli.load_library().slikl_dense_grad_workspace_size(ctypes.byref(dense_problem()), None, None) \
+        == sli.SLIKL_ERR_INNER_NULLPTR
+
+
+def test_dense_workspace_holds_the_index_rows(lib):
+    """The dense workspace is the sparse problem's (topk = the row length) plus the index rows
+    [T1 x Ld] int32 and a flag word."""
+    pr = dense_problem(row_len=128)
+    code, dense_bytes = dense_code(pr)
+    assert code == sli.SLIKL_OK
+    sp = sli.slikl_problem()
+    for f in ("dtype", "layout_q", "layout_k", "deterministic", "B", "S1", "S2", "T1", "T2",
+              "N1", "D"):
+        setattr(sp, f, getattr(pr, f))
+    sp.topk = 128
+    sparse = sli.slikl_grad_workspace_size(sp)
+    T1 = pr.B * pr.S1
+    assert dense_bytes >= sparse + T1 * 128 * 4 + 4
+    assert dense_bytes <= (sparse + 255) // 256 * 256 + (T1 * 128 * 4 + 255) // 256 * 256 + 256
+
+
+def test_dense_launch_rejects_bad_arguments_without_a_gpu(lib):
+    """Argument errors are found on the host, before any CUDA call."""
+    pr = dense_problem()
+    tn = sli.slikl_dense_tensors()
+    rc = sli.load_library().slikl_dense_grad(ctypes.byref(pr), None, None, 0, None, None)
+    assert rc == sli.SLIKL_ERR_PARAM_NULLPTR
+    rc = sli.load_library().slikl_dense_grad(ctypes.byref(pr), ctypes.byref(tn), None, 0, None, None)
+    assert rc == sli.SLIKL_ERR_PARAM_NULLPTR
+    rc = sli.load_library().slikl_dense_grad(ctypes.byref(pr), ctypes.byref(tn), 256, 16, None, None)
+    assert rc == sli.SLIKL_ERR_WORKSPACE_TOO_SMALL
+    need = dense_code(pr)[1]
+    rc = sli.load_library().slikl_dense_grad(ctypes.byref(pr), ctypes.byref(tn), 256, need, None, None)
+    assert rc == sli.SLIKL_ERR_PARAM_NULLPTR          # tensors not given
+
+
+def test_dense_dk_path_query(lib):
+    """The dense call's dK path is the sparse operator's choice for top-k = the row length:
+    key-major for N1 <= 64 in atomic mode, scatter otherwise; an impossible request is refused."""
+    assert sli.slikl_dense_grad_dk_path(dense_problem()) == sli.SLIKL_DK_KEYMAJOR
+    assert sli.slikl_dense_grad_dk_path(dense_problem(N1=128)) == sli.SLIKL_DK_SCATTER
+    assert sli.slikl_dense_grad_dk_path(dense_problem(deterministic=1)) == sli.SLIKL_DK_SCATTER
+    assert sli.slikl_dense_grad_dk_path(dense_problem(), sli.make_options("scatter")) \
+        == sli.SLIKL_DK_SCATTER
+    with pytest.raises(sli.SliklError):
+        sli.slikl_dense_grad_dk_path(dense_problem(N1=128), sli.make_options("keymajor"))
+    with pytest.raises(sli.SliklError):
+        sli.slikl_dense_grad_dk_path(dense_problem(mask_mode=1))
+    assert sli.load_library().slikl_dense_grad_dk_path(ctypes.byref(dense_problem()), None, None) \
+        == sli.SLIKL_ERR_INNER_NULLPTR

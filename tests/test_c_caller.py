@@ -47,7 +47,9 @@ def c_output(tmp_path_factory):
 
 def test_struct_layouts_match_the_binding(c_output):
     mirrors = {"slikl_problem": sli.slikl_problem, "slikl_tensors": sli.slikl_tensors,
-               "slikl_options": sli.slikl_options}
+               "slikl_options": sli.slikl_options,
+               "slikl_dense_problem": sli.slikl_dense_problem,
+               "slikl_dense_tensors": sli.slikl_dense_tensors}
     seen = set()
     for line in c_output:
         parts = line.split()
