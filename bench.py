@@ -361,12 +361,17 @@ def step_roofline_ms(stats, peaks, peak_tf):
 def per_config_lines(sli, dev, stream, flush, peaks, steps, warmup):
     """The other full-size workloads, timed the same way as the headline (device time, L2
     flushed before every step): configs 2, 3 and 4 on the auto dK path, the deterministic
-    reduction on configs 4 and 1, and the dense variant's causal workload in both modes."""
+    reduction on configs 4 and 1, the 128-head causal workload, and the dense variant's causal
+    workload in both modes."""
     import torch
     out = []
-    for cid, det in ((2, False), (3, False), (4, False), (4, True), (1, True), ("dense", False),
-                     ("dense", True)):
-        if cid == "dense":
+    for cid, det in ((2, False), (3, False), (4, False), (4, True), (1, True), ("n1_128", False),
+                     ("dense", False), ("dense", True)):
+        if cid == "n1_128":
+            wl = si.wide_heads()
+            stats = workload_stats(wl)
+            r = Runner(sli, wl, dev, stream, det, "auto")
+        elif cid == "dense":
             wl = si.dense_full()
             stats = dense_stats(wl)
             r = DenseRunner(sli, wl, dev, stream, det, "auto")

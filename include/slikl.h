@@ -150,9 +150,10 @@ SLIKL_API slikl_status slikl_grad(const slikl_problem *problem, const slikl_tens
  *   SLIKL_DK_KEYMAJOR  the fused kernel stores, per named (query row, key), dI and the heads
  *                      with S > 0; a second tensor-core kernel then forms dK one 256-key block
  *                      at a time from every query row that names a key of the block.
- *                      Needs N1 <= 64, deterministic = 0 and a key-range bound
+ *                      Needs deterministic = 0 and a key-range bound
  *                      (BSND: S2; TND: problem->S2 > 0) of at most 16384 keys; its workspace
- *                      holds T1 x roundup(S2, 256) records of 8 (N1 <= 32) or 16 bytes.
+ *                      holds T1 x roundup(S2, 256) records of 8 (N1 <= 32), 16 (N1 <= 64)
+ *                      or 32 bytes.
  *   SLIKL_DK_AUTO      the key-major path when it is possible, the key range is at most 16x
  *                      topk and its records take at most 8 GiB; else the scatter path.
  * The workspace size depends on the path: size and launch with the same options.

@@ -383,6 +383,16 @@ def dense_small(seed: int, layout: str = "BSND", B: int = 2, S1: int = 40, S2: i
                          p=pt.contiguous(), cu_seqlens_q=cuq, cu_seqlens_k=cuk)
 
 
+WIDE_HEADS_NAME = "causal-bsnd B1 S4096 N1=128 D128 K2048 bf16"
+
+
+def wide_heads(seed: int = SEED_BASE + 110) -> Workload:
+    """The 128-head workload: the causal S=4096, topk=2048 recipe with N1 = 128 query heads
+    (w of variance 1/128)."""
+    return causal_bsnd(WIDE_HEADS_NAME, 1, 4096, 128, 128, 2048, torch.bfloat16, 0.1,
+                       1.0 / 128, seed)
+
+
 DENSE_FULL_NAME = "dense-causal-bsnd B1 S4096 N1=64 D128 mask3 bf16"
 
 

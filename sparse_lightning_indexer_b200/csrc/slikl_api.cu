@@ -57,11 +57,11 @@ slikl_status validate(const slikl_problem *pr, Derived *out) {
 // caller's bound in problem->S2 (0 = none given).
 int64_t key_range_bound(const slikl_problem *pr) { return pr->S2 > 0 ? pr->S2 : 0; }
 
-// Whether the key-major dK path can run this problem: the tensor-core kernels (N1 <= 64), a
-// known key-range bound of at most 16384 keys, atomic mode.
+// Whether the key-major dK path can run this problem: a known key-range bound of at most
+// 16384 keys, atomic mode.
 bool km_possible(const slikl_problem *pr) {
     const int64_t s2 = key_range_bound(pr);
-    return pr->N1 <= 64 && pr->deterministic == 0 && s2 > 0 && s2 <= 16384;
+    return pr->deterministic == 0 && s2 > 0 && s2 <= 16384;
 }
 
 // Picks the dK path. The key-major path does work in proportion to the (query row, 256-key
@@ -76,7 +76,7 @@ slikl_status choose_dk_path(const slikl_problem *pr, Derived *dv, int32_t path) 
     bool use = false;
     if (possible) {
         const int64_t s2m = (key_range_bound(pr) + 255) / 256 * 256;
-        const int rb = pr->N1 > 32 ? 16 : 8;
+        const int rb = pr->N1 > 64 ? 32 : (pr->N1 > 32 ? 16 : 8);   // record bytes
         const double rec_bytes = (double)dv->T1 * (double)s2m * rb;
         use = path == SLIKL_DK_KEYMAJOR ||
               (path == SLIKL_DK_AUTO && key_range_bound(pr) <= 16 * pr->topk &&
@@ -318,12 +318,7 @@ slikl_status slikl_grad_ex(const slikl_problem *problem, const slikl_tensors *te
     if (P.km && launch_km_metadata(P, workers, s) != cudaSuccess) return SLIKL_ERR_CUDA;
     if (fused_begin && cudaEventRecord(static_cast<cudaEvent_t>(fused_begin), s) != cudaSuccess)
         return SLIKL_ERR_CUDA;
-    if (dv.T1 > 0) {
-        bool handled = false;
-        if (launch_fused_sm100(P, workers, s, &handled) != cudaSuccess) return SLIKL_ERR_CUDA;
-        if (!handled && launch_fused_simt(P, workers, s) != cudaSuccess) return SLIKL_ERR_CUDA;
-        if (P.km && !handled) return SLIKL_ERR_CUDA;   // key-major records need the sm100 kernel
-    }
+    if (dv.T1 > 0 && launch_fused_sm100(P, workers, s) != cudaSuccess) return SLIKL_ERR_CUDA;
     if (fused_end && cudaEventRecord(static_cast<cudaEvent_t>(fused_end), s) != cudaSuccess)
         return SLIKL_ERR_CUDA;
     if (options && options->loss && launch_kl_loss(P, options->loss, s) != cudaSuccess)

@@ -49,7 +49,7 @@ struct Params {
     int S2m;              // record row length in keys: longest key range rounded up to 256
     int64_t kbound;       // the longest key range the caller promised
     int nkpw;             // 32-bit words per token in tok_pairs
-    int rec_bytes;        // 8 (N1 <= 32) or 16 (N1 <= 64)
+    int rec_bytes;        // 8 (N1 <= 32), 16 (N1 <= 64) or 32 (N1 <= 128)
     uint32_t *tok_pairs;  // [T1][nkpw] bit kp: the token names a key of [256 kp, 256 kp + 256)
     void *rec;            // [T1][S2m] records {dI, ReLU(S) > 0 mask of the heads}
     int4 *units;          // [units_max] {first token, first key row, local key | keys << 16,
@@ -144,8 +144,7 @@ __device__ __forceinline__ int32_t slot_row(int32_t v, int32_t kbase, int32_t kl
 
 // kernels (defined in the .cu files)
 cudaError_t launch_metadata(const Params &P, int workers, int mode, cudaStream_t s);
-cudaError_t launch_fused_simt(const Params &P, int workers, cudaStream_t s);
-cudaError_t launch_fused_sm100(const Params &P, int workers, cudaStream_t s, bool *handled);
+cudaError_t launch_fused_sm100(const Params &P, int workers, cudaStream_t s);
 cudaError_t launch_cast(const Params &P, cudaStream_t s);
 cudaError_t launch_deterministic_reduce(const Params &P, cudaStream_t s);
 cudaError_t launch_km_metadata(const Params &P, int workers, cudaStream_t s);

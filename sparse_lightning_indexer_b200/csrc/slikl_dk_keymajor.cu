@@ -42,8 +42,18 @@ namespace {
 using namespace sm100;
 
 constexpr int kKmThreads = 768;
-constexpr int kKmStages = 4;
+constexpr int kKmStages = 4;             // most stages of any instance (barrier arrays)
 constexpr int kKmTmemCols = 512;         // two dK^T buffers of 256 columns
+
+// Per instance: record bytes (mask words of the heads, dI), stages, and the dS tile of a
+// stage ([256 keys x N1P heads] as 64-head column blocks of 256 x 128 B)
+template <int N1P> __host__ __device__ constexpr int km_rec_bytes() {
+    return N1P > 64 ? 32 : (N1P > 32 ? 16 : 8);
+}
+template <int N1P> __host__ __device__ constexpr int km_stages() { return N1P > 64 ? 2 : kKmStages; }
+template <int N1P> __host__ __device__ constexpr uint32_t km_ds_bytes() {
+    return N1P > 64 ? 2u * 256u * 128u : 256u * 128u;
+}
 
 struct KmBarriers {
     uint64_t full[kKmStages];            // q, w, records landed (producer, TMA bytes)
@@ -60,18 +70,17 @@ struct KmPlan {
 
 __host__ __device__ constexpr uint32_t round_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
-template <int N1P, int RB>
+template <int N1P>
 __host__ __device__ constexpr KmPlan km_plan() {
-    // [stage][2 column blocks][N1P heads][128 B] | [stage][256 keys][128 B] |
+    // [stage][2 column blocks][N1P heads][128 B] | [stage][dS tile] |
     // [stage][256 records] | [stage][N1P] | barriers
+    constexpr uint32_t S = km_stages<N1P>(), RB = km_rec_bytes<N1P>(), DS = km_ds_bytes<N1P>();
     return KmPlan{0u,
-                  kKmStages * N1P * 256u,
-                  kKmStages * N1P * 256u + kKmStages * 256u * 128u,
-                  kKmStages * N1P * 256u + kKmStages * 256u * 128u + kKmStages * 256u * RB,
-                  round_up(kKmStages * N1P * 256u + kKmStages * 256u * 128u +
-                               kKmStages * 256u * RB + kKmStages * N1P * 4u, 8),
-                  round_up(kKmStages * N1P * 256u + kKmStages * 256u * 128u +
-                               kKmStages * 256u * RB + kKmStages * N1P * 4u, 8) +
+                  S * N1P * 256u,
+                  S * N1P * 256u + S * DS,
+                  S * N1P * 256u + S * DS + S * 256u * RB,
+                  round_up(S * N1P * 256u + S * DS + S * 256u * RB + S * N1P * 4u, 8),
+                  round_up(S * N1P * 256u + S * DS + S * 256u * RB + S * N1P * 4u, 8) +
                       (uint32_t)sizeof(KmBarriers) + 1024u};
 }
 
@@ -143,8 +152,10 @@ __global__ void __launch_bounds__(kKmThreads, 1)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    constexpr int RB = N1P > 32 ? 16 : 8;
-    constexpr KmPlan SP = km_plan<N1P, RB>();
+    constexpr int RB = km_rec_bytes<N1P>();
+    constexpr int kSt = km_stages<N1P>();
+    constexpr uint32_t kDs = km_ds_bytes<N1P>();
+    constexpr KmPlan SP = km_plan<N1P>();
     constexpr int kFmt = std::is_same<T, __nv_bfloat16>::value ? 1 : 0;
     constexpr uint32_t kIdesc = idesc_f16(kFmt, 128, 256, 1, 0);
     constexpr uint32_t kTx = (D / 64) * N1P * 128 + 256 * RB;   // q boxes + records
@@ -157,7 +168,7 @@ __global__ void __launch_bounds__(kKmThreads, 1)
 
     if (threadIdx.x == 0) {
         abort_flag = 0;
-        for (int s = 0; s < kKmStages; ++s) {
+        for (int s = 0; s < kSt; ++s) {
             mbar_init(&bars->full[s], 1);
             mbar_init(&bars->dsr[s], 16);
             mbar_init(&bars->empty[s], 1);
@@ -171,7 +182,7 @@ __global__ void __launch_bounds__(kKmThreads, 1)
     }
     if (D == 64) {
         // the upper column block of every q stage stays zero (rows d >= 64 of q^T)
-        for (uint32_t i = threadIdx.x; i < kKmStages * N1P * 128 / 16; i += kKmThreads) {
+        for (uint32_t i = threadIdx.x; i < kSt * N1P * 128 / 16; i += kKmThreads) {
             const uint32_t st = i / (N1P * 8), r = i % (N1P * 8);
             reinterpret_cast<uint4 *>(smem + SP.q + st * N1P * 256 + N1P * 128)[r] =
                 make_uint4(0, 0, 0, 0);
@@ -211,8 +222,8 @@ __global__ void __launch_bounds__(kKmThreads, 1)
             KmItem nx;
             const bool have_nx = iter.next(nx);
             if (have_nx) load_w(nx.t, wnxt);
-            const int s = i % kKmStages;
-            if (!wait_bar(&bars->empty[s], ((i / kKmStages) & 1) ^ 1, &abort_flag, P.status)) { ok = false; break; }
+            const int s = i % kSt;
+            if (!wait_bar(&bars->empty[s], ((i / kSt) & 1) ^ 1, &abort_flag, P.status)) { ok = false; break; }
             float *wd = reinterpret_cast<float *>(smem + SP.w + s * N1P * 4);
 #pragma unroll
             for (int k = 0; k < (N1P + 31) / 32; ++k)
@@ -236,9 +247,9 @@ __global__ void __launch_bounds__(kKmThreads, 1)
         }
         if (!ok && lane == 0) {
             // wait (bounded) for the copies already issued before the CTA leaves
-            for (uint32_t j = i > kKmStages ? i - kKmStages : 0; j < i; ++j) {
+            for (uint32_t j = i > kSt ? i - kSt : 0; j < i; ++j) {
                 const long long st = clock64();
-                while (!mbar_try_wait(&bars->full[j % kKmStages], (j / kKmStages) & 1) &&
+                while (!mbar_try_wait(&bars->full[j % kSt], (j / kSt) & 1) &&
                        clock64() - st < kWaitCycles) {}
             }
         }
@@ -246,18 +257,19 @@ __global__ void __launch_bounds__(kKmThreads, 1)
         // =============================== MMA issuer ===============================
         uint32_t i = 0, nrun = 0;
         while (iter.next(it)) {
-            const int s = i % kKmStages;
+            const int s = i % kSt;
             const int ab = nrun & 1;
-            if (!wait_bar(&bars->dsr[s], (i / kKmStages) & 1, &abort_flag, P.status)) break;
+            if (!wait_bar(&bars->dsr[s], (i / kSt) & 1, &abort_flag, P.status)) break;
             if (it.first && !wait_bar(&bars->acce[ab], ((nrun >> 1) & 1) ^ 1, &abort_flag, P.status)) break;
             tc_fence_after();
             if (lane == 0) {
                 const uint32_t qa = smem_u32(smem + SP.q + s * N1P * 256);
-                const uint32_t da = smem_u32(smem + SP.ds + s * 256 * 128);
+                const uint32_t da = smem_u32(smem + SP.ds + s * kDs);
 #pragma unroll
                 for (int ks = 0; ks < N1P / 16; ++ks) {
                     const uint64_t a = sdesc(qa + ks * 2048, N1P * 128, 1024);   // q^T, MN-major
-                    const uint64_t b = sdesc(da + ks * 32, 16, 1024);            // dS, K-major
+                    // dS, K-major: 16 heads per step, 64-head column blocks of 256 rows
+                    const uint64_t b = sdesc(da + (ks >> 2) * (256 * 128) + (ks & 3) * 32, 16, 1024);
                     umma_f16(tacc + ab * 256, a, b, kIdesc, (it.first && ks == 0) ? 0u : 1u);
                 }
                 umma_commit(&bars->empty[s]);
@@ -301,44 +313,49 @@ __global__ void __launch_bounds__(kKmThreads, 1)
         }
     } else if (warp >= 8) {
         // =============================== dS builders ===============================
-        // two threads per key of the pair: heads [32 h, 32 h + 32) of key e
+        // two threads per key of the pair: half of its heads each (32, or 64 with 128 heads)
         const int e = (threadIdx.x - 256) >> 1;   // key of the pair, 0..255
         const int half = threadIdx.x & 1;
         constexpr int kChunks = N1P / 8;          // 16-byte chunks of 8 heads per row
-        constexpr int kHalfChunks = kChunks < 4 ? kChunks : 4;
-        const bool has_work = half * 4 < kChunks;
+        constexpr int kPer = N1P > 64 ? 8 : (kChunks < 4 ? kChunks : 4);   // chunks per thread
+        const bool has_work = half * kPer < kChunks;
         uint32_t i = 0;
         while (iter.next(it)) {
-            const int s = i % kKmStages;
-            if (!wait_bar(&bars->full[s], (i / kKmStages) & 1, &abort_flag, P.status)) break;
+            const int s = i % kSt;
+            if (!wait_bar(&bars->full[s], (i / kSt) & 1, &abort_flag, P.status)) break;
             if (has_work) {
-                uint32_t m;
+                uint32_t m0, m1 = 0;              // mask bits of this thread's heads
                 float dI;
                 const uint8_t *rp = smem + SP.rec + s * 256 * RB + e * RB;
-                if (RB == 16) {
+                if (RB == 32) {
                     const uint4 r = *reinterpret_cast<const uint4 *>(rp);
-                    m = half ? r.y : r.x;
+                    m0 = half ? r.z : r.x;
+                    m1 = half ? r.w : r.y;
+                    dI = *reinterpret_cast<const float *>(rp + 16);
+                } else if (RB == 16) {
+                    const uint4 r = *reinterpret_cast<const uint4 *>(rp);
+                    m0 = half ? r.y : r.x;
                     dI = __uint_as_float(r.z);
                 } else {
                     const uint2 r = *reinterpret_cast<const uint2 *>(rp);
-                    m = r.x;
+                    m0 = r.x;
                     dI = __uint_as_float(r.y);
                 }
-                const float *ws = reinterpret_cast<const float *>(smem + SP.w + s * N1P * 4) + 32 * half;
-                uint8_t *row = smem + SP.ds + s * 256 * 128 + e * 128;
+                const float *ws = reinterpret_cast<const float *>(smem + SP.w + s * N1P * 4) + 8 * kPer * half;
+                uint8_t *row = smem + SP.ds + s * kDs + e * 128;
 #pragma unroll
-                for (int cc = 0; cc < kHalfChunks; ++cc) {   // 8 heads = one 16-byte chunk
-                    const int c = half * 4 + cc;
+                for (int cc = 0; cc < kPer; ++cc) {   // 8 heads = one 16-byte chunk
+                    const int c = half * kPer + cc;   // chunk of the row; column block c / 8
                     const float4 wa = *reinterpret_cast<const float4 *>(ws + 8 * cc);
                     const float4 wb = *reinterpret_cast<const float4 *>(ws + 8 * cc + 4);
-                    const uint32_t mb = (m >> (cc * 8)) & 0xFFu;
+                    const uint32_t mb = ((cc < 4 ? m0 : m1) >> ((cc & 3) * 8)) & 0xFFu;
                     const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
                     float d[8];
 #pragma unroll
                     for (int h = 0; h < 8; ++h) d[h] = ((mb >> h) & 1u) ? dI * wv[h] : 0.f;
                     const uint4 o = make_uint4(pack2<T>(d[0], d[1]), pack2<T>(d[2], d[3]),
                                                pack2<T>(d[4], d[5]), pack2<T>(d[6], d[7]));
-                    *reinterpret_cast<uint4 *>(row + (((c ^ e) & 7) << 4)) = o;
+                    *reinterpret_cast<uint4 *>(row + (c >> 3) * (256 * 128) + ((((c & 7) ^ e) & 7) << 4)) = o;
                 }
             }
             fence_proxy_async();
@@ -360,8 +377,7 @@ __global__ void __launch_bounds__(kKmThreads, 1)
 
 template <int N1P, int D, typename T>
 cudaError_t launch_km_t(const Params &P, int workers, cudaStream_t s) {
-    constexpr int RB = N1P > 32 ? 16 : 8;
-    constexpr KmPlan sp = km_plan<N1P, RB>();
+    constexpr KmPlan sp = km_plan<N1P>();
     static_assert(sp.total <= 227 * 1024, "key-major kernel shared memory");
     CUtensorMap qmap;
     cudaError_t e = encode_q_map<N1P, T>(P, &qmap);
@@ -386,12 +402,13 @@ cudaError_t launch_km_n(const Params &P, int workers, cudaStream_t s) {
 
 }  // namespace
 
-// Shapes: N1 <= 64, D in {64, 128}.
+// Shapes: N1 <= 128, D in {64, 128}.
 cudaError_t launch_dk_keymajor(const Params &P, int workers, cudaStream_t s) {
-    if (P.N1 > 64 || (P.D != 64 && P.D != 128)) return cudaErrorInvalidValue;
+    if (P.N1 > 128 || (P.D != 64 && P.D != 128)) return cudaErrorInvalidValue;
     if (P.N1 <= 16) return launch_km_n<16>(P, workers, s);
     if (P.N1 <= 32) return launch_km_n<32>(P, workers, s);
-    return launch_km_n<64>(P, workers, s);
+    if (P.N1 <= 64) return launch_km_n<64>(P, workers, s);
+    return launch_km_n<128>(P, workers, s);
 }
 
 }  // namespace slikl

@@ -70,6 +70,14 @@ struct SmemPlan {
 constexpr int kRingSlot = 136;            // int32 entries per slot
 constexpr int kRowsStride = 132;          // int32 entries per key-row buffer (16-byte multiple)
 
+// dS tiles [128 keys x N1P heads] are column blocks of 64 heads (128-byte rows, 16 KB per
+// block); with 128 heads there is room for one tile (and one dK^T buffer in TMEM), else two
+template <int N1P> __host__ __device__ constexpr int n_ds_tiles() { return N1P > 64 ? 1 : 2; }
+template <int N1P> __host__ __device__ constexpr int ds_bytes() { return N1P > 64 ? 32768 : 16384; }
+template <int N1P> __host__ __device__ constexpr int red_stride() { return N1P > 64 ? N1P : 64; }
+// K stages: four of 32 KB; three with 128 heads (q and dS tiles are twice as large)
+template <int N1P> __host__ __device__ constexpr int kv_stages() { return N1P > 64 ? 3 : 4; }
+
 template <int N1P>
 __host__ __device__ inline SmemPlan plan_smem(int stages) {
     SmemPlan s{};
@@ -83,10 +91,10 @@ __host__ __device__ inline SmemPlan plan_smem(int stages) {
     s.stages = stages;
     s.kv = take(stages * kStageBytes, 1024);
     s.q = take(2 * N1P * 256, 1024);                 // two buffers, 2 column blocks each
-    s.ds = take(2 * 128 * 128, 1024);                // two buffers [128 keys x 64 heads]
+    s.ds = take(n_ds_tiles<N1P>() * ds_bytes<N1P>(), 1024);   // dS tiles [128 keys x N1P heads]
     s.w = take(2 * N1P * 4, 16);                     // w of two tokens
-    s.rows = take(2 * kRowsStride * 4, 16);          // key rows of two dS tiles
-    s.red = take(2 * 4 * 64 * 4, 16);               // dW partials of two tokens
+    s.rows = take(2 * kRowsStride * 4, 16);          // key rows of the dS tiles
+    s.red = take(2 * 4 * red_stride<N1P>() * 4, 16); // dW partials of two tokens
     s.ring = take(7 * 4 * kRingSlot * 4, 16);       // up to 7 producer warps
     s.bar = take(sizeof(Barriers) + 16, 8);
     s.total = off + 1024;                            // slack for aligning the dynamic base
@@ -194,9 +202,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t kIdescDk = idesc_f16(kFmt, 128, 128, 1, 0);
     constexpr int kDChunks = D / 8;          // 16-byte chunks per key row
     constexpr int kC = N1P < 32 ? N1P : 32;  // S columns per TMEM load
-    constexpr int kRecBytes = N1P > 32 ? 16 : 8;  // record: ReLU mask word(s), dI
+    // record: ReLU mask word(s), dI (padded to 8, 16 or 32 bytes)
+    constexpr int kRecBytes = N1P > 64 ? 32 : (N1P > 32 ? 16 : 8);
     // producer warps: 0-2, and in record mode also 4-7 (the scatter group has no work there)
     constexpr int kProd = kRec ? 7 : 3;
+    // S^T buffers in TMEM, dS tiles in smem (and dK^T buffers in TMEM, scatter mode)
+    constexpr int kNs = (N1P > 64 && !kRec) ? 1 : 2;
+    constexpr int kNd = n_ds_tiles<N1P>();
+    constexpr uint32_t kDsBytes = ds_bytes<N1P>();
+    // TMEM columns: S^T buffers from 0, then dq^T, the per-slot dW partials and the dK^T
+    // buffers (up to 64 heads: 0 / 128 / 192 / 256; 128 heads: S^T x kNs, then 128 each)
+    constexpr uint32_t kColDq = N1P <= 64 ? 128 : kNs * 128;
+    constexpr uint32_t kColDw = N1P <= 64 ? 192 : kColDq + 128;
+    constexpr uint32_t kColDk = N1P <= 64 ? 256 : kColDw + 128;
+    static_assert(kColDw + N1P <= kTmemCols, "TMEM columns");
+    static_assert(kRec || kColDk + kNd * 128 <= kTmemCols, "TMEM columns (dK^T buffers)");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t0 = P.meta[kMetaHeader + 2 * blockIdx.x];
@@ -226,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     // zero the dS tiles once: heads past N1P stay 0
-    for (uint32_t i = threadIdx.x; i < 2 * 16384 / 16; i += kThreads)
+    for (uint32_t i = threadIdx.x; i < kNd * kDsBytes / 16; i += kThreads)
         reinterpret_cast<uint4 *>(smem + SP.ds)[i] = make_uint4(0, 0, 0, 0);
     // zero the q buffers once: padded heads and, for D = 64, the upper column block stay 0;
     // for D = 64 also the upper column block of every K stage (never written by the gather)
@@ -248,10 +268,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ctl.tmem_base;
-    const uint32_t tm_s = tmem;              // S^T buffers: columns [0, 2*N1P)
-    const uint32_t tm_dq = tmem + 128;       // dq^T: columns [128, 128 + N1P)
-    const uint32_t tm_dw = tmem + 192;       // per-slot dW partial sums: columns [192, 192 + N1P)
-    const uint32_t tm_dk = tmem + 256;       // dK^T buffers: columns [256, 512)
+    const uint32_t tm_s = tmem;              // S^T buffers: columns [0, kNs * N1P)
+    const uint32_t tm_dq = tmem + kColDq;    // dq^T: N1P columns
+    const uint32_t tm_dw = tmem + kColDw;    // per-slot dW partial sums: N1P columns
+    const uint32_t tm_dk = tmem + kColDk;    // dK^T buffers: kNd x 128 columns (scatter mode)
     int32_t *rows_s = reinterpret_cast<int32_t *>(smem + SP.rows);   // [2][kRowsStride]
 
     Sched sc;
@@ -379,12 +399,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ds0 = smem_u32(smem + SP.ds);
         // S^T of item gk into S buffer gk % 2 (pass-A stages are released right away)
         auto issue_s = [&](const Item &it, int &stage) -> bool {
-            const int s = gk % stages, b = gk & 1;
+            const int s = gk % stages, b = gk % kNs;
             const int qb = it.ord & 1;
             if (it.kind == 0 && it.first &&
                 !wait_bar(&bars->q_full[qb], (it.ord >> 1) & 1, &ctl.abort, P.status)) return false;
             if (!wait_bar(&bars->kv_full[s], (gk / stages) & 1, &ctl.abort, P.status)) return false;
-            if (!wait_bar(&bars->s_empty[b], ((gk >> 1) & 1) ^ 1, &ctl.abort, P.status)) return false;
+            if (!wait_bar(&bars->s_empty[b], ((gk / kNs) & 1) ^ 1, &ctl.abort, P.status)) return false;
             tc_fence_after();
             if (lane == 0) {
                 const uint32_t kaddr = kv0 + s * kStageBytes;
@@ -411,14 +431,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const Item nxt = sc.next();
             if (nxt.kind >= 0 && !issue_s(nxt, st_nxt)) { ok = false; break; }
             if (cur.kind == 1) {
-                const int b = gd & 1;
+                const int b = gd % kNd;
                 if (cur.first && !wait_bar(&bars->dq_empty, (nb & 1) ^ 1, &ctl.abort, P.status)) { ok = false; break; }
-                if (!wait_bar(&bars->ds_full[b], (gd >> 1) & 1, &ctl.abort, P.status)) { ok = false; break; }
-                if (!kRec && !wait_bar(&bars->dk_empty[b], ((gd >> 1) & 1) ^ 1, &ctl.abort, P.status)) { ok = false; break; }
+                if (!wait_bar(&bars->ds_full[b], (gd / kNd) & 1, &ctl.abort, P.status)) { ok = false; break; }
+                if (!kRec && !wait_bar(&bars->dk_empty[b], ((gd / kNd) & 1) ^ 1, &ctl.abort, P.status)) { ok = false; break; }
                 tc_fence_after();
                 if (lane == 0) {
                     const uint32_t kaddr = kv0 + st_cur * kStageBytes;
-                    const uint32_t dsaddr = ds0 + b * 16384;
+                    const uint32_t dsaddr = ds0 + b * kDsBytes;
                     const uint32_t qaddr = q0 + (cur.ord & 1) * N1P * 256;
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks) {        // 128 keys, 16 per step
@@ -433,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int ks = 0; ks < N1P / 16; ++ks) {  // N1P heads, 16 per step
                             const uint64_t a = sdesc(qaddr + ks * 2048, N1P * 128, 1024);
-                            const uint64_t bd = sdesc(dsaddr + ks * 32, 16, 1024);
+                            const uint64_t bd = sdesc(dsaddr + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
                             umma_f16(tm_dk + b * 128, a, bd, kIdescDk, ks > 0);
                         }
                         umma_commit(&bars->dk_full[b]);
@@ -470,9 +490,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const Item it = sc.next();
             if (it.kind < 0) break;
             if (it.kind != 1) continue;
-            const int b = gd & 1;
-            if (!wait_bar(&bars->rows_full[b], (gd >> 1) & 1, &ctl.abort, P.status)) { ok = false; break; }
-            if (!wait_bar(&bars->dk_full[b], (gd >> 1) & 1, &ctl.abort, P.status)) { ok = false; break; }
+            const int b = gd % kNd;
+            if (!wait_bar(&bars->rows_full[b], (gd / kNd) & 1, &ctl.abort, P.status)) { ok = false; break; }
+            if (!wait_bar(&bars->dk_full[b], (gd / kNd) & 1, &ctl.abort, P.status)) { ok = false; break; }
             tc_fence_after();
             if (quad * 32 < D) {
                 // 4 chunks of 32 keys, one compact loop body (the instruction cache of a
@@ -558,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // pass-A items load the next item's inputs right away; pass-B items after their
             // proxy fence (which would otherwise also wait for these loads)
             if (nx.kind >= 0 && it.kind == 0) prefetch(nx, it, nxt);
-            const int sb = gk & 1;
+            const int sb = gk % kNs;
             const float *ws = wsm + (it.ord & 1) * N1P;
             const int32_t kl = cur.kl;
             const int j = it.tile * 128 + lrow;
@@ -591,7 +611,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const int32_t v = cur.v;
                 const bool valid = v >= 0 && v < kl;   // (the metadata pass checked the index)
-                if (!wait_bar(&bars->s_full[sb], (gk >> 1) & 1, &ctl.abort, P.status)) { ok = false; break; }
+                if (!wait_bar(&bars->s_full[sb], (gk / kNs) & 1, &ctl.abort, P.status)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t sa = tm_s + sb * N1P + lane_addr;
                 float sv[32];
@@ -650,7 +670,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     M_b = M_n;
                     iZ_b = iZ_n;
                 }
-                const int b = gd & 1;
+                const int b = gd % kNd;
                 const int32_t v = cur.v;
                 const bool valid = v >= 0 && v < kl;
                 float dI = 0.f, y = 0.f;
@@ -660,14 +680,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     dI = valid ? y - cur.p : 0.f;
                 }
                 // dS tile / key rows of buffer b free once the scatter of its previous use ended
-                if (!wait_bar(&bars->dk_empty[b], ((gd >> 1) & 1) ^ 1, &ctl.abort, P.status)) { ok = false; break; }
-                if (!wait_bar(&bars->s_full[sb], (gk >> 1) & 1, &ctl.abort, P.status)) { ok = false; break; }
+                if (!wait_bar(&bars->dk_empty[b], ((gd / kNd) & 1) ^ 1, &ctl.abort, P.status)) { ok = false; break; }
+                if (!wait_bar(&bars->s_full[sb], (gk / kNs) & 1, &ctl.abort, P.status)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t sa = tm_s + sb * N1P + lane_addr;
                 const uint32_t dwa = tm_dw + lane_addr;
-                // this slot's row of the [keys x heads] dS tile: 128 bytes, 16-byte chunks swizzled
-                uint8_t *dsrow = ds_tiles + b * 16384 + lrow * 128;
-                uint64_t smask = 0;                 // heads with S > 0 (record mode)
+                // this slot's row of the [keys x heads] dS tile: 128 bytes per 64-head column
+                // block, 16-byte chunks swizzled
+                uint8_t *dsrow = ds_tiles + b * kDsBytes + lrow * 128;
+                uint64_t smask = 0, smask_hi = 0;   // heads with S > 0 (record mode)
                 // 16 heads at a time: dS to smem; this slot's dW partial sums stay in TMEM
 #pragma unroll 1
                 for (int c = 0; c < N1P; c += 16) {
@@ -689,12 +710,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                         pk[h >> 1] = pack2<T>(s0 > 0.f ? dI * wv[h] : 0.f, s1 > 0.f ? dI * wv[h + 1] : 0.f);
                         if (kRec) m16 |= (s0 > 0.f ? 1u : 0u) << h | (s1 > 0.f ? 2u : 0u) << h;
                     }
-                    const int c8 = c >> 3;          // 16-byte chunk of heads c .. c + 7
-                    *reinterpret_cast<uint4 *>(dsrow + (((c8 ^ lrow) & 7) << 4)) =
+                    const int c8 = (c & 63) >> 3;   // 16-byte chunk of heads c .. c + 7
+                    uint8_t *dsblk = dsrow + (c >> 6) * 16384;
+                    *reinterpret_cast<uint4 *>(dsblk + (((c8 ^ lrow) & 7) << 4)) =
                         make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    *reinterpret_cast<uint4 *>(dsrow + ((((c8 + 1) ^ lrow) & 7) << 4)) =
+                    *reinterpret_cast<uint4 *>(dsblk + ((((c8 + 1) ^ lrow) & 7) << 4)) =
                         make_uint4(pk[4], pk[5], pk[6], pk[7]);
-                    if (kRec) smask |= (uint64_t)m16 << c;
+                    if (kRec) {
+                        if (c < 64) smask |= (uint64_t)m16 << c;
+                        else smask_hi |= (uint64_t)m16 << (c - 64);
+                    }
                     tmem_st16(dwa + c, acc);
                 }
                 tmem_wait_st();
@@ -713,7 +738,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // naming the key; dI is added, so repeated slots of a key sum their dI
                     if (valid && v < P.S2m) {
                         char *rp = static_cast<char *>(P.rec) + ((int64_t)it.t * P.S2m + v) * kRecBytes;
-                        if (kRecBytes == 16) {
+                        if (kRecBytes == 32) {
+                            *reinterpret_cast<uint4 *>(rp) =
+                                make_uint4((uint32_t)smask, (uint32_t)(smask >> 32),
+                                           (uint32_t)smask_hi, (uint32_t)(smask_hi >> 32));
+                            red_add_f32(reinterpret_cast<float *>(rp + 16), dI);
+                        } else if (kRecBytes == 16) {
                             *reinterpret_cast<uint2 *>(rp) = make_uint2((uint32_t)smask, (uint32_t)(smask >> 32));
                             red_add_f32(reinterpret_cast<float *>(rp + 8), dI);
                         } else {
@@ -733,29 +763,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if ((mask >> tl) & 1) continue;
                         for (int jz = tl * 128 + et; jz < (tl + 1) * 128 && jz < K; jz += 128) P.y[row_off + jz] = 0.f;
                     }
-                    constexpr int kV = N1P < 32 ? 32 : N1P;
-                    float vv[kV];
-#pragma unroll
-                    for (int h = 0; h < kV; ++h) vv[h] = 0.f;
-#pragma unroll
-                    for (int c = 0; c < N1P; c += 16) tmem_ld16(tm_dw + lane_addr + c, vv + c);
-                    tmem_wait_ld();
-                    int len = kV;
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) {
-                        const int half = len >> 1;
-                        const bool upper = (lane & o) != 0;
-#pragma unroll
-                        for (int h = 0; h < kV / 2; ++h) {
-                            if (h < half) {
-                                const float mine = upper ? vv[h + half] : vv[h];
-                                const float other = upper ? vv[h] : vv[h + half];
-                                vv[h] = mine + __shfl_xor_sync(0xffffffffu, other, o);
-                            }
-                        }
-                        len = half;
-                    }
-                    int base = 0, span = kV;
+                    // per 64-head block (32 columns at least): the 32 lanes' partials summed
+                    // by a butterfly that leaves each lane kVW / 32 heads, then the 4 warps
+                    // summed in a fixed order through shared memory
+                    constexpr int kVW = N1P < 32 ? 32 : (N1P > 64 ? 64 : N1P);
+                    constexpr int kRS = red_stride<N1P>();
+                    int base = 0, span = kVW;
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) {
                         span >>= 1;
@@ -765,13 +778,38 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // before the others have read this one (nothing in between waits on them);
                     // it writes this buffer again two tokens on, after the next token's group
                     // sync, which every warp reaches only after its reads below
-                    float *rd = red + (it.ord & 1) * 256;
+                    float *rd = red + (it.ord & 1) * 4 * kRS;
 #pragma unroll
-                    for (int h = 0; h < kV / 32; ++h) rd[ew * 64 + base + h] = vv[h];
+                    for (int hb = 0; hb < N1P; hb += kVW) {
+                        float vv[kVW];
+#pragma unroll
+                        for (int h = 0; h < kVW; ++h) vv[h] = 0.f;
+#pragma unroll
+                        for (int c = 0; c < kVW && hb + c < N1P; c += 16)
+                            tmem_ld16(tm_dw + lane_addr + hb + c, vv + c);
+                        tmem_wait_ld();
+                        int len = kVW;
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) {
+                            const int half = len >> 1;
+                            const bool upper = (lane & o) != 0;
+#pragma unroll
+                            for (int h = 0; h < kVW / 2; ++h) {
+                                if (h < half) {
+                                    const float mine = upper ? vv[h + half] : vv[h];
+                                    const float other = upper ? vv[h] : vv[h + half];
+                                    vv[h] = mine + __shfl_xor_sync(0xffffffffu, other, o);
+                                }
+                            }
+                            len = half;
+                        }
+#pragma unroll
+                        for (int h = 0; h < kVW / 32; ++h) rd[ew * kRS + hb + base + h] = vv[h];
+                    }
                     if (!group_sync(&bars->sm_sync, ph, &ctl.abort, P.status)) { ok = false; break; }
                     for (int h = et; h < P.N1; h += 128) {
                         float a = 0.f;
-                        for (int i = 0; i < 4; ++i) a += rd[i * 64 + h];
+                        for (int i = 0; i < 4; ++i) a += rd[i * kRS + h];
                         P.dw[(int64_t)it.t * P.N1 + h] = a;
                     }
                     // dq^T readback (lane = d): columns = heads
@@ -815,7 +853,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int N1P, int D, typename T>
 cudaError_t launch_t(const Params &P, int workers, cudaStream_t s) {
-    const int stages = 4;
+    const int stages = kv_stages<N1P>();
     const SmemPlan sp = plan_smem<N1P>(stages);
     if (sp.total > 226 * 1024) return cudaErrorInvalidConfiguration;
     auto k = P.km ? fused_sm100<N1P, D, T, true> : fused_sm100<N1P, D, T, false>;
@@ -841,15 +879,14 @@ cudaError_t launch_n(const Params &P, int workers, cudaStream_t s) {
 
 }  // namespace
 
-// Shapes this kernel covers: N1 <= 64 (padded to 16/32/64 heads), D in {64, 128},
-// topk <= 8192 (at most 64 tiles). Everything else goes to the CUDA-core kernel.
-cudaError_t launch_fused_sm100(const Params &P, int workers, cudaStream_t s, bool *handled) {
-    *handled = false;
-    if (P.N1 > 64 || (P.D != 64 && P.D != 128) || P.K > 64 * 128) return cudaSuccess;
-    *handled = true;
+// Shapes: N1 <= 128 (padded to 16/32/64/128 heads), D in {64, 128}, topk <= 8192 (at most
+// 64 tiles): every problem the entry points accept.
+cudaError_t launch_fused_sm100(const Params &P, int workers, cudaStream_t s) {
+    if (P.N1 > 128 || (P.D != 64 && P.D != 128) || P.K > 64 * 128) return cudaErrorInvalidValue;
     if (P.N1 <= 16) return launch_n<16>(P, workers, s);
     if (P.N1 <= 32) return launch_n<32>(P, workers, s);
-    return launch_n<64>(P, workers, s);
+    if (P.N1 <= 64) return launch_n<64>(P, workers, s);
+    return launch_n<128>(P, workers, s);
 }
 
 }  // namespace slikl

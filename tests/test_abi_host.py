@@ -165,8 +165,10 @@ def test_dk_path_choice(lib):
     # key range (4096) within 16x topk: key-major on auto
     assert dk_path(lib, base_problem()) == (sli.SLIKL_OK, sli.SLIKL_DK_KEYMAJOR)
     assert dk_path(lib, base_problem(), "scatter") == (sli.SLIKL_OK, sli.SLIKL_DK_SCATTER)
-    # deterministic mode, long key ranges, N1 > 64: scatter on auto, key-major refused
-    for kw in (dict(deterministic=1), dict(S2=131072), dict(N1=128), dict(S2=20000, topk=4096)):
+    # up to 128 heads on key-major (32-byte records)
+    assert dk_path(lib, base_problem(N1=128)) == (sli.SLIKL_OK, sli.SLIKL_DK_KEYMAJOR)
+    # deterministic mode, long key ranges: scatter on auto, key-major refused
+    for kw in (dict(deterministic=1), dict(S2=131072), dict(S2=20000, topk=4096)):
         assert dk_path(lib, base_problem(**kw)) == (sli.SLIKL_OK, sli.SLIKL_DK_SCATTER), kw
         assert dk_path(lib, base_problem(**kw), "keymajor")[0] == sli.SLIKL_ERR_PARAM_INVALID, kw
     # key range above 16x topk: scatter on auto, key-major still possible on request
@@ -191,6 +193,9 @@ def test_keymajor_workspace_holds_the_records(lib):
     pr32 = base_problem(N1=32, S2=1000)        # 8-byte records, rows rounded up to 1024 keys
     rc, n32 = ws_ex(lib, pr32, "keymajor")
     assert rc == sli.SLIKL_OK and n32 - ws_ex(lib, pr32, "scatter")[1] >= 4096 * 1024 * 8
+    pr128 = base_problem(N1=128)               # 32-byte records
+    rc, n128 = ws_ex(lib, pr128, "keymajor")
+    assert rc == sli.SLIKL_OK and n128 - ws_ex(lib, pr128, "scatter")[1] >= 4096 * 4096 * 32
     # the plain size call is the auto path
     assert ws_rc(lib, pr)[1] == n_k
 
@@ -214,7 +219,7 @@ def test_grad_ex_host_validation(lib):
     # unknown path, key-major on a problem it cannot run
     assert grad_ex_rc(lib, pr, tn, 1 << 20, need_auto, sli.make_options(5)) == \
         sli.SLIKL_ERR_PARAM_INVALID
-    assert grad_ex_rc(lib, base_problem(N1=128), tn, 1 << 20, 1 << 40,
+    assert grad_ex_rc(lib, base_problem(deterministic=1), tn, 1 << 20, 1 << 40,
                       sli.make_options("keymajor")) == sli.SLIKL_ERR_PARAM_INVALID
     # loss output and used-length inputs must be 4-byte aligned
     assert grad_ex_rc(lib, pr, tn, 1 << 20, need_auto, sli.make_options(loss=0x1002)) == \
@@ -369,14 +374,14 @@ def test_dense_launch_rejects_bad_arguments_without_a_gpu(lib):
 
 def test_dense_dk_path_query(lib):
     """The dense call's dK path is the sparse operator's choice for top-k = the row length:
-    key-major for N1 <= 64 in atomic mode, scatter otherwise; an impossible request is refused."""
+    key-major in atomic mode, scatter in deterministic mode; an impossible request is refused."""
     assert sli.slikl_dense_grad_dk_path(dense_problem()) == sli.SLIKL_DK_KEYMAJOR
-    assert sli.slikl_dense_grad_dk_path(dense_problem(N1=128)) == sli.SLIKL_DK_SCATTER
+    assert sli.slikl_dense_grad_dk_path(dense_problem(N1=128)) == sli.SLIKL_DK_KEYMAJOR
     assert sli.slikl_dense_grad_dk_path(dense_problem(deterministic=1)) == sli.SLIKL_DK_SCATTER
     assert sli.slikl_dense_grad_dk_path(dense_problem(), sli.make_options("scatter")) \
         == sli.SLIKL_DK_SCATTER
     with pytest.raises(sli.SliklError):
-        sli.slikl_dense_grad_dk_path(dense_problem(N1=128), sli.make_options("keymajor"))
+        sli.slikl_dense_grad_dk_path(dense_problem(deterministic=1), sli.make_options("keymajor"))
     with pytest.raises(sli.SliklError):
         sli.slikl_dense_grad_dk_path(dense_problem(mask_mode=1))
     assert sli.load_library().slikl_dense_grad_dk_path(ctypes.byref(dense_problem()), None, None) \

@@ -90,9 +90,11 @@ def schedule(masks):
     return items
 
 
-def build(items, rec, stages=4, owner_producers=False):
+def build(items, rec, stages=4, owner_producers=False, ns=2, nd=2):
     """Roles of one CTA. rec: record mode (key-major dK; no scatter group, the MMA releases the
-    dS tile after the dq product). owner_producers: the known-bad variant."""
+    dS tile after the dq product). owner_producers: the known-bad variant. ns / nd: S^T
+    buffers in TMEM and dS tiles (with their dK^T buffers); the 128-head instances use one S
+    buffer (scatter mode) or two (record mode) and one dS tile, with three K stages."""
     nprod = 7 if rec else 3
     bars = {}
 
@@ -117,8 +119,8 @@ def build(items, rec, stages=4, owner_producers=False):
 
     # safety bookkeeping: how many times each buffer was filled, and released by each of the
     # warps that read it (a buffer is free again only when every reader is done with it)
-    st = dict(stage_free=[0] * stages, s_fill=[0, 0], s_free=[[0, 0] for _ in range(4)],
-              ds_fill=[[0, 0] for _ in range(4)], ds_free=[[0, 0] for _ in range(4)])
+    st = dict(stage_free=[0] * stages, s_fill=[0] * ns, s_free=[[0] * ns for _ in range(4)],
+              ds_fill=[[0] * nd for _ in range(4)], ds_free=[[0] * nd for _ in range(4)])
 
     def freed(key, b):
         return min(w[b] for w in st[key])
@@ -158,12 +160,12 @@ def build(items, rec, stages=4, owner_producers=False):
 
         def issue_s(it):
             nonlocal gk
-            s, b = gk % stages, gk & 1
+            s, b = gk % stages, gk % ns
             if it["kind"] == 0 and it["first"]:
                 yield from wait(f"q_full{it['ord'] & 1}", (it["ord"] >> 1) & 1)
             yield from wait(f"kv_full{s}", (gk // stages) & 1)
-            yield from wait(f"s_empty{b}", ((gk >> 1) & 1) ^ 1)
-            if freed("s_free", b) < gk >> 1:
+            yield from wait(f"s_empty{b}", ((gk // ns) & 1) ^ 1)
+            if freed("s_free", b) < gk // ns:
                 raise Violation(f"S buffer {b} overwritten (item {gk}) before it was read")
             st["s_fill"][b] += 1
             bars[f"s_full{b}"].arrive()
@@ -183,13 +185,13 @@ def build(items, rec, stages=4, owner_producers=False):
             if i + 1 < len(items):
                 stage_nxt = yield from issue_s(items[i + 1])
             if cur["kind"] == 1:
-                b = gd & 1
+                b = gd % nd
                 if cur["first"]:
                     yield from wait("dq_empty", (nb & 1) ^ 1)
-                yield from wait(f"ds_full{b}", (gd >> 1) & 1)
+                yield from wait(f"ds_full{b}", (gd // nd) & 1)
                 if not rec:
-                    yield from wait(f"dk_empty{b}", ((gd >> 1) & 1) ^ 1)
-                if min(w[b] for w in st["ds_fill"]) != (gd >> 1) + 1:
+                    yield from wait(f"dk_empty{b}", ((gd // nd) & 1) ^ 1)
+                if min(w[b] for w in st["ds_fill"]) != gd // nd + 1:
                     raise Violation(f"dq product read dS buffer {b} not holding item {gd}")
                 st["stage_free"][stage_cur] += 1
                 bars[f"kv_empty{stage_cur}"].arrive()
@@ -213,9 +215,9 @@ def build(items, rec, stages=4, owner_producers=False):
         for it in items:
             if it["kind"] != 1:
                 continue
-            b = gd & 1
-            yield from wait(f"rows_full{b}", (gd >> 1) & 1)
-            yield from wait(f"dk_full{b}", (gd >> 1) & 1)
+            b = gd % nd
+            yield from wait(f"rows_full{b}", (gd // nd) & 1)
+            yield from wait(f"dk_full{b}", (gd // nd) & 1)
             st["ds_free"][wq][b] += 1
             bars[f"dk_empty{b}"].arrive()
             gd += 1
@@ -231,12 +233,12 @@ def build(items, rec, stages=4, owner_producers=False):
     def softmax(wq):
         gk = gd = nb = 0
         for it in items:
-            sb = gk & 1
+            sb = gk % ns
             if it["kind"] == 0:
                 if it["first"]:
                     yield from group_sync(wq)
-                yield from wait(f"s_full{sb}", (gk >> 1) & 1)
-                if st["s_fill"][sb] != (gk >> 1) + 1:
+                yield from wait(f"s_full{sb}", (gk // ns) & 1)
+                if st["s_fill"][sb] != gk // ns + 1:
                     raise Violation(f"pass A read S buffer {sb} not holding item {gk}")
                 st["s_free"][wq][sb] += 1
                 bars[f"s_empty{sb}"].arrive()
@@ -244,12 +246,12 @@ def build(items, rec, stages=4, owner_producers=False):
                     yield from group_sync(wq)
                     yield from group_sync(wq)
             else:
-                b = gd & 1
-                yield from wait(f"dk_empty{b}", ((gd >> 1) & 1) ^ 1)
-                if freed("ds_free", b) < gd >> 1:
+                b = gd % nd
+                yield from wait(f"dk_empty{b}", ((gd // nd) & 1) ^ 1)
+                if freed("ds_free", b) < gd // nd:
                     raise Violation(f"dS buffer {b} overwritten (item {gd}) before it was read")
-                yield from wait(f"s_full{sb}", (gk >> 1) & 1)
-                if st["s_fill"][sb] != (gk >> 1) + 1:
+                yield from wait(f"s_full{sb}", (gk // ns) & 1)
+                if st["s_fill"][sb] != gk // ns + 1:
                     raise Violation(f"pass B read S buffer {sb} not holding item {gk}")
                 st["s_free"][wq][sb] += 1
                 st["ds_fill"][wq][b] += 1
@@ -330,6 +332,18 @@ def test_protocol_finishes_and_is_safe(rec):
     for i, masks in enumerate(cases):
         for seed in range(3):
             stuck = run(masks, rec, seed=1000 * i + seed)
+            assert stuck is None, f"deadlock with masks {masks}: {stuck}"
+
+
+@pytest.mark.parametrize("rec", [False, True], ids=["scatter", "record"])
+def test_protocol_128_heads_finishes_and_is_safe(rec):
+    """The 128-head instances: three K stages, one dS tile (and dK^T buffer), and one S^T
+    buffer in scatter mode (two in record mode, which has no dK^T buffers)."""
+    rnd = random.Random(20261203 + rec)
+    cases = EDGE_MASKS + [random_masks(rnd) for _ in range(250)]
+    for i, masks in enumerate(cases):
+        for seed in range(3):
+            stuck = run(masks, rec, seed=1000 * i + seed, stages=3, ns=2 if rec else 1, nd=1)
             assert stuck is None, f"deadlock with masks {masks}: {stuck}"
 
 
@@ -490,13 +504,15 @@ def km_run(runs, seed, **kw):
     return None
 
 
-def test_keymajor_protocol_finishes_and_is_safe():
+@pytest.mark.parametrize("stages", [4, 2], ids=["4stages", "2stages_128heads"])
+def test_keymajor_protocol_finishes_and_is_safe(stages):
     rnd = random.Random(20261203)
     cases = [[1], [1, 1, 1], [32], [1, 32, 1], [5, 5, 5, 5, 5]]
     cases += [[rnd.randint(1, 12) for _ in range(rnd.randint(1, 8))] for _ in range(150)]
     for i, runs in enumerate(cases):
         for seed in range(3):
-            assert km_run(runs, seed=1000 * i + seed) is None, f"deadlock with runs {runs}"
+            assert km_run(runs, seed=1000 * i + seed, stages=stages) is None, \
+                f"deadlock with runs {runs}"
 
 
 def test_keymajor_planted_mistake_is_caught():

@@ -90,8 +90,6 @@ MODES = [(False, "auto"), (False, "scatter"), (False, "keymajor"), (True, "auto"
 @pytest.mark.parametrize("mode", MODES, ids=["auto", "scatter", "keymajor", "det"])
 def test_dense_parity(case, mode):
     det, path = mode
-    if path == "keymajor" and case["N1"] > 64:
-        pytest.skip("the key-major dK path needs N1 <= 64")
     wl = si.dense_small(**case)
     ref = oracle.dense_grad(wl)
     got = run_dense(wl, deterministic=det, dk_path=path)

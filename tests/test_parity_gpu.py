@@ -108,6 +108,13 @@ SMALL = [
          pattern="uniform"),
     dict(seed=12, layout="TND", B=4, S1=70, S2=900, N1=48, D=64, K=700, dtype=torch.float16,
          pattern="causal", invalid_frac=0.1),
+    # 64 < N1 <= 128: the 128-head tensor-core instances (heads past N1 padded with zeros)
+    dict(seed=13, layout="BSND", B=1, S1=24, S2=2100, N1=128, D=128, K=2048, qk_scale=0.1,
+         w_var=1 / 128),
+    dict(seed=14, layout="TND", B=2, S1=30, S2=500, N1=96, D=64, K=300, dtype=torch.float16,
+         pattern="causal"),
+    dict(seed=15, layout="BSND", B=2, S1=25, S2=200, N1=65, D=128, K=130, pattern="dup",
+         invalid_frac=0.2),
 ]
 
 
@@ -115,16 +122,10 @@ MODES = [(False, "scatter"), (False, "keymajor"), (True, "scatter")]
 MODE_IDS = ["scatter", "keymajor", "det"]
 
 
-def keymajor_possible(case):
-    return case["N1"] <= 64
-
-
 @pytest.mark.parametrize("case", SMALL, ids=lambda c: f"s{c['seed']}")
 @pytest.mark.parametrize("mode", MODES, ids=MODE_IDS)
 def test_small_parity(case, mode):
     det, path = mode
-    if path == "keymajor" and not keymajor_possible(case):
-        pytest.skip("key-major dK path needs N1 <= 64")
     wl = si.small(**case)
     ref = oracle.grad(wl)
     got = run_gpu(wl, deterministic=det, dk_path=path)
@@ -192,6 +193,18 @@ def test_full_size_parity(cid):
         check_against(wl, got, ref)
         del got
     _CFG_CACHE.pop(cid, None)
+
+
+def test_full_size_parity_128_heads():
+    """The 128-head workload (causal S=4096, topk=2048, N1=128) in full on each dK mode."""
+    wl = si.wide_heads()
+    ref = oracle.grad(wl)
+    for det, path in [(False, "auto"), (False, "scatter"), (True, "auto")]:
+        got = run_gpu(wl, deterministic=det, dk_path=path)
+        assert got["flags"] == 0, (det, path)
+        check_exact(wl, got)
+        check_against(wl, got, ref)
+        del got
 
 
 @pytest.mark.parametrize("cid", [1, 3])
@@ -338,8 +351,6 @@ def test_metadata_weighted_hand_worked():
 def test_kl_loss_output(case, path):
     """The optional per-row KL loss output against the oracle's L_t (rel-L2 <= 1e-5, rows
     without a valid slot exactly 0), on the dK paths that can run the case."""
-    if path == "keymajor" and not keymajor_possible(case):
-        pytest.skip("key-major dK path needs N1 <= 64")
     wl = si.small(**case)
     ref = oracle.grad(wl)
     res = sli.grad_workload(wl, dk_path=path, loss=True)
@@ -425,8 +436,6 @@ SEQ_USED = [
 def test_seq_used_parity(sc, mode):
     det, path = mode
     case = sc["case"]
-    if path == "keymajor" and not keymajor_possible(case):
-        pytest.skip("the key-major path needs N1 <= 64")
     wl = si.small(**case)
     lq, lk = lengths(wl)
     qu, ku = sc["used"](lq, lk)
