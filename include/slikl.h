@@ -127,8 +127,8 @@ SLIKL_API slikl_status slikl_grad_workspace_size(const slikl_problem *problem, s
 
 /*
  * Phase 2. Re-validates, then queues on `stream`: zeroing of the status word and of the
- * fp32 dk accumulator, the work-split kernel, the fused per-token kernel, and (atomic mode)
- * the dk cast or (deterministic mode) the key-major sort and fixed-order reduction.
+ * fp32 dk accumulator, the work-split kernel, the fused per-token kernel, the dK stage of the
+ * chosen path (below) and the dk cast.
  * Writes dq, dk, dw and softmax_out in full.
  * `workspace` (device, >= the phase-1 size, 256-byte aligned) is scratch owned by the
  * caller for the duration of the call; its first 256 bytes hold the device status word
@@ -146,14 +146,16 @@ SLIKL_API slikl_status slikl_grad(const slikl_problem *problem, const slikl_tens
  * dK paths (slikl_options.dk_path). Both give the same dK up to the order of fp32 additions.
  *   SLIKL_DK_SCATTER   every named slot adds its dK row into an fp32 accumulator with
  *                      atomic adds (the page's default), or, deterministic = 1, stores it for
- *                      the key-major sort and fixed-order reduction;
+ *                      a sort by key and a fixed-order reduction;
  *   SLIKL_DK_KEYMAJOR  the fused kernel stores, per named (query row, key), dI and the heads
  *                      with S > 0; a second tensor-core kernel then forms dK one 256-key block
  *                      at a time from every query row that names a key of the block.
- *                      Needs deterministic = 0 and a key-range bound
- *                      (BSND: S2; TND: problem->S2 > 0) of at most 16384 keys; its workspace
- *                      holds T1 x roundup(S2, 256) records of 8 (N1 <= 32), 16 (N1 <= 64)
- *                      or 32 bytes.
+ *                      Needs a key-range bound (BSND: S2; TND: problem->S2 > 0) of at most
+ *                      16384 keys; its workspace holds T1 x roundup(S2, 256) records of 8
+ *                      (N1 <= 32), 16 (N1 <= 64; also N1 <= 32 with deterministic = 1) or 32
+ *                      bytes. With deterministic = 1 repeated slots of a key sum their dI as
+ *                      64-bit fixed-point integers and every key row is summed in a fixed
+ *                      order, so the result is bitwise repeatable.
  *   SLIKL_DK_AUTO      the key-major path when it is possible, the key range is at most 16x
  *                      topk and its records take at most 8 GiB; else the scatter path.
  * The workspace size depends on the path: size and launch with the same options.

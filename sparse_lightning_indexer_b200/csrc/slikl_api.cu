@@ -58,10 +58,10 @@ slikl_status validate(const slikl_problem *pr, Derived *out) {
 int64_t key_range_bound(const slikl_problem *pr) { return pr->S2 > 0 ? pr->S2 : 0; }
 
 // Whether the key-major dK path can run this problem: a known key-range bound of at most
-// 16384 keys, atomic mode.
+// 16384 keys.
 bool km_possible(const slikl_problem *pr) {
     const int64_t s2 = key_range_bound(pr);
-    return pr->deterministic == 0 && s2 > 0 && s2 <= 16384;
+    return s2 > 0 && s2 <= 16384;
 }
 
 // Picks the dK path. The key-major path does work in proportion to the (query row, 256-key
@@ -76,7 +76,9 @@ slikl_status choose_dk_path(const slikl_problem *pr, Derived *dv, int32_t path) 
     bool use = false;
     if (possible) {
         const int64_t s2m = (key_range_bound(pr) + 255) / 256 * 256;
-        const int rb = pr->N1 > 64 ? 32 : (pr->N1 > 32 ? 16 : 8);   // record bytes
+        // record bytes: the mask words of the heads, then dI (fp32, or a 64-bit fixed-point
+        // number in deterministic mode)
+        const int rb = pr->N1 > 64 ? 32 : (pr->N1 > 32 || pr->deterministic ? 16 : 8);
         const double rec_bytes = (double)dv->T1 * (double)s2m * rb;
         use = path == SLIKL_DK_KEYMAJOR ||
               (path == SLIKL_DK_AUTO && key_range_bound(pr) <= 16 * pr->topk &&
@@ -155,6 +157,7 @@ Params make_params(const slikl_problem *pr, const Derived &dv, const slikl_tenso
         P.unit_off = reinterpret_cast<int64_t *>(base + L.unit_off);
         P.unit_prefix = reinterpret_cast<int64_t *>(base + L.unit_prefix);
         P.km_range = reinterpret_cast<int32_t *>(base + L.km_range);
+        P.km_scratch = reinterpret_cast<float *>(base + L.km_scratch);
     }
     return P;
 }
@@ -311,11 +314,15 @@ slikl_status slikl_grad_ex(const slikl_problem *problem, const slikl_tensors *te
 
     const int workers = sms < kMaxWorkers ? sms : kMaxWorkers;
     if (cudaMemsetAsync(P.status, 0, 256, s) != cudaSuccess) return SLIKL_ERR_CUDA;
-    if (!P.deterministic && dv.T2 > 0 &&
+    // deterministic mode on the scatter path: sorted per-slot rows; otherwise the fp32 rows
+    const bool sorted = P.deterministic && !P.km;
+    // the key-major kernel's CTAs (its deterministic scratch holds kKmDetWorkers of them)
+    const int km_workers = P.deterministic && workers > kKmDetWorkers ? kKmDetWorkers : workers;
+    if (!sorted && dv.T2 > 0 &&
         cudaMemsetAsync(P.dk_acc, 0, sizeof(float) * (size_t)dv.T2 * problem->D, s) != cudaSuccess)
         return SLIKL_ERR_CUDA;
     if (launch_metadata(P, workers, 1, s) != cudaSuccess) return SLIKL_ERR_CUDA;
-    if (P.km && launch_km_metadata(P, workers, s) != cudaSuccess) return SLIKL_ERR_CUDA;
+    if (P.km && launch_km_metadata(P, km_workers, s) != cudaSuccess) return SLIKL_ERR_CUDA;
     if (fused_begin && cudaEventRecord(static_cast<cudaEvent_t>(fused_begin), s) != cudaSuccess)
         return SLIKL_ERR_CUDA;
     if (dv.T1 > 0 && launch_fused_sm100(P, workers, s) != cudaSuccess) return SLIKL_ERR_CUDA;
@@ -327,8 +334,12 @@ slikl_status slikl_grad_ex(const slikl_problem *problem, const slikl_tensors *te
     void *dk_end = options ? options->dk_end : nullptr;
     if (dk_begin && cudaEventRecord(static_cast<cudaEvent_t>(dk_begin), s) != cudaSuccess)
         return SLIKL_ERR_CUDA;
-    if (P.km && dv.T1 > 0 && launch_dk_keymajor(P, workers, s) != cudaSuccess) return SLIKL_ERR_CUDA;
-    cudaError_t e = P.deterministic ? launch_deterministic_reduce(P, s) : launch_cast(P, s);
+    if (P.km && dv.T1 > 0) {
+        if (launch_dk_keymajor(P, km_workers, s) != cudaSuccess) return SLIKL_ERR_CUDA;
+        if (P.deterministic && launch_km_det_combine(P, km_workers, s) != cudaSuccess)
+            return SLIKL_ERR_CUDA;
+    }
+    cudaError_t e = sorted ? launch_deterministic_reduce(P, s) : launch_cast(P, s);
     if (e != cudaSuccess) return SLIKL_ERR_CUDA;
     if (dk_end && cudaEventRecord(static_cast<cudaEvent_t>(dk_end), s) != cudaSuccess)
         return SLIKL_ERR_CUDA;

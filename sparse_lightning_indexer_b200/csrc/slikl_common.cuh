@@ -12,6 +12,8 @@
 namespace slikl {
 
 constexpr int kMaxWorkers = 4096;        // metadata capacity (workers = CTAs of the fused kernel)
+constexpr int kKmDetWorkers = 256;       // most CTAs of the key-major kernel in deterministic mode
+                                         // (its per-CTA scratch is sized for this many)
 constexpr int kSlotTile = 128;           // top-k slots per tile of the fused kernel
 constexpr int kMetaHeader = 8;
 
@@ -49,7 +51,7 @@ struct Params {
     int S2m;              // record row length in keys: longest key range rounded up to 256
     int64_t kbound;       // the longest key range the caller promised
     int nkpw;             // 32-bit words per token in tok_pairs
-    int rec_bytes;        // 8 (N1 <= 32), 16 (N1 <= 64) or 32 (N1 <= 128)
+    int rec_bytes;        // 8 (N1 <= 32; 16 in deterministic mode), 16 (N1 <= 64), 32 (N1 <= 128)
     uint32_t *tok_pairs;  // [T1][nkpw] bit kp: the token names a key of [256 kp, 256 kp + 256)
     void *rec;            // [T1][S2m] records {dI, ReLU(S) > 0 mask of the heads}
     int4 *units;          // [units_max] {first token, first key row, local key | keys << 16,
@@ -59,6 +61,11 @@ struct Params {
     int64_t *unit_prefix; // [units_max + 1] exclusive prefix of the unit costs
     int32_t *km_range;    // [kMaxWorkers + 1] first unit of each worker of the key-major kernel
     int64_t units_max;
+    // deterministic key-major path: the runs of 256-key block pairs that a CTA's unit range
+    // cuts (its first run, continued from the previous CTA, and its last, continued by the
+    // next) are stored here instead of added, [kKmDetWorkers][2][256][D], and summed in CTA
+    // order afterwards
+    float *km_scratch;
 };
 
 // Shape of the key-major dK path of one call (km = 0: scatter path).
@@ -72,7 +79,7 @@ struct KmShape {
 struct WsLayout {
     size_t status, meta, tok_kbase, tok_klen, tok_cost, tok_tiles, cost_prefix;
     size_t dk_acc, partials, keys0, vals0, keys1, vals1, hist, row_ptr;
-    size_t tok_pairs, rec, units, units_c, unit_off, unit_prefix, km_range;
+    size_t tok_pairs, rec, units, units_c, unit_off, unit_prefix, km_range, km_scratch;
     size_t total;
 };
 
@@ -92,17 +99,18 @@ inline WsLayout make_layout(int64_t T1, int64_t T2, int64_t K, int64_t D, int de
     L.tok_cost = take(sizeof(int32_t) * (size_t)T1);
     L.tok_tiles = take(sizeof(uint64_t) * (size_t)T1);
     L.cost_prefix = take(sizeof(int64_t) * (size_t)(T1 + 1));
-    L.dk_acc = take(det ? 0 : sizeof(float) * (size_t)T2 * (size_t)D);
+    const bool k = km.km != 0;
+    const bool sorted = det && !k;           // deterministic mode on the scatter path
+    L.dk_acc = take(sorted ? 0 : sizeof(float) * (size_t)T2 * (size_t)D);
     size_t n = (size_t)T1 * (size_t)K;
     size_t sort_blocks = (n + kSortTile - 1) / kSortTile;
-    L.partials = take(det ? sizeof(float) * n * (size_t)D : 0);
-    L.keys0 = take(det ? sizeof(int32_t) * n : 0);
-    L.vals0 = take(det ? sizeof(int32_t) * n : 0);
-    L.keys1 = take(det ? sizeof(int32_t) * n : 0);
-    L.vals1 = take(det ? sizeof(int32_t) * n : 0);
-    L.hist = take(det ? sizeof(int32_t) * 256 * sort_blocks : 0);
-    L.row_ptr = take(det ? sizeof(int32_t) * (size_t)(T2 + 2) : 0);
-    const bool k = km.km != 0;
+    L.partials = take(sorted ? sizeof(float) * n * (size_t)D : 0);
+    L.keys0 = take(sorted ? sizeof(int32_t) * n : 0);
+    L.vals0 = take(sorted ? sizeof(int32_t) * n : 0);
+    L.keys1 = take(sorted ? sizeof(int32_t) * n : 0);
+    L.vals1 = take(sorted ? sizeof(int32_t) * n : 0);
+    L.hist = take(sorted ? sizeof(int32_t) * 256 * sort_blocks : 0);
+    L.row_ptr = take(sorted ? sizeof(int32_t) * (size_t)(T2 + 2) : 0);
     L.tok_pairs = take(k ? sizeof(uint32_t) * (size_t)T1 * km.nkpw : 0);
     L.rec = take(k ? (size_t)T1 * (size_t)km.S2m * km.rec_bytes : 0);
     L.units = take(k ? 16 * (size_t)km.units_max : 0);
@@ -110,6 +118,7 @@ inline WsLayout make_layout(int64_t T1, int64_t T2, int64_t K, int64_t D, int de
     L.unit_off = take(k ? sizeof(int64_t) * (size_t)(B + 1) : 0);
     L.unit_prefix = take(k ? sizeof(int64_t) * (size_t)(km.units_max + 1) : 0);
     L.km_range = take(k ? sizeof(int32_t) * (kMaxWorkers + 1) : 0);
+    L.km_scratch = take(k && det ? sizeof(float) * (size_t)kKmDetWorkers * 2 * 256 * (size_t)D : 0);
     L.total = off;
     return L;
 }
@@ -135,6 +144,22 @@ __device__ __forceinline__ void red_add_f32(float *addr, float v) {
     asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
 }
 
+// Key-major records: the mask words of the heads, then dI at this byte offset. In
+// deterministic mode dI is a signed 64-bit fixed-point number (units of 2^-48) summed with
+// integer adds, so repeated slots of a key give the same sum in any order; |dI| <= 1 per slot
+// and at most 8192 slots per row keep the sum below 2^61.
+__host__ __device__ constexpr int rec_di_offset(int rec_bytes) { return rec_bytes == 8 ? 4 : rec_bytes / 2; }
+constexpr float kDiFixedOne = 281474976710656.0f;    // 2^48
+
+__device__ __forceinline__ void red_add_di_fixed(void *addr, float dI) {
+    const long long v = __float2ll_rn(dI * kDiFixedOne);
+    asm volatile("red.global.add.u64 [%0], %1;" ::"l"(addr), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ float di_from_fixed(long long v) {
+    return __ll2float_rn(v) * (1.0f / kDiFixedOne);
+}
+
 // Key row of slot value v for a token whose keys in use are [kbase, kbase + klen), or -1.
 // (Values that break the index contract were flagged by the metadata pass; here they are
 // simply invalid.)
@@ -149,6 +174,7 @@ cudaError_t launch_cast(const Params &P, cudaStream_t s);
 cudaError_t launch_deterministic_reduce(const Params &P, cudaStream_t s);
 cudaError_t launch_km_metadata(const Params &P, int workers, cudaStream_t s);
 cudaError_t launch_dk_keymajor(const Params &P, int workers, cudaStream_t s);
+cudaError_t launch_km_det_combine(const Params &P, int workers, cudaStream_t s);
 cudaError_t launch_dense_indices(int32_t *idx, int64_t T1, int64_t B, int64_t S1, int64_t S2,
                                  int Ld, int layout_q, int layout_k, int mask,
                                  const int32_t *cu_q, const int32_t *cu_k, const int32_t *used_q,

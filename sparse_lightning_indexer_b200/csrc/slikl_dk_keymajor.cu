@@ -19,7 +19,10 @@
 // key-major metadata kernels). Each CTA takes a contiguous, cost-balanced range of units;
 // consecutive units on the same pair form a run that accumulates in one of two TMEM
 // buffers and is flushed once, with red.global.add.f32 of 32 consecutive d per warp
-// instruction, into the fp32 dK rows.
+// instruction, into the fp32 dK rows. In deterministic mode (section "确定性计算": bitwise
+// repeatable results) the records carry dI as 64-bit fixed point, a run that is the only
+// contribution to its key rows is stored, and the pieces of a run cut by the CTA ranges go
+// to a per-CTA scratch that km_det_combine sums in CTA order.
 //
 // Warp roles (768 threads):
 //   warp 0      producer: per query row, TMA of q_t (128-byte swizzle, zero heads past N1)
@@ -45,11 +48,10 @@ constexpr int kKmThreads = 768;
 constexpr int kKmStages = 4;             // most stages of any instance (barrier arrays)
 constexpr int kKmTmemCols = 512;         // two dK^T buffers of 256 columns
 
-// Per instance: record bytes (mask words of the heads, dI), stages, and the dS tile of a
-// stage ([256 keys x N1P heads] as 64-head column blocks of 256 x 128 B)
-template <int N1P> __host__ __device__ constexpr int km_rec_bytes() {
-    return N1P > 64 ? 32 : (N1P > 32 ? 16 : 8);
-}
+// Per instance: the largest record (mask words of the heads, dI; 8-byte records of N1 <= 32
+// grow to 16 in deterministic mode), stages, and the dS tile of a stage ([256 keys x N1P
+// heads] as 64-head column blocks of 256 x 128 B)
+template <int N1P> __host__ __device__ constexpr int km_rec_bytes() { return N1P > 64 ? 32 : 16; }
 template <int N1P> __host__ __device__ constexpr int km_stages() { return N1P > 64 ? 2 : kKmStages; }
 template <int N1P> __host__ __device__ constexpr uint32_t km_ds_bytes() {
     return N1P > 64 ? 2u * 256u * 128u : 256u * 128u;
@@ -158,7 +160,8 @@ __global__ void __launch_bounds__(kKmThreads, 1)
     constexpr KmPlan SP = km_plan<N1P>();
     constexpr int kFmt = std::is_same<T, __nv_bfloat16>::value ? 1 : 0;
     constexpr uint32_t kIdesc = idesc_f16(kFmt, 128, 256, 1, 0);
-    constexpr uint32_t kTx = (D / 64) * N1P * 128 + 256 * RB;   // q boxes + records
+    const int rb = P.rec_bytes;                                  // record bytes of this call
+    const uint32_t kTx = (D / 64) * N1P * 128 + 256 * rb;       // q boxes + records
     KmBarriers *bars = reinterpret_cast<KmBarriers *>(smem + SP.bar);
     __shared__ volatile int abort_flag;
     __shared__ uint32_t tmem_base;
@@ -235,8 +238,8 @@ __global__ void __launch_bounds__(kKmThreads, 1)
                 tma_load_3d(qd, &qmap, 0, 0, it.t, &bars->full[s]);
                 if (D == 128) tma_load_3d(qd + N1P * 128, &qmap, 64, 0, it.t, &bars->full[s]);
                 bulk_g2s(smem_u32(smem + SP.rec + s * 256 * RB),
-                         static_cast<const char *>(P.rec) + ((int64_t)it.t * P.S2m + it.kloc) * RB,
-                         256 * RB, &bars->full[s]);
+                         static_cast<const char *>(P.rec) + ((int64_t)it.t * P.S2m + it.kloc) * rb,
+                         256 * rb, &bars->full[s]);
             }
             __syncwarp();
             ++i;
@@ -287,6 +290,16 @@ __global__ void __launch_bounds__(kKmThreads, 1)
         // =============================== flush ===============================
         const int quad = warp & 3;
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+        // deterministic mode: a run is the only contribution to its key rows, stored as it is,
+        // unless this CTA's unit range cuts it (the first run, continued from the previous
+        // range: scratch slot 0; the last, continued by the next range: slot 1); the pieces of
+        // a cut run are summed in CTA order by km_det_combine
+        const bool det = P.deterministic != 0;
+        const int n_units = P.km_range[gridDim.x];
+        const bool cut_head = det && u0 < u1 && u0 > 0 && P.units_c[u0].y == P.units_c[u0 - 1].y;
+        const bool cut_tail = det && u0 < u1 && u1 < n_units && P.units_c[u1].y == P.units_c[u1 - 1].y;
+        const int head_key = u0 < u1 ? P.units_c[u0].y : -1;
+        const int tail_key = u0 < u1 ? P.units_c[u1 - 1].y : -1;
         uint32_t nrun = 0;
         while (iter.next(it)) {
             if (!it.last) continue;
@@ -294,16 +307,27 @@ __global__ void __launch_bounds__(kKmThreads, 1)
             if (!wait_bar(&bars->accf[ab], (nrun >> 1) & 1, &abort_flag, P.status)) break;
             tc_fence_after();
             if (quad * 32 < D) {
-                float *dst = P.dk_acc + (int64_t)it.key0 * D + quad * 32 + lane;
+                float *dst = P.dk_acc + (int64_t)it.key0 * D;
+                if (cut_head && it.key0 == head_key)
+                    dst = P.km_scratch + (int64_t)(2 * blockIdx.x) * 256 * D;
+                else if (cut_tail && it.key0 == tail_key)
+                    dst = P.km_scratch + (int64_t)(2 * blockIdx.x + 1) * 256 * D;
+                dst += quad * 32 + lane;
 #pragma unroll 1
                 for (int c = 0; c < 256; c += 32) {
                     if (c >= it.nkeys) break;
                     float v[32];
                     tmem_ld32(tacc + ab * 256 + lane_addr + c, v);
                     tmem_wait_ld();
+                    if (det) {
 #pragma unroll
-                    for (int k = 0; k < 32; ++k)
-                        if (c + k < it.nkeys) red_add_f32(dst + (int64_t)(c + k) * D, v[k]);
+                        for (int k = 0; k < 32; ++k)
+                            if (c + k < it.nkeys) dst[(int64_t)(c + k) * D] = v[k];
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 32; ++k)
+                            if (c + k < it.nkeys) red_add_f32(dst + (int64_t)(c + k) * D, v[k]);
+                    }
                 }
             }
             tc_fence_before();
@@ -326,21 +350,20 @@ __global__ void __launch_bounds__(kKmThreads, 1)
             if (has_work) {
                 uint32_t m0, m1 = 0;              // mask bits of this thread's heads
                 float dI;
-                const uint8_t *rp = smem + SP.rec + s * 256 * RB + e * RB;
-                if (RB == 32) {
+                const uint8_t *rp = smem + SP.rec + s * 256 * RB + e * rb;
+                if (N1P > 64) {
                     const uint4 r = *reinterpret_cast<const uint4 *>(rp);
                     m0 = half ? r.z : r.x;
                     m1 = half ? r.w : r.y;
-                    dI = *reinterpret_cast<const float *>(rp + 16);
-                } else if (RB == 16) {
-                    const uint4 r = *reinterpret_cast<const uint4 *>(rp);
-                    m0 = half ? r.y : r.x;
-                    dI = __uint_as_float(r.z);
-                } else {
+                } else if (N1P > 32) {
                     const uint2 r = *reinterpret_cast<const uint2 *>(rp);
-                    m0 = r.x;
-                    dI = __uint_as_float(r.y);
+                    m0 = half ? r.y : r.x;
+                } else {
+                    m0 = *reinterpret_cast<const uint32_t *>(rp);
                 }
+                const uint8_t *dp = rp + rec_di_offset(rb);
+                dI = P.deterministic ? di_from_fixed(*reinterpret_cast<const long long *>(dp))
+                                     : *reinterpret_cast<const float *>(dp);
                 const float *ws = reinterpret_cast<const float *>(smem + SP.w + s * N1P * 4) + 8 * kPer * half;
                 uint8_t *row = smem + SP.ds + s * kDs + e * 128;
 #pragma unroll
@@ -375,6 +398,42 @@ __global__ void __launch_bounds__(kKmThreads, 1)
     }
 }
 
+// Deterministic mode: the 256-key block pairs whose run of units the CTA ranges cut. Block c
+// starts a chain when its last run goes on into the next range and began inside its own; the
+// pieces (c's last run, then the first run of each following non-empty range while the run
+// goes on) are summed in that order into the fp32 key rows, which no other piece touches.
+// Grid: (workers, 16); blockIdx.y takes 16 of the pair's 256 keys.
+__global__ void km_det_combine(Params P, int workers) {
+    __shared__ int chain[kKmDetWorkers];
+    __shared__ int nchain;
+    const int c = blockIdx.x;
+    const int u0 = P.km_range[c], u1 = P.km_range[c + 1], n = P.km_range[workers];
+    if (u0 >= u1 || u1 >= n) return;
+    const int key0 = P.units_c[u1 - 1].y;
+    if (P.units_c[u1].y != key0) return;                       // the last run ends here
+    if (u0 > 0 && P.units_c[u0].y == key0 && P.units_c[u0 - 1].y == key0) return;  // began before
+    if (threadIdx.x == 0) {
+        int m = 0;
+        for (int c2 = c + 1; c2 < workers; ++c2) {
+            const int a = P.km_range[c2], b = P.km_range[c2 + 1];
+            if (a >= b) continue;                               // empty range
+            chain[m++] = c2;                                    // its first run goes on with ours
+            if (!(P.units_c[b - 1].y == key0 && b < n && P.units_c[b].y == key0)) break;
+        }
+        nchain = m;
+    }
+    __syncthreads();
+    const int nkeys = (int)((uint32_t)P.units_c[u1 - 1].z >> 16);
+    const int kend = 16 * ((int)blockIdx.y + 1) < nkeys ? 16 * ((int)blockIdx.y + 1) : nkeys;
+    const int64_t piece = (int64_t)256 * P.D;
+    const float *first = P.km_scratch + (2 * (int64_t)c + 1) * piece;
+    for (int e = 16 * (int)blockIdx.y * P.D + threadIdx.x; e < kend * P.D; e += blockDim.x) {
+        float acc = first[e];
+        for (int m = 0; m < nchain; ++m) acc += P.km_scratch[2 * (int64_t)chain[m] * piece + e];
+        P.dk_acc[(int64_t)key0 * P.D + e] = acc;
+    }
+}
+
 template <int N1P, int D, typename T>
 cudaError_t launch_km_t(const Params &P, int workers, cudaStream_t s) {
     constexpr KmPlan sp = km_plan<N1P>();
@@ -401,6 +460,12 @@ cudaError_t launch_km_n(const Params &P, int workers, cudaStream_t s) {
 }
 
 }  // namespace
+
+cudaError_t launch_km_det_combine(const Params &P, int workers, cudaStream_t s) {
+    if (workers > kKmDetWorkers) return cudaErrorInvalidValue;
+    km_det_combine<<<dim3(workers, 16), 256, 0, s>>>(P, workers);
+    return cudaGetLastError();
+}
 
 // Shapes: N1 <= 128, D in {64, 128}.
 cudaError_t launch_dk_keymajor(const Params &P, int workers, cudaStream_t s) {

@@ -11,9 +11,9 @@
 //           - scatter mode: dK^T[D x 128 keys] = q^T . dS (tcgen05), scattered into the fp32
 //             key rows with red.global.add.f32, 32 consecutive d per warp instruction (one
 //             128-byte line), or stored per slot (deterministic mode);
-//           - record mode: a record per named (token, key) - the heads with S > 0 and dI -
-//             for the key-major dK kernel, after zero-filling the token's named 256-key block
-//             pairs during pass A.
+//           - record mode: a record per named (token, key) - the heads with S > 0 and dI
+//             (fp32, or 64-bit fixed point in deterministic mode) - for the key-major dK
+//             kernel, after zero-filling the token's named 256-key block pairs during pass A.
 //   after the last pass-B tile: dW reduced in a fixed order, dq^T read back from TMEM.
 //
 // Schedule. All roles walk one deterministic item sequence in which pass A of the CTA's next
@@ -184,9 +184,12 @@ struct Sched {
 // ------------------------------------------------------------------------------------------
 // The kernel
 // ------------------------------------------------------------------------------------------
-template <int N1P, int D, typename T, bool kRec>
+// kMode: 0 = scatter mode; 1 = record mode; 2 = record mode, deterministic (dI in 64-bit
+// fixed point, 8-byte records widened to 16)
+template <int N1P, int D, typename T, int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_sm100(Params P, int stages, const __grid_constant__ CUtensorMap qmap) {
+    constexpr bool kRec = kMode != 0;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -202,8 +205,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t kIdescDk = idesc_f16(kFmt, 128, 128, 1, 0);
     constexpr int kDChunks = D / 8;          // 16-byte chunks per key row
     constexpr int kC = N1P < 32 ? N1P : 32;  // S columns per TMEM load
-    // record: ReLU mask word(s), dI (padded to 8, 16 or 32 bytes)
-    constexpr int kRecBytes = N1P > 64 ? 32 : (N1P > 32 ? 16 : 8);
+    // record: the ReLU mask word(s) (4, 8 or 16 bytes), then dI (fp32, or 64-bit fixed point)
+    constexpr int kRecBytes = N1P > 64 ? 32 : (N1P > 32 || kMode == 2 ? 16 : 8);
     // producer warps: 0-2, and in record mode also 4-7 (the scatter group has no work there)
     constexpr int kProd = kRec ? 7 : 3;
     // S^T buffers in TMEM, dS tiles in smem (and dK^T buffers in TMEM, scatter mode)
@@ -594,14 +597,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         // then adds the named keys (the group syncs that end pass A order
                         // these stores before those)
                         const uint32_t *pw = P.tok_pairs + (int64_t)it.t * P.nkpw;
+                        constexpr int rb = kRecBytes;
                         for (int wd = 0; wd < P.nkpw; ++wd) {
                             uint32_t bits = pw[wd];
                             while (bits) {
                                 const int kp = wd * 32 + __ffs(bits) - 1;
                                 bits &= bits - 1;
                                 uint4 *dst = reinterpret_cast<uint4 *>(
-                                    static_cast<char *>(P.rec) + ((int64_t)it.t * P.S2m + 256 * kp) * kRecBytes);
-                                for (int i = et; i < 256 * kRecBytes / 16; i += 128) dst[i] = make_uint4(0, 0, 0, 0);
+                                    static_cast<char *>(P.rec) + ((int64_t)it.t * P.S2m + 256 * kp) * rb);
+                                for (int i = et; i < 256 * rb / 16; i += 128) dst[i] = make_uint4(0, 0, 0, 0);
                             }
                         }
                     }
@@ -737,19 +741,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // record of this (token, key): the mask words are the same for every slot
                     // naming the key; dI is added, so repeated slots of a key sum their dI
                     if (valid && v < P.S2m) {
-                        char *rp = static_cast<char *>(P.rec) + ((int64_t)it.t * P.S2m + v) * kRecBytes;
-                        if (kRecBytes == 32) {
+                        constexpr int rb = kRecBytes;
+                        char *rp = static_cast<char *>(P.rec) + ((int64_t)it.t * P.S2m + v) * rb;
+                        if (N1P > 64) {
                             *reinterpret_cast<uint4 *>(rp) =
                                 make_uint4((uint32_t)smask, (uint32_t)(smask >> 32),
                                            (uint32_t)smask_hi, (uint32_t)(smask_hi >> 32));
-                            red_add_f32(reinterpret_cast<float *>(rp + 16), dI);
-                        } else if (kRecBytes == 16) {
+                        } else if (N1P > 32) {
                             *reinterpret_cast<uint2 *>(rp) = make_uint2((uint32_t)smask, (uint32_t)(smask >> 32));
-                            red_add_f32(reinterpret_cast<float *>(rp + 8), dI);
                         } else {
                             *reinterpret_cast<uint32_t *>(rp) = (uint32_t)smask;
-                            red_add_f32(reinterpret_cast<float *>(rp + 4), dI);
                         }
+                        if constexpr (kMode == 2) red_add_di_fixed(rp + rec_di_offset(rb), dI);
+                        else red_add_f32(reinterpret_cast<float *>(rp + rec_di_offset(rb)), dI);
                     }
                 }
                 if (j < K) P.y[row_off + j] = y;
@@ -856,7 +860,8 @@ cudaError_t launch_t(const Params &P, int workers, cudaStream_t s) {
     const int stages = kv_stages<N1P>();
     const SmemPlan sp = plan_smem<N1P>(stages);
     if (sp.total > 226 * 1024) return cudaErrorInvalidConfiguration;
-    auto k = P.km ? fused_sm100<N1P, D, T, true> : fused_sm100<N1P, D, T, false>;
+    auto k = !P.km ? fused_sm100<N1P, D, T, 0>
+                   : (P.deterministic ? fused_sm100<N1P, D, T, 2> : fused_sm100<N1P, D, T, 1>);
     CUtensorMap qmap;
     cudaError_t e = encode_q_map<N1P, T>(P, &qmap);
     if (e != cudaSuccess) return e;

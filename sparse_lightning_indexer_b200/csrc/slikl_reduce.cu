@@ -1,9 +1,9 @@
 // dK finishing kernels.
 //
-// Atomic mode (the page's default, "确定性计算": non-deterministic): the fused kernel has
-// scatter-added fp32 dK rows into dk_acc; cast_dk converts them to the input dtype.
+// Atomic mode (the page's default, "确定性计算": non-deterministic), and deterministic mode on
+// the key-major path: fp32 dK rows are in dk_acc; cast_dk converts them to the input dtype.
 //
-// Deterministic mode: the fused kernel stored one fp32 dK row per slot (t, j) in
+// Deterministic mode on the scatter path: the fused kernel stored one fp32 dK row per slot (t, j) in
 // `partials`. The slots are then inverted into key-major order by a stable LSD radix sort
 // on (key row, slot id) — hand-written, 8-bit digits — giving a CSR over key rows, and every
 // key row sums its slots in ascending slot-id order, so the result is bitwise reproducible.

@@ -55,9 +55,14 @@ def test_workspace_size_valid(lib):
     assert rc == sli.SLIKL_OK
     # fp32 dk accumulator alone is T2*D*4 bytes
     assert n >= 4096 * 128 * 4
-    rc, n_det = ws_rc(lib, base_problem(deterministic=1))
+    # deterministic mode on the scatter path: one fp32 dK row per slot
+    rc, n_det = ws_ex(lib, base_problem(deterministic=1), "scatter")
     assert rc == sli.SLIKL_OK
-    assert n_det >= 4096 * 2048 * 128 * 4       # one fp32 dK row per slot
+    assert n_det >= 4096 * 2048 * 128 * 4
+    # ... on the key-major path (auto here): records, the fp32 rows and the per-CTA scratch
+    rc, n_km = ws_rc(lib, base_problem(deterministic=1))
+    assert rc == sli.SLIKL_OK
+    assert 4096 * 4096 * 16 + 4096 * 128 * 4 + 256 * 2 * 256 * 128 * 4 <= n_km < n_det
 
 
 @pytest.mark.parametrize("field,value", [
@@ -165,10 +170,11 @@ def test_dk_path_choice(lib):
     # key range (4096) within 16x topk: key-major on auto
     assert dk_path(lib, base_problem()) == (sli.SLIKL_OK, sli.SLIKL_DK_KEYMAJOR)
     assert dk_path(lib, base_problem(), "scatter") == (sli.SLIKL_OK, sli.SLIKL_DK_SCATTER)
-    # up to 128 heads on key-major (32-byte records)
+    # up to 128 heads on key-major (32-byte records), deterministic mode too
     assert dk_path(lib, base_problem(N1=128)) == (sli.SLIKL_OK, sli.SLIKL_DK_KEYMAJOR)
-    # deterministic mode, long key ranges: scatter on auto, key-major refused
-    for kw in (dict(deterministic=1), dict(S2=131072), dict(S2=20000, topk=4096)):
+    assert dk_path(lib, base_problem(deterministic=1)) == (sli.SLIKL_OK, sli.SLIKL_DK_KEYMAJOR)
+    # long key ranges: scatter on auto, key-major refused
+    for kw in (dict(S2=131072), dict(S2=20000, topk=4096), dict(S2=131072, deterministic=1)):
         assert dk_path(lib, base_problem(**kw)) == (sli.SLIKL_OK, sli.SLIKL_DK_SCATTER), kw
         assert dk_path(lib, base_problem(**kw), "keymajor")[0] == sli.SLIKL_ERR_PARAM_INVALID, kw
     # key range above 16x topk: scatter on auto, key-major still possible on request
@@ -193,6 +199,11 @@ def test_keymajor_workspace_holds_the_records(lib):
     pr32 = base_problem(N1=32, S2=1000)        # 8-byte records, rows rounded up to 1024 keys
     rc, n32 = ws_ex(lib, pr32, "keymajor")
     assert rc == sli.SLIKL_OK and n32 - ws_ex(lib, pr32, "scatter")[1] >= 4096 * 1024 * 8
+    # deterministic mode: 16-byte records (64-bit fixed-point dI) and no sort buffers
+    prd = base_problem(N1=32, S2=1000, deterministic=1)
+    rc_d, n_d = ws_ex(lib, prd, "keymajor")
+    rc_ds, n_ds = ws_ex(lib, prd, "scatter")
+    assert rc_d == rc_ds == sli.SLIKL_OK and n_d >= 4096 * 1024 * 16 and n_d < n_ds
     pr128 = base_problem(N1=128)               # 32-byte records
     rc, n128 = ws_ex(lib, pr128, "keymajor")
     assert rc == sli.SLIKL_OK and n128 - ws_ex(lib, pr128, "scatter")[1] >= 4096 * 4096 * 32
@@ -219,7 +230,7 @@ def test_grad_ex_host_validation(lib):
     # unknown path, key-major on a problem it cannot run
     assert grad_ex_rc(lib, pr, tn, 1 << 20, need_auto, sli.make_options(5)) == \
         sli.SLIKL_ERR_PARAM_INVALID
-    assert grad_ex_rc(lib, base_problem(deterministic=1), tn, 1 << 20, 1 << 40,
+    assert grad_ex_rc(lib, base_problem(S2=131072), tn, 1 << 20, 1 << 40,
                       sli.make_options("keymajor")) == sli.SLIKL_ERR_PARAM_INVALID
     # loss output and used-length inputs must be 4-byte aligned
     assert grad_ex_rc(lib, pr, tn, 1 << 20, need_auto, sli.make_options(loss=0x1002)) == \
@@ -373,15 +384,15 @@ def test_dense_launch_rejects_bad_arguments_without_a_gpu(lib):
 
 
 def test_dense_dk_path_query(lib):
-    """The dense call's dK path is the sparse operator's choice for top-k = the row length:
-    key-major in atomic mode, scatter in deterministic mode; an impossible request is refused."""
+    """The dense call's dK path is the sparse operator's choice for top-k = the row length
+    (key-major: the key range never exceeds the row length); an unknown request is refused."""
     assert sli.slikl_dense_grad_dk_path(dense_problem()) == sli.SLIKL_DK_KEYMAJOR
     assert sli.slikl_dense_grad_dk_path(dense_problem(N1=128)) == sli.SLIKL_DK_KEYMAJOR
-    assert sli.slikl_dense_grad_dk_path(dense_problem(deterministic=1)) == sli.SLIKL_DK_SCATTER
+    assert sli.slikl_dense_grad_dk_path(dense_problem(deterministic=1)) == sli.SLIKL_DK_KEYMAJOR
     assert sli.slikl_dense_grad_dk_path(dense_problem(), sli.make_options("scatter")) \
         == sli.SLIKL_DK_SCATTER
     with pytest.raises(sli.SliklError):
-        sli.slikl_dense_grad_dk_path(dense_problem(deterministic=1), sli.make_options("keymajor"))
+        sli.slikl_dense_grad_dk_path(dense_problem(), sli.make_options(7))
     with pytest.raises(sli.SliklError):
         sli.slikl_dense_grad_dk_path(dense_problem(mask_mode=1))
     assert sli.load_library().slikl_dense_grad_dk_path(ctypes.byref(dense_problem()), None, None) \

@@ -27,8 +27,8 @@ PROBLEMS = [
     (sli.SLIKL_BF16, sli.SLIKL_BSND, 4, 8192, 8192, 0, 0, 16, 128, 512, 1, sli.SLIKL_DK_AUTO),
     (sli.SLIKL_BF16, sli.SLIKL_BSND, 1, 256, 256, 0, 0, 8, 64, 64, 0, sli.SLIKL_DK_KEYMAJOR),
     (sli.SLIKL_BF16, sli.SLIKL_BSND, 1, 64, 64, 0, 0, 200, 128, 64, 0, sli.SLIKL_DK_AUTO),  # N1 too large
-    # key-major asked for in deterministic mode
-    (sli.SLIKL_BF16, sli.SLIKL_BSND, 1, 64, 64, 0, 0, 128, 128, 64, 1, sli.SLIKL_DK_KEYMAJOR),
+    # key-major asked for on a key range above its limit
+    (sli.SLIKL_BF16, sli.SLIKL_BSND, 1, 64, 131072, 0, 0, 128, 128, 64, 1, sli.SLIKL_DK_KEYMAJOR),
 ]
 
 

@@ -118,8 +118,8 @@ SMALL = [
 ]
 
 
-MODES = [(False, "scatter"), (False, "keymajor"), (True, "scatter")]
-MODE_IDS = ["scatter", "keymajor", "det"]
+MODES = [(False, "scatter"), (False, "keymajor"), (True, "scatter"), (True, "keymajor")]
+MODE_IDS = ["scatter", "keymajor", "det", "det_keymajor"]
 
 
 @pytest.mark.parametrize("case", SMALL, ids=lambda c: f"s{c['seed']}")
@@ -170,12 +170,13 @@ def cfg(cid):
 
 
 # dK modes compared in full at each full-size workload: the auto path (key-major where the
-# key range allows it), the scatter path, and the deterministic reduction on configs 1 and 4
+# key range allows it), the scatter path, and deterministic mode on configs 1 and 4 on both
+# paths (key-major with fixed-point records, and the sorted per-slot reduction)
 FULL_MODES = {
-    1: [(False, "auto"), (False, "scatter"), (True, "auto")],
+    1: [(False, "auto"), (False, "scatter"), (True, "auto"), (True, "scatter")],
     2: [(False, "auto"), (False, "scatter")],
     3: [(False, "auto")],
-    4: [(False, "auto"), (False, "scatter"), (True, "auto")],
+    4: [(False, "auto"), (False, "scatter"), (True, "auto"), (True, "scatter")],
 }
 
 
@@ -228,17 +229,30 @@ def bits(t):
     return t.view(torch.int16) if t.element_size() == 2 else t.view(torch.int32)
 
 
-@pytest.mark.parametrize("cid", [1, 4])
-def test_deterministic_bitwise_repeat(cid):
+def repeat_case(name):
+    if name == "dup":
+        # every key named about eight times per row: the key-major records sum many dI
+        return si.small(seed=41, layout="BSND", B=2, S1=64, S2=64, N1=32, D=128, K=512,
+                        pattern="dup")
+    return si.config(name)
+
+
+@pytest.mark.parametrize("cid,path", [(1, "auto"), (4, "auto"), (4, "scatter"), ("dup", "auto"),
+                                      ("dup", "scatter")],
+                         ids=["cfg1-keymajor", "cfg4-keymajor", "cfg4-sorted", "dup-keymajor",
+                              "dup-sorted"])
+def test_deterministic_bitwise_repeat(cid, path):
     """Deterministic mode: ten calls on the same inputs give bit-identical outputs."""
-    wl = si.config(cid)
+    wl = repeat_case(cid)
     dev = torch.device("cuda")
     t = {n: getattr(wl, n).to(dev) for n in ("q", "k", "w", "p", "idx")}
+    cuq = wl.cu_seqlens_q.to(dev) if wl.cu_seqlens_q is not None else None
+    cuk = wl.cu_seqlens_k.to(dev) if wl.cu_seqlens_k is not None else None
     first = None
     ws = None
     for rep in range(10):
-        res = sli.grad(t["q"], t["k"], t["w"], t["p"], t["idx"], deterministic=True,
-                       workspace=ws)
+        res = sli.grad(t["q"], t["k"], t["w"], t["p"], t["idx"], wl.layout, wl.layout, cuq, cuk,
+                       deterministic=True, workspace=ws, dk_path=path)
         ws = res["workspace"]
         cur = [bits(res[n]).clone() for n in ("dq", "dk", "dw", "softmax_out")]
         if first is None:
