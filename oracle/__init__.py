@@ -16,9 +16,11 @@ the key tensor has a single head, so
 * BSND: query row of (b, s) = b*S1 + s; key rows of batch b start at b*S2.
 * TND:  query rows of batch b start at cu_seqlens_q[b]; key rows at cu_seqlens_k[b].
 
-Every function here is pinned by tests/test_oracle_pins.py (finite differences of
-the KL loss, a dense one-hot brute force, torch fp64 autograd, closed forms and
-invariants).
+Every function here is pinned: the sparse operator by tests/test_oracle_pins.py (finite
+differences of the KL loss, a dense one-hot brute force, torch fp64 autograd, closed forms
+and invariants), the dense variant by tests/test_dense_oracle_pins.py, and the target
+distribution formed from the main attention by tests/test_main_p_oracle_pins.py (a library
+softmax, hand-worked cases, invariances, planted mistakes).
 """
 
 from __future__ import annotations
@@ -271,3 +273,76 @@ def dense_grad(wl, seq_used_q: Optional[Sequence[int]] = None,
     cuk = None if wl.cu_seqlens_k is None else wl.cu_seqlens_k.numpy()
     qs, ks = row_starts(wl.layout, wl.layout, wl.B, wl.S1, wl.S2, cuq, cuk)
     return dense_grad_arrays(q, k, w, p, qs, ks, wl.mask_mode, seq_used_q, seq_used_k)
+
+
+# ---------------------------------------------------------------------------------------------
+# The old fused variant's target distribution (SparseLightningIndexerGradKLLoss)
+#
+# aclnnSparseLightningIndexerKLLossGrad (功能说明 and 计算公式) says that the older operator
+# computed p inside its kernel from the main attention's scores, summed over the heads and
+# L1-normalised, and that attn_softmax_l1norm now carries that result. The pages give none of
+# that operator's inputs. The reading taken here: a main-attention query q_m [T1, Nm, Dm], one
+# main-attention key head k_m [T2, Dm] on the same key rows as k, and a softmax scale; each
+# head's attention is the softmax of scale * q_m[t, h] . k_m[j] over the row's valid top-k
+# slots (the keys a sparse main attention attends to); p is the sum over heads, divided by its
+# sum over the slots (the L1 norm). Invalid slots and rows without a valid slot get 0.
+# ---------------------------------------------------------------------------------------------
+
+def main_softmax_l1norm_arrays(q_m: np.ndarray, k_m: np.ndarray, idx: np.ndarray,
+                               q_start: np.ndarray, k_start: np.ndarray, scale: float,
+                               q_used: Optional[Sequence[int]] = None,
+                               k_used: Optional[Sequence[int]] = None) -> np.ndarray:
+    """p [T1, K] (fp64) from q_m [T1, Nm, Dm], k_m [T2, Dm], idx [T1, K]; valid slots and
+    padding rows as in grad_arrays (q_used / k_used the optional used lengths)."""
+    q_m = np.asarray(q_m, dtype=np.float64)
+    k_m = np.asarray(k_m, dtype=np.float64)
+    idx = np.asarray(idx)
+    T1, K = idx.shape
+    p = np.zeros((T1, K))
+    B = len(q_start) - 1
+    for b in range(B):
+        q0, q1 = int(q_start[b]), int(q_start[b + 1])
+        k0, k1 = int(k_start[b]), int(k_start[b + 1])
+        qlen = q1 - q0 if q_used is None else int(q_used[b])
+        klen = k1 - k0 if k_used is None else int(k_used[b])
+        for t in range(q0, q0 + qlen):
+            v = idx[t].astype(np.int64)
+            slots = np.nonzero((v >= 0) & (v < klen))[0]
+            if slots.size == 0:
+                continue
+            S = scale * (q_m[t] @ k_m[k0 + v[slots]].T)          # [Nm, valid slots]
+            A = np.exp(S - S.max(axis=1, keepdims=True))
+            A /= A.sum(axis=1, keepdims=True)                   # softmax over the slots, per head
+            hsum = A.sum(axis=0)                                # sum over the heads
+            p[t, slots] = hsum / np.abs(hsum).sum()             # L1 normalisation
+    return p
+
+
+def main_softmax_l1norm(wl, main, seq_used_q: Optional[Sequence[int]] = None,
+                        seq_used_k: Optional[Sequence[int]] = None) -> np.ndarray:
+    """main_softmax_l1norm_arrays on a slikl_inputs.Workload and its MainAttention inputs."""
+    T1, T2, K = wl.T1, wl.T2, wl.K
+    q_m = main.q.double().numpy().reshape(T1, main.Nm, main.Dm)
+    k_m = main.k.double().numpy().reshape(T2, main.Dm)
+    idx = wl.idx.numpy().reshape(T1, K)
+    cuq = None if wl.cu_seqlens_q is None else wl.cu_seqlens_q.numpy()
+    cuk = None if wl.cu_seqlens_k is None else wl.cu_seqlens_k.numpy()
+    qs, ks = row_starts(wl.layout, wl.layout, wl.B, wl.S1, wl.S2, cuq, cuk)
+    return main_softmax_l1norm_arrays(q_m, k_m, idx, qs, ks, main.scale, seq_used_q, seq_used_k)
+
+
+def grad_recompute_p(wl, main, seq_used_q: Optional[Sequence[int]] = None,
+                     seq_used_k: Optional[Sequence[int]] = None) -> dict:
+    """The old variant end to end: p from the main attention, then the backward of the KL loss
+    with that p (grad's outputs, loss included, plus p itself)."""
+    p = main_softmax_l1norm(wl, main, seq_used_q, seq_used_k)
+    T1, T2, N1, D, K = wl.T1, wl.T2, wl.N1, wl.D, wl.K
+    cuq = None if wl.cu_seqlens_q is None else wl.cu_seqlens_q.numpy()
+    cuk = None if wl.cu_seqlens_k is None else wl.cu_seqlens_k.numpy()
+    qs, ks = row_starts(wl.layout, wl.layout, wl.B, wl.S1, wl.S2, cuq, cuk)
+    out = grad_arrays(wl.q.double().numpy().reshape(T1, N1, D),
+                      wl.k.double().numpy().reshape(T2, D),
+                      wl.w.double().numpy().reshape(T1, N1), p,
+                      wl.idx.numpy().reshape(T1, K), qs, ks, q_used=seq_used_q, k_used=seq_used_k)
+    out["p"] = p
+    return out

@@ -413,3 +413,38 @@ def dense_visible_slots(wl: DenseWorkload) -> int:
         lq, lk = [wl.S1] * wl.B, [wl.S2] * wl.B
     return int(sum(min(_visible_count(wl.mask_mode, s, int(a), int(b)), wl.Ld)
                    for a, b in zip(lq, lk) for s in range(int(a))))
+
+
+# ----------------------------------------------------------------------------
+# main-attention inputs of the variant that forms p itself
+# ----------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class MainAttention:
+    """Main-attention query q [.., Nm, Dm] (same rows as the indexer's q) and one key head
+    k [.., 1, Dm] (same rows as the indexer's k), with the softmax scale."""
+
+    q: torch.Tensor
+    k: torch.Tensor
+    Nm: int
+    Dm: int
+    scale: float
+
+
+def main_attention(wl: Workload, Nm: int, Dm: int = 128, seed: int = 7,
+                   dtype: Optional[torch.dtype] = None, qk_scale: float = 1.0,
+                   scale: Optional[float] = None) -> MainAttention:
+    """Seeded N(0,1) * qk_scale draws in the workload's layout and dtype; softmax scale
+    1/sqrt(Dm) unless given."""
+    rng = np.random.default_rng(seed)
+    dt = wl.dtype if dtype is None else dtype
+    q = _round(rng.standard_normal((wl.T1, Nm, Dm)) * qk_scale, dt)
+    k = _round(rng.standard_normal((wl.T2, Dm)) * qk_scale, dt)
+    if wl.layout == "BSND":
+        q = q.reshape(wl.B, wl.S1, Nm, Dm)
+        k = k.reshape(wl.B, wl.S2, 1, Dm)
+    else:
+        q = q.reshape(wl.T1, Nm, Dm)
+        k = k.reshape(wl.T2, 1, Dm)
+    return MainAttention(q=q.contiguous(), k=k.contiguous(), Nm=Nm, Dm=Dm,
+                         scale=float(1.0 / np.sqrt(Dm)) if scale is None else float(scale))
