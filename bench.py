@@ -340,6 +340,31 @@ class DenseRunner(Runner):
                                   self.stream.cuda_stream, opt)
 
 
+class RecomputePRunner(Runner):
+    """A workload with main-attention inputs, called through slikl_grad_recompute_p (p formed
+    from the main attention, then the backward); timing, flush and status as Runner."""
+
+    def __init__(self, sli, wl, main, dev, stream, deterministic, dk_path):
+        super().__init__(sli, wl, dev, stream, deterministic, dk_path)
+        self.qm, self.km = main.q.to(dev), main.k.to(dev)
+        self.main = sli.make_main_attention(self.qm, main.scale)
+        self.p_out = torch_empty_like_f32(self.idx)
+        self.nbytes = sli.slikl_grad_recompute_p_workspace_size(self.pr, self.main, self.opt)
+
+    def step(self, evs=None, tn=None):
+        opt = self.opt if evs is None else self.sli.make_options(self.dk_path_arg,
+                                                                 *(int(e) for e in evs))
+        self.sli.slikl_grad_recompute_p(self.pr, self.main, tn or self.tn, self.qm.data_ptr(),
+                                        self.km.data_ptr(), self.p_out.data_ptr(),
+                                        self.ws.data_ptr(), self.nbytes,
+                                        self.stream.cuda_stream, opt)
+
+
+def torch_empty_like_f32(t):
+    import torch
+    return torch.empty(t.shape, dtype=torch.float32, device=t.device)
+
+
 def dense_stats(wl):
     """workload_stats for a dense problem: the slots are the Ld positions of every query row,
     the valid ones those the mask leaves visible; the compulsory bytes are every key row once,
@@ -361,13 +386,19 @@ def step_roofline_ms(stats, peaks, peak_tf):
 def per_config_lines(sli, dev, stream, flush, peaks, steps, warmup):
     """The other full-size workloads, timed the same way as the headline (device time, L2
     flushed before every step): configs 2, 3 and 4 on the auto dK path, the deterministic
-    reduction on configs 4 and 1, the 128-head causal workload, and the dense variant's causal
-    workload in both modes."""
+    reduction on configs 4 and 1, the 128-head causal workload, the dense variant's causal
+    workload in both modes, and the causal workload with p formed from a 128-head main
+    attention (the p kernel's time falls in the memset-and-split stage)."""
     import torch
     out = []
     for cid, det in ((2, False), (3, False), (4, False), (4, True), (1, True), ("n1_128", False),
-                     ("dense", False), ("dense", True)):
-        if cid == "n1_128":
+                     ("dense", False), ("dense", True), ("recompute_p", False)):
+        if cid == "recompute_p":
+            wl = si.config(1)
+            stats = workload_stats(wl)
+            r = RecomputePRunner(sli, wl, si.main_attention(wl, 128, 128, seed=123, qk_scale=0.5),
+                                 dev, stream, det, "auto")
+        elif cid == "n1_128":
             wl = si.wide_heads()
             stats = workload_stats(wl)
             r = Runner(sli, wl, dev, stream, det, "auto")

@@ -371,6 +371,59 @@ SLIKL_API slikl_status slikl_dense_grad(const slikl_dense_problem *problem,
 SLIKL_API slikl_status slikl_dense_grad_dk_path(const slikl_dense_problem *problem,
                                                 const slikl_options *options, int32_t *path);
 
+/*
+ * ---------------------------------------------------------------------------------------
+ * The older fused variant: p formed from the main attention
+ * (aclnnSparseLightningIndexerKLLossGrad, sections 功能说明 and 计算公式: the older operator,
+ * SparseLightningIndexerGradKLLoss, computed attn_softmax_l1norm inside its kernel from the
+ * main attention's scores, summed over the heads and L1-normalised, and output the loss).
+ * The pages give none of that operator's inputs; the reading taken here:
+ *   - a main-attention query q_main with Nm heads of Dm, laid out like q
+ *     (BSND [B][S1][Nm][Dm] or TND [T1][Nm][Dm]), and one main-attention key head k_main on
+ *     the same key rows as k (BSND [B][S2][1][Dm] or TND [T2][1][Dm]), both of problem->dtype;
+ *   - for query row t and head h, A_h(t, j) = softmax over the row's valid slots j of
+ *     scale * q_main[t, h] . k_main[key(t, j)] (the keys a sparse main attention attends to;
+ *     valid slots as for the sparse operator, used lengths included);
+ *   - p(t, j) = sum_h A_h(t, j) / sum_j sum_h A_h(t, j) = sum_h A_h(t, j) / Nm, 0 at invalid
+ *     slots and on rows without a valid slot.
+ * The backward then runs on that p exactly as slikl_grad_ex; options->loss returns the
+ * per-row KL loss the older operator output.
+ * ---------------------------------------------------------------------------------------
+ */
+typedef struct slikl_main_attention {
+    int32_t Nm;                 /* main-attention query heads, 1..128 */
+    int32_t Dm;                 /* their head dimension: 64 or 128 */
+    float scale;                /* softmax scale of the main attention (e.g. 1 / sqrt(Dm)) */
+    int32_t reserved;           /* 0 */
+} slikl_main_attention;
+
+/*
+ * Phase 1 (host only, no CUDA call): the workspace size of slikl_grad_recompute_p, equal to
+ * slikl_grad_workspace_size_ex for the same problem and options.
+ * Errors: SLIKL_ERR_PARAM_NULLPTR (main NULL), SLIKL_ERR_PARAM_INVALID (Nm outside 1..128,
+ * Dm not 64 or 128, scale not finite, reserved != 0), and those of
+ * slikl_grad_workspace_size_ex.
+ */
+SLIKL_API slikl_status slikl_grad_recompute_p_workspace_size(const slikl_problem *problem,
+                                                             const slikl_main_attention *main,
+                                                             const slikl_options *options,
+                                                             size_t *workspace_bytes);
+/*
+ * Phase 2: forms p from q_main and k_main (device, 16-byte aligned, layouts above) into
+ * p_out (device fp32 [T1][topk], 4-byte aligned, written in full), then runs the backward
+ * of slikl_grad_ex with it; tensors->attn_softmax_l1norm is not read. Same streams,
+ * workspace and status-word rules as slikl_grad_ex.
+ * Errors: as phase 1; SLIKL_ERR_PARAM_NULLPTR for NULL tensors, q_main or p_out (when there
+ * are query rows) or k_main (when there are key rows); SLIKL_ERR_PARAM_INVALID for a
+ * misaligned q_main, k_main or p_out; and those of slikl_grad_ex.
+ */
+SLIKL_API slikl_status slikl_grad_recompute_p(const slikl_problem *problem,
+                                              const slikl_main_attention *main,
+                                              const slikl_tensors *tensors, const void *q_main,
+                                              const void *k_main, float *p_out, void *workspace,
+                                              size_t workspace_bytes, void *stream,
+                                              const slikl_options *options);
+
 /* Human-readable name of a status code (static string, never NULL). */
 SLIKL_API const char *slikl_status_string(slikl_status status);
 

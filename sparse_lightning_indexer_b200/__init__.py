@@ -49,7 +49,8 @@ EXPORTED = ("slikl_grad_workspace_size", "slikl_grad", "slikl_grad_with_events",
             "slikl_read_device_status",
             "slikl_grad_metadata_size", "slikl_grad_metadata_workspace_size",
             "slikl_grad_metadata", "slikl_status_string", "slikl_grad_noalloc",
-            "slikl_dense_grad_workspace_size", "slikl_dense_grad", "slikl_dense_grad_dk_path")
+            "slikl_dense_grad_workspace_size", "slikl_dense_grad", "slikl_dense_grad_dk_path",
+            "slikl_grad_recompute_p_workspace_size", "slikl_grad_recompute_p")
 
 SLIKL_NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -81,6 +82,11 @@ class slikl_dense_tensors(ctypes.Structure):
     _fields_ = [(name, ctypes.c_void_p) for name in
                 ("q", "k", "w", "attn_softmax_l1norm", "cu_seqlens_q", "cu_seqlens_k", "dq",
                  "dk", "dw", "softmax_out")]
+
+
+class slikl_main_attention(ctypes.Structure):
+    _fields_ = [("Nm", ctypes.c_int32), ("Dm", ctypes.c_int32), ("scale", ctypes.c_float),
+                ("reserved", ctypes.c_int32)]
 
 
 class slikl_options(ctypes.Structure):
@@ -152,6 +158,13 @@ def load_library() -> ctypes.CDLL:
         lib.slikl_dense_grad_dk_path.argtypes = [P(slikl_dense_problem), P(slikl_options),
                                                  P(ctypes.c_int32)]
         lib.slikl_dense_grad_dk_path.restype = ctypes.c_int32
+        lib.slikl_grad_recompute_p_workspace_size.argtypes = [
+            P(slikl_problem), P(slikl_main_attention), P(slikl_options), P(ctypes.c_size_t)]
+        lib.slikl_grad_recompute_p_workspace_size.restype = ctypes.c_int32
+        lib.slikl_grad_recompute_p.argtypes = [P(slikl_problem), P(slikl_main_attention),
+                                               P(slikl_tensors), VP, VP, VP, VP, ctypes.c_size_t,
+                                               VP, P(slikl_options)]
+        lib.slikl_grad_recompute_p.restype = ctypes.c_int32
         lib.slikl_status_string.argtypes = [ctypes.c_int32]
         lib.slikl_status_string.restype = ctypes.c_char_p
         for name in ("slikl_grad_workspace_size", "slikl_grad", "slikl_grad_with_events",
@@ -388,6 +401,96 @@ def grad(q, k, w, attn_softmax_l1norm, sparse_indices, layout_q="BSND", layout_k
     if loss_t is not None:
         res["loss"] = loss_t
     return res
+
+
+def slikl_grad_recompute_p_workspace_size(problem: slikl_problem, main: slikl_main_attention,
+                                          options: Optional[slikl_options] = None) -> int:
+    n = ctypes.c_size_t(0)
+    rc = load_library().slikl_grad_recompute_p_workspace_size(
+        ctypes.byref(problem), ctypes.byref(main),
+        ctypes.byref(options) if options is not None else None, ctypes.byref(n))
+    if rc != SLIKL_OK:
+        raise SliklError(rc, "slikl_grad_recompute_p_workspace_size")
+    return int(n.value)
+
+
+def slikl_grad_recompute_p(problem: slikl_problem, main: slikl_main_attention,
+                           tensors: slikl_tensors, q_main: int, k_main: int, p_out: int,
+                           workspace: int, workspace_bytes: int, stream: int = 0,
+                           options: Optional[slikl_options] = None) -> None:
+    rc = load_library().slikl_grad_recompute_p(
+        ctypes.byref(problem), ctypes.byref(main), ctypes.byref(tensors), q_main, k_main, p_out,
+        workspace, workspace_bytes, stream, ctypes.byref(options) if options is not None else None)
+    if rc != SLIKL_OK:
+        raise SliklError(rc, "slikl_grad_recompute_p")
+
+
+def make_main_attention(q_main: torch.Tensor, scale: float) -> slikl_main_attention:
+    """Main-attention shape from q_main [.., Nm, Dm] and the softmax scale."""
+    m = slikl_main_attention()
+    m.Nm, m.Dm = int(q_main.shape[-2]), int(q_main.shape[-1])
+    m.scale = float(scale)
+    m.reserved = 0
+    return m
+
+
+def grad_recompute_p(q, k, w, sparse_indices, q_main, k_main, scale, layout_q="BSND",
+                     layout_k="BSND", cu_seqlens_q=None, cu_seqlens_k=None, deterministic=False,
+                     stream=None, workspace=None, dk_path="auto", key_range_bound=0, loss=False,
+                     seq_used_q=None, seq_used_k=None):
+    """Run slikl_grad_recompute_p on CUDA tensors: p from the main attention (q_main
+    [.., Nm, Dm], k_main [.., 1, Dm], softmax scale), then the backward with it.
+    Returns dict(dq, dk, dw, softmax_out, p, workspace[, loss])."""
+    B = None
+    if layout_q == "TND":
+        B = cu_seqlens_q.numel() - 1
+    elif layout_k == "TND":
+        B = cu_seqlens_k.numel() - 1
+    pr = make_problem(q, k, sparse_indices, layout_q, layout_k, deterministic, B,
+                      key_range_bound)
+    main = make_main_attention(q_main, scale)
+    loss_t = torch.empty(pr.T1, dtype=torch.float32, device=q.device) if loss else None
+    opt = make_options(dk_path, loss=loss_t.data_ptr() if loss_t is not None else 0,
+                       seq_used_q=_ptr(seq_used_q) or 0, seq_used_k=_ptr(seq_used_k) or 0)
+    nbytes = slikl_grad_recompute_p_workspace_size(pr, main, opt)
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device)
+    p = torch.empty(sparse_indices.shape, dtype=torch.float32, device=q.device)
+    out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dw=torch.empty_like(w),
+               softmax_out=torch.empty(sparse_indices.shape, dtype=torch.float32, device=q.device))
+    tn = slikl_tensors()
+    tn.q, tn.k, tn.w = _ptr(q), _ptr(k), _ptr(w)
+    tn.attn_softmax_l1norm = None
+    tn.sparse_indices = _ptr(sparse_indices)
+    tn.cu_seqlens_q = _ptr(cu_seqlens_q) if layout_q == "TND" else None
+    tn.cu_seqlens_k = _ptr(cu_seqlens_k) if layout_k == "TND" else None
+    tn.dq, tn.dk, tn.dw = _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dw"])
+    tn.softmax_out = _ptr(out["softmax_out"])
+    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+    slikl_grad_recompute_p(pr, main, tn, _ptr(q_main), _ptr(k_main), p.data_ptr(),
+                           workspace.data_ptr(), workspace.numel(), s.cuda_stream, opt)
+    res = dict(out)
+    res["p"] = p
+    res["workspace"] = workspace
+    if loss_t is not None:
+        res["loss"] = loss_t
+    return res
+
+
+def grad_recompute_p_workload(wl, main, device="cuda", deterministic=False, stream=None,
+                              dk_path="auto", loss=False, seq_used_q=None, seq_used_k=None):
+    """Move a slikl_inputs.Workload and its MainAttention to the device and run
+    grad_recompute_p (seq_used_q / seq_used_k: host lists of B used lengths, or None)."""
+    dev = torch.device(device)
+    t = {n: getattr(wl, n).to(dev) for n in ("q", "k", "w", "idx")}
+    cuq = wl.cu_seqlens_q.to(dev) if wl.cu_seqlens_q is not None else None
+    cuk = wl.cu_seqlens_k.to(dev) if wl.cu_seqlens_k is not None else None
+    uq = None if seq_used_q is None else torch.tensor(list(seq_used_q), dtype=torch.int32, device=dev)
+    uk = None if seq_used_k is None else torch.tensor(list(seq_used_k), dtype=torch.int32, device=dev)
+    return grad_recompute_p(t["q"], t["k"], t["w"], t["idx"], main.q.to(dev), main.k.to(dev),
+                            main.scale, wl.layout, wl.layout, cuq, cuk, deterministic, stream,
+                            dk_path=dk_path, key_range_bound=key_range_bound_of(wl), loss=loss,
+                            seq_used_q=uq, seq_used_k=uk)
 
 
 def key_range_bound_of(wl) -> int:

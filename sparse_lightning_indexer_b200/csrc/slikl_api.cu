@@ -217,6 +217,28 @@ struct DenseLayout {
     size_t sparse, idx, flag, total;
 };
 
+// The variant that forms p from the main attention: its inputs, checked on the host.
+struct MainP {
+    const void *q_main, *k_main;
+    float *p_out;
+    float scale;
+    int Nm, Dm;
+};
+
+slikl_status check_main(const slikl_main_attention *m) {
+    if (!m) return SLIKL_ERR_PARAM_NULLPTR;
+    if (m->Nm < 1 || m->Nm > 128 || (m->Dm != 64 && m->Dm != 128) || m->reserved != 0 ||
+        !(m->scale == m->scale) || m->scale > 3.0e38f || m->scale < -3.0e38f)
+        return SLIKL_ERR_PARAM_INVALID;
+    return SLIKL_OK;
+}
+
+// Validation, workspace layout and the launch sequence of one call; with mp, the main
+// attention's target distribution is formed right after the work split and used as p.
+slikl_status run_grad(const slikl_problem *problem, const slikl_tensors *tensors,
+                      void *workspace, size_t workspace_bytes, void *stream,
+                      const slikl_options *options, const MainP *mp);
+
 }  // namespace
 
 slikl_status dense_layout(const slikl_problem *sp, const slikl_options *options, int64_t ld,
@@ -284,6 +306,47 @@ slikl_status slikl_grad_with_events(const slikl_problem *problem, const slikl_te
 slikl_status slikl_grad_ex(const slikl_problem *problem, const slikl_tensors *tensors,
                            void *workspace, size_t workspace_bytes, void *stream,
                            const slikl_options *options) {
+    return run_grad(problem, tensors, workspace, workspace_bytes, stream, options, nullptr);
+}
+
+slikl_status slikl_grad_recompute_p_workspace_size(const slikl_problem *problem,
+                                                   const slikl_main_attention *main,
+                                                   const slikl_options *options,
+                                                   size_t *workspace_bytes) {
+    const slikl_status st = check_main(main);
+    if (st != SLIKL_OK) return st;
+    return slikl_grad_workspace_size_ex(problem, options, workspace_bytes);
+}
+
+slikl_status slikl_grad_recompute_p(const slikl_problem *problem, const slikl_main_attention *main,
+                                    const slikl_tensors *tensors, const void *q_main,
+                                    const void *k_main, float *p_out, void *workspace,
+                                    size_t workspace_bytes, void *stream,
+                                    const slikl_options *options) {
+    slikl_status st = check_main(main);
+    if (st != SLIKL_OK) return st;
+    Derived dv;
+    st = validate(problem, &dv);
+    if (st != SLIKL_OK) return st;
+    if (!tensors) return SLIKL_ERR_PARAM_NULLPTR;
+    if ((dv.T1 > 0 && (!q_main || !p_out)) || (dv.T2 > 0 && !k_main)) return SLIKL_ERR_PARAM_NULLPTR;
+    if ((reinterpret_cast<uintptr_t>(q_main) & 15) || (reinterpret_cast<uintptr_t>(k_main) & 15) ||
+        (reinterpret_cast<uintptr_t>(p_out) & 3))
+        return SLIKL_ERR_PARAM_INVALID;
+    slikl_tensors tn = *tensors;
+    tn.attn_softmax_l1norm = p_out;            // the computed p is the backward's target
+    const MainP mp{q_main, k_main, p_out, main->scale, main->Nm, main->Dm};
+    return run_grad(problem, &tn, workspace, workspace_bytes, stream, options, &mp);
+}
+
+}  // extern "C"
+
+namespace slikl {
+namespace {
+
+slikl_status run_grad(const slikl_problem *problem, const slikl_tensors *tensors,
+                      void *workspace, size_t workspace_bytes, void *stream,
+                      const slikl_options *options, const MainP *mp) {
     Derived dv;
     slikl_status st = validate(problem, &dv);
     if (st != SLIKL_OK) return st;
@@ -323,6 +386,9 @@ slikl_status slikl_grad_ex(const slikl_problem *problem, const slikl_tensors *te
         return SLIKL_ERR_CUDA;
     if (launch_metadata(P, workers, 1, s) != cudaSuccess) return SLIKL_ERR_CUDA;
     if (P.km && launch_km_metadata(P, km_workers, s) != cudaSuccess) return SLIKL_ERR_CUDA;
+    if (mp && launch_main_p(P, mp->q_main, mp->k_main, mp->p_out, mp->scale, mp->Nm, mp->Dm,
+                            workers, s) != cudaSuccess)
+        return SLIKL_ERR_CUDA;
     if (fused_begin && cudaEventRecord(static_cast<cudaEvent_t>(fused_begin), s) != cudaSuccess)
         return SLIKL_ERR_CUDA;
     if (dv.T1 > 0 && launch_fused_sm100(P, workers, s) != cudaSuccess) return SLIKL_ERR_CUDA;
@@ -345,6 +411,11 @@ slikl_status slikl_grad_ex(const slikl_problem *problem, const slikl_tensors *te
         return SLIKL_ERR_CUDA;
     return SLIKL_OK;
 }
+
+}  // namespace
+}  // namespace slikl
+
+extern "C" {
 
 slikl_status slikl_read_device_status(const void *workspace, void *stream, uint32_t *flags) {
     if (!flags) return SLIKL_ERR_INNER_NULLPTR;

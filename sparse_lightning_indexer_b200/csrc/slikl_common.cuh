@@ -175,6 +175,8 @@ cudaError_t launch_deterministic_reduce(const Params &P, cudaStream_t s);
 cudaError_t launch_km_metadata(const Params &P, int workers, cudaStream_t s);
 cudaError_t launch_dk_keymajor(const Params &P, int workers, cudaStream_t s);
 cudaError_t launch_km_det_combine(const Params &P, int workers, cudaStream_t s);
+cudaError_t launch_main_p(const Params &P, const void *q_main, const void *k_main, float *p_out,
+                          float scale, int Nm, int Dm, int workers, cudaStream_t s);
 cudaError_t launch_dense_indices(int32_t *idx, int64_t T1, int64_t B, int64_t S1, int64_t S2,
                                  int Ld, int layout_q, int layout_k, int mask,
                                  const int32_t *cu_q, const int32_t *cu_k, const int32_t *used_q,

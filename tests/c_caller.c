@@ -44,6 +44,9 @@ static void layouts(void) {
     FIELD(slikl_dense_tensors, cu_seqlens_k); FIELD(slikl_dense_tensors, dq);
     FIELD(slikl_dense_tensors, dk); FIELD(slikl_dense_tensors, dw);
     FIELD(slikl_dense_tensors, softmax_out);
+    printf("size slikl_main_attention %zu\n", sizeof(slikl_main_attention));
+    FIELD(slikl_main_attention, Nm); FIELD(slikl_main_attention, Dm);
+    FIELD(slikl_main_attention, scale); FIELD(slikl_main_attention, reserved);
 }
 
 int main(int argc, char **argv) {

@@ -397,3 +397,50 @@ def test_dense_dk_path_query(lib):
         sli.slikl_dense_grad_dk_path(dense_problem(mask_mode=1))
     assert sli.load_library().slikl_dense_grad_dk_path(ctypes.byref(dense_problem()), None, None) \
         == sli.SLIKL_ERR_INNER_NULLPTR
+
+
+# ---------------------------------------------------------------------------
+# variant that forms p from the main attention: host-side checks (no CUDA call)
+# ---------------------------------------------------------------------------
+
+def main_attn(**kw):
+    m = sli.slikl_main_attention()
+    m.Nm, m.Dm, m.scale, m.reserved = 16, 128, 0.125, 0
+    for f, v in kw.items():
+        setattr(m, f, v)
+    return m
+
+
+def test_recompute_p_workspace_and_validation(lib):
+    pr = base_problem()
+    opt = sli.make_options("auto")
+    assert sli.slikl_grad_recompute_p_workspace_size(pr, main_attn(), opt) == \
+        sli.slikl_grad_workspace_size_ex(pr, opt)
+    n = ctypes.c_size_t(0)
+    for bad in (dict(Nm=0), dict(Nm=129), dict(Dm=96), dict(reserved=1),
+                dict(scale=float("nan")), dict(scale=float("inf"))):
+        rc = lib.slikl_grad_recompute_p_workspace_size(
+            ctypes.byref(pr), ctypes.byref(main_attn(**bad)), None, ctypes.byref(n))
+        assert rc == sli.SLIKL_ERR_PARAM_INVALID, bad
+    assert lib.slikl_grad_recompute_p_workspace_size(ctypes.byref(pr), None, None,
+                                                     ctypes.byref(n)) == sli.SLIKL_ERR_PARAM_NULLPTR
+
+
+def test_recompute_p_launch_rejects_bad_arguments_without_a_gpu(lib):
+    pr = base_problem()
+    m = main_attn()
+    tn = fake_tensors()
+    need = sli.slikl_grad_recompute_p_workspace_size(pr, m)
+
+    def rc(q_main, k_main, p_out, tensors=tn, ws=1 << 20, nbytes=need):
+        return lib.slikl_grad_recompute_p(ctypes.byref(pr), ctypes.byref(m),
+                                          ctypes.byref(tensors) if tensors is not None else None,
+                                          q_main, k_main, p_out, ws, nbytes, None, None)
+
+    assert rc(0x1000, 0x2000, 0x3000, tensors=None) == sli.SLIKL_ERR_PARAM_NULLPTR
+    assert rc(None, 0x2000, 0x3000) == sli.SLIKL_ERR_PARAM_NULLPTR
+    assert rc(0x1000, None, 0x3000) == sli.SLIKL_ERR_PARAM_NULLPTR
+    assert rc(0x1000, 0x2000, None) == sli.SLIKL_ERR_PARAM_NULLPTR
+    assert rc(0x1008, 0x2000, 0x3000) == sli.SLIKL_ERR_PARAM_INVALID      # q_main not 16-aligned
+    assert rc(0x1000, 0x2000, 0x3002) == sli.SLIKL_ERR_PARAM_INVALID      # p_out not 4-aligned
+    assert rc(0x1000, 0x2000, 0x3000, nbytes=need - 1) == sli.SLIKL_ERR_WORKSPACE_TOO_SMALL

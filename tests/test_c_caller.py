@@ -50,7 +50,8 @@ def test_struct_layouts_match_the_binding(c_output):
     mirrors = {"slikl_problem": sli.slikl_problem, "slikl_tensors": sli.slikl_tensors,
                "slikl_options": sli.slikl_options,
                "slikl_dense_problem": sli.slikl_dense_problem,
-               "slikl_dense_tensors": sli.slikl_dense_tensors}
+               "slikl_dense_tensors": sli.slikl_dense_tensors,
+               "slikl_main_attention": sli.slikl_main_attention}
     seen = set()
     for line in c_output:
         parts = line.split()
