@@ -147,7 +147,7 @@ def raw_elapsed_ms(a, b):
 
 # DRAM bytes (read + write) of one fused-kernel launch on the headline workload, read from an
 # ncu capture of that launch (dram__bytes_read.sum + dram__bytes_write.sum). The figure holds
-# only while the kernel's sources are the ones captured (hash of the three files below);
+# only while the kernel's sources are the ones captured (hash of the four files below);
 # otherwise the traffic is reported as unknown (null).
 FUSED_TRAFFIC = {"sources_sha256_16": "585d0d6c2ddf69bf", "workload_config": 1,
                  "dk_path": "keymajor", "bytes": 121.169152e6 + 193.834496e6}
@@ -156,7 +156,8 @@ FUSED_TRAFFIC = {"sources_sha256_16": "585d0d6c2ddf69bf", "workload_config": 1,
 def fused_sources_hash():
     import hashlib
     h = hashlib.sha256()
-    for f in ("slikl_fused_sm100.cu", "slikl_sm100.cuh", "slikl_common.cuh"):
+    for f in ("slikl_fused_sm100.cu", "slikl_fused_pair_sm100.cu", "slikl_sm100.cuh",
+              "slikl_common.cuh"):
         with open(os.path.join(ROOT, "sparse_lightning_indexer_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -575,7 +576,9 @@ def main():
                                        f"hbm {peaks['hbm_gbs']} GB/s ({peak_src})"},
             "roofline": {"bound": "tensor", "achieved": achieved_tf, "peak": peak_tf,
                          "unit": "TFLOP/s", "frac": achieved_tf / peak_tf, "traffic": traffic,
-                         "kernel": "fused_sm100 (fused per-token kernel)",
+                         "kernel": ("fused_pair_sm100 (fused per-token kernel, items of two slot "
+                                    "tiles)" if dk_path == "keymajor" and wl.N1 <= 64 else
+                                    "fused_sm100 (fused per-token kernel)"),
                          "algorithmic_flop_per_launch": kflop,
                          "flop_basis": "valid slots (tiles without a valid slot are skipped)",
                          "achieved_nominal_slots": kflop_nom / k_avg / 1e12,

@@ -170,6 +170,7 @@ __device__ __forceinline__ int32_t slot_row(int32_t v, int32_t kbase, int32_t kl
 // kernels (defined in the .cu files)
 cudaError_t launch_metadata(const Params &P, int workers, int mode, cudaStream_t s);
 cudaError_t launch_fused_sm100(const Params &P, int workers, cudaStream_t s);
+cudaError_t launch_fused_pair_sm100(const Params &P, int workers, cudaStream_t s);
 cudaError_t launch_cast(const Params &P, cudaStream_t s);
 cudaError_t launch_deterministic_reduce(const Params &P, cudaStream_t s);
 cudaError_t launch_km_metadata(const Params &P, int workers, cudaStream_t s);

@@ -888,6 +888,8 @@ cudaError_t launch_n(const Params &P, int workers, cudaStream_t s) {
 // 64 tiles): every problem the entry points accept.
 cudaError_t launch_fused_sm100(const Params &P, int workers, cudaStream_t s) {
     if (P.N1 > 128 || (P.D != 64 && P.D != 128) || P.K > 64 * 128) return cudaErrorInvalidValue;
+    // record mode up to 64 heads: items of two slot tiles
+    if (P.km && P.N1 <= 64) return launch_fused_pair_sm100(P, workers, s);
     if (P.N1 <= 16) return launch_n<16>(P, workers, s);
     if (P.N1 <= 32) return launch_n<32>(P, workers, s);
     if (P.N1 <= 64) return launch_n<64>(P, workers, s);

@@ -335,6 +335,17 @@ def test_protocol_finishes_and_is_safe(rec):
             assert stuck is None, f"deadlock with masks {masks}: {stuck}"
 
 
+def test_protocol_paired_items_finishes_and_is_safe():
+    """The record-mode kernel with items of two slot tiles: two K stages, two S buffers, one
+    dS tile (the same barriers and hand-offs over fewer buffers)."""
+    rnd = random.Random(20261204)
+    cases = EDGE_MASKS + [random_masks(rnd) for _ in range(250)]
+    for i, masks in enumerate(cases):
+        for seed in range(3):
+            stuck = run(masks, True, seed=1000 * i + seed, stages=2, ns=2, nd=1)
+            assert stuck is None, f"deadlock with masks {masks}: {stuck}"
+
+
 @pytest.mark.parametrize("rec", [False, True], ids=["scatter", "record"])
 def test_protocol_128_heads_finishes_and_is_safe(rec):
     """The 128-head instances: three K stages, one dS tile (and dK^T buffer), and one S^T
