@@ -149,8 +149,8 @@ def raw_elapsed_ms(a, b):
 # ncu capture of that launch (dram__bytes_read.sum + dram__bytes_write.sum). The figure holds
 # only while the kernel's sources are the ones captured (hash of the four files below);
 # otherwise the traffic is reported as unknown (null).
-FUSED_TRAFFIC = {"sources_sha256_16": "585d0d6c2ddf69bf", "workload_config": 1,
-                 "dk_path": "keymajor", "bytes": 121.169152e6 + 193.834496e6}
+FUSED_TRAFFIC = {"sources_sha256_16": "42232891e61ee697", "workload_config": 1,
+                 "dk_path": "keymajor", "bytes": 122.011904e6 + 193.474560e6}
 
 
 def fused_sources_hash():
@@ -541,10 +541,14 @@ def main():
     step_avg = t_total / args.steps
     t_roof = step_roofline_ms(stats, peaks, peak_tf) / 1e3
     t_roof_nom = step_roofline_ms(stats, peaks, NOMINAL_BF16_TFLOPS) / 1e3
-    # our kernels per call: 3 work-split + fused + (cast | sort init, 3 per radix pass,
-    # row pointers, segmented reduce); the key-major path adds 2 metadata kernels and its dK kernel
+    # our kernels per call: 3 work-split + fused + cast; the key-major path adds 2 metadata
+    # kernels and its dK kernel (and in deterministic mode the combine of cut runs); the sorted
+    # reduction replaces the cast by sort init, 3 per radix pass, row pointers and the
+    # segmented reduce
     launches_per_step = 5 + (3 if dk_path == "keymajor" else 0)
-    if args.deterministic:
+    if args.deterministic and dk_path == "keymajor":
+        launches_per_step += 1
+    elif args.deterministic:
         passes = (int(wl.T2).bit_length() + 7) // 8
         launches_per_step = 3 + 1 + 1 + 3 * passes + 2
     cpu = None

@@ -42,7 +42,7 @@ constexpr int kMpThreads = 256;
 constexpr int kMpStages = 2;             // key-row stages of 128 rows x 256 B
 constexpr int kMpTmemCols = 256;         // two S buffers [128 heads x 128 slots]
 constexpr int kMpStageBytes = 128 * 256;
-constexpr int kEStride = 129;            // floats per head row of the weight tile
+constexpr int kEStride = 132;            // floats per head row of the weight tile (16-byte rows)
 constexpr int kMaskRing = 4;
 
 struct MpBarriers {
@@ -309,25 +309,39 @@ __global__ void __launch_bounds__(kMpThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars->s_empty[b]);
             } else {
-                // weights of head h into row h of the tile (heads past Nm are never summed)
-                float *erow = E + h * kEStride;
+                // weights of head h into row h of the tile (heads past Nm are never summed);
+                // 16-byte stores: lanes h and h + 8 share banks, four wavefronts per store
+                float4 *erow = reinterpret_cast<float4 *>(E + h * kEStride);
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     float v[32];
                     tmem_ld32(sa + 32 * c, v);
                     tmem_wait_ld();
                     const uint32_t bits = c == 0 ? w0 : (c == 1 ? w1 : (c == 2 ? w2 : w3));
+                    float e[32];
 #pragma unroll
                     for (int k = 0; k < 32; ++k)
-                        erow[32 * c + k] = ((bits >> k) & 1u) ? __expf(A.scale * v[k] - m) * iz : 0.f;
+                        e[k] = ((bits >> k) & 1u) ? __expf(A.scale * v[k] - m) * iz : 0.f;
+#pragma unroll
+                    for (int k = 0; k < 32; k += 4)
+                        erow[(32 * c + k) >> 2] = make_float4(e[k], e[k + 1], e[k + 2], e[k + 3]);
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars->s_empty[b]);
                 if (!group_sync(&bars->sm_sync, ph, &abort_flag, P.status)) { ok = false; break; }
-                // slot h of the tile: its weights summed over the heads in order
-                float acc = 0.f;
-                for (int hh = 0; hh < A.Nm; ++hh) acc += E[hh * kEStride + h];
+                // slot h of the tile: its weights summed over the heads in a fixed order (eight
+                // interleaved partial sums, combined pairwise), so the loads overlap
+                float a8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                int hh = 0;
+                for (; hh + 8 <= A.Nm; hh += 8) {
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) a8[u] += E[(hh + u) * kEStride + h];
+                }
+#pragma unroll
+                for (int u = 0; u < 7; ++u)                   // the last Nm % 8 heads
+                    if (hh + u < A.Nm) a8[u] += E[(hh + u) * kEStride + h];
+                const float acc = ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
                 const int j = it.tile * 128 + h;
                 if (j < K) A.p[(int64_t)it.t * K + j] = acc * inv_nm;
                 if (!group_sync(&bars->sm_sync, ph, &abort_flag, P.status)) { ok = false; break; }
