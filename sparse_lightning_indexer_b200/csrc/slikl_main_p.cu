@@ -20,12 +20,15 @@
 // In pass 2 each head writes its weights into an fp32 [heads x slots] tile in shared memory
 // and each slot sums its column over the heads in a fixed order.
 //
-// Warp roles (256 threads):
+// Warp roles (384 threads):
 //   warps 0-2   producers: the key rows of every tile gathered with cp.async (16-byte chunks,
 //               zero-fill for invalid slots); warp 0 also loads q_m[t] by TMA (heads past Nm
 //               read as zero) and writes the tile's valid-slot mask into a 4-entry ring
 //   warp 3      MMA issuer (one thread) and TMEM owner
-//   warps 4-7   softmax group: thread = head (pass 1 and 2), then thread = slot (column sums)
+//   warps 4-11  softmax groups: thread = head (pass 1 and 2; warps 4-7 take the slot columns
+//               0-63, warps 8-11 the columns 64-127, two warps per TMEM lane quadrant so
+//               that the exponentials of a sub-partition come from two instruction streams),
+//               then thread = slot (column sums)
 // Every mbarrier wait is bounded (about one second of SM clock); on expiry the CTA sets
 // SLIKL_DEV_WAIT_TIMEOUT, every role stops, in-flight copies and MMAs are drained, TMEM is
 // freed and the kernel returns.
@@ -38,7 +41,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kMpThreads = 256;
+constexpr int kMpThreads = 384;
 constexpr int kMpStages = 2;             // key-row stages of 128 rows x 256 B
 constexpr int kMpTmemCols = 256;         // two S buffers [128 heads x 128 slots]
 constexpr int kMpStageBytes = 128 * 256;
@@ -50,7 +53,7 @@ struct MpBarriers {
     uint64_t q_full[2], q_empty[2];                     // q_m tiles: producer 0 -> MMA -> producer 0
     uint64_t s_full[2], s_empty[2];                     // S in TMEM: MMA -> softmax -> MMA
     uint64_t mask_full[kMaskRing];                      // tile masks: producer 0 -> softmax
-    uint64_t sm_sync;                                   // the 4 softmax warps
+    uint64_t sm_sync;                                   // the 8 softmax warps
     uint64_t drain;
 };
 
@@ -150,10 +153,10 @@ __global__ void __launch_bounds__(kMpThreads, 1)
             mbar_init(&bars->q_full[b], 1);
             mbar_init(&bars->q_empty[b], 1);
             mbar_init(&bars->s_full[b], 1);
-            mbar_init(&bars->s_empty[b], 4);
+            mbar_init(&bars->s_empty[b], 8);
         }
         for (int r = 0; r < kMaskRing; ++r) mbar_init(&bars->mask_full[r], 1);
-        mbar_init(&bars->sm_sync, 4);
+        mbar_init(&bars->sm_sync, 8);
         mbar_init(&bars->drain, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -213,13 +216,27 @@ __global__ void __launch_bounds__(kMpThreads, 1)
                 }
             }
             const uint32_t dst = smem_u32(smem + SP.kv + s * kMpStageBytes) + (chunk >> 3) * 16384;
+            // this warp's row groups i = warp, warp + 3, ...: every slot index into registers
+            // first (one load latency per tile), then the copies back to back
             constexpr int kGroups = 128 / kRowsPerPass;
-            for (int i = warp; i < kGroups; i += kProd) {
+            constexpr int kPer = (kGroups + kProd - 1) / kProd;
+            int32_t vv[kPer];
+#pragma unroll
+            for (int j = 0; j < kPer; ++j) {
+                const int i = warp + kProd * j;
                 const int r = rsub + kRowsPerPass * i;
-                const int32_t v = r < jlim ? irow[r] : -1;
-                const bool valid = v >= 0 && v < kl;
-                const char *src = kbase_ptr + (valid ? ((int64_t)(kb + v) * (Dm * 2) + chunk * 16) : 0);
-                cp_async16(dst + sw128(r, (chunk & 7) * 8), src, valid ? 16 : 0);
+                vv[j] = (i < kGroups && r < jlim) ? irow[r] : -1;
+            }
+#pragma unroll
+            for (int j = 0; j < kPer; ++j) {
+                const int i = warp + kProd * j;
+                if (i < kGroups) {
+                    const int r = rsub + kRowsPerPass * i;
+                    const int32_t v = vv[j];
+                    const bool valid = v >= 0 && v < kl;
+                    const char *src = kbase_ptr + (valid ? ((int64_t)(kb + v) * (Dm * 2) + chunk * 16) : 0);
+                    cp_async16(dst + sw128(r, (chunk & 7) * 8), src, valid ? 16 : 0);
+                }
             }
             asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&bars->kv_full[s]))
                          : "memory");
@@ -260,36 +277,43 @@ __global__ void __launch_bounds__(kMpThreads, 1)
         const long long st = clock64();
         while (!mbar_try_wait(&bars->drain, 0) && clock64() - st < kWaitCycles) {}
     } else {
-        // =============================== softmax group ===============================
-        const int h = threadIdx.x - 128;             // head in passes 1 and 2, slot in the sums
+        // =============================== softmax groups ===============================
+        // warps 4-7 take the slot columns 0-63 of every tile, warps 8-11 the columns 64-127;
+        // thread = head (lane quadrant warp % 4) in passes 1 and 2, then thread = slot for
+        // the column sums (threads 0-127 of the 256)
+        const int sw = warp - 4;                     // softmax warp 0..7
+        const int half = sw >> 2;                    // column half of the tile
         const int quad = warp & 3;
+        const int h = quad * 32 + lane;              // head
+        const int et = threadIdx.x - 128;            // 0..255: slot in the sums when < 128
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
         float *E = reinterpret_cast<float *>(smem + SP.e);
         const float inv_nm = 1.f / (float)A.Nm;
+        __shared__ float st_m[2][128], st_z[2][128];   // per column half: head max and sum
         uint32_t ph = 0, g = 0;
         bool ok = true;
         // rows of the range without a non-empty tile: p = 0
         for (int t = t0; t < t1; ++t) {
             if (P.tok_tiles[t]) continue;
-            for (int j = h; j < K; j += 128) A.p[(int64_t)t * K + j] = 0.f;
+            for (int j = et; j < K; j += 256) A.p[(int64_t)t * K + j] = 0.f;
         }
         float m = -INFINITY, z = 0.f, iz = 0.f;
         for (MpItem it = sc.next(); ok && it.pass >= 0; it = sc.next(), ++g) {
             const int b = g & 1;
             if (!wait_bar(&bars->mask_full[g % kMaskRing], (g / kMaskRing) & 1, &abort_flag, P.status)) { ok = false; break; }
-            const uint32_t *mw = mask_ring + (g % kMaskRing) * 4;
-            const uint32_t w0 = mw[0], w1 = mw[1], w2 = mw[2], w3 = mw[3];
+            const uint32_t *mw = mask_ring + (g % kMaskRing) * 4 + 2 * half;
+            const uint32_t w0 = mw[0], w1 = mw[1];   // valid-slot bits of this half's two chunks
             if (!wait_bar(&bars->s_full[b], (g >> 1) & 1, &abort_flag, P.status)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t sa = tm_s + b * 128 + lane_addr;
+            const uint32_t sa = tm_s + b * 128 + 64 * half + lane_addr;
             if (it.pass == 0) {
                 if (it.first) { m = -INFINITY; z = 0.f; }
 #pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < 2; ++c) {
                     float v[32];
                     tmem_ld32(sa + 32 * c, v);
                     tmem_wait_ld();
-                    const uint32_t bits = c == 0 ? w0 : (c == 1 ? w1 : (c == 2 ? w2 : w3));
+                    const uint32_t bits = c == 0 ? w0 : w1;
                     float cm = -INFINITY;
 #pragma unroll
                     for (int k = 0; k < 32; ++k)
@@ -304,20 +328,34 @@ __global__ void __launch_bounds__(kMpThreads, 1)
                         if ((bits >> k) & 1u) zs += __expf(A.scale * v[k] - m);
                     z += zs;
                 }
-                if (it.last) iz = z > 0.f ? 1.f / z : 0.f;
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars->s_empty[b]);
+                if (it.last) {
+                    // the head's max and sum: this half's, then combined with the other half's
+                    // (half 0 first) once every warp has written its own
+                    st_m[half][h] = m;
+                    st_z[half][h] = z;
+                    if (!group_sync(&bars->sm_sync, ph, &abort_flag, P.status)) { ok = false; break; }
+                    const float m0 = st_m[0][h], m1 = st_m[1][h];
+                    const float M = fmaxf(m0, m1);
+                    const float Z = (m0 == -INFINITY ? 0.f : st_z[0][h] * __expf(m0 - M)) +
+                                    (m1 == -INFINITY ? 0.f : st_z[1][h] * __expf(m1 - M));
+                    m = M;
+                    iz = Z > 0.f ? 1.f / Z : 0.f;
+                    // st_m / st_z are rewritten at the next row's pass-1 end, after that row's
+                    // pass-2 group syncs, which every warp reaches only after these reads
+                }
             } else {
-                // weights of head h into row h of the tile (heads past Nm are never summed);
-                // 16-byte stores: lanes h and h + 8 share banks, four wavefronts per store
-                float4 *erow = reinterpret_cast<float4 *>(E + h * kEStride);
+                // weights of head h into row h of the tile, this half's 64 columns (heads past
+                // Nm are never summed); 16-byte stores, four wavefronts each
+                float4 *erow = reinterpret_cast<float4 *>(E + h * kEStride + 64 * half);
 #pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < 2; ++c) {
                     float v[32];
                     tmem_ld32(sa + 32 * c, v);
                     tmem_wait_ld();
-                    const uint32_t bits = c == 0 ? w0 : (c == 1 ? w1 : (c == 2 ? w2 : w3));
+                    const uint32_t bits = c == 0 ? w0 : w1;
                     float e[32];
 #pragma unroll
                     for (int k = 0; k < 32; ++k)
@@ -330,27 +368,29 @@ __global__ void __launch_bounds__(kMpThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars->s_empty[b]);
                 if (!group_sync(&bars->sm_sync, ph, &abort_flag, P.status)) { ok = false; break; }
-                // slot h of the tile: its weights summed over the heads in a fixed order (eight
-                // interleaved partial sums, combined pairwise), so the loads overlap
-                float a8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                int hh = 0;
-                for (; hh + 8 <= A.Nm; hh += 8) {
+                if (et < 128) {
+                    // slot et of the tile: its weights summed over the heads in a fixed order
+                    // (eight interleaved partial sums, combined pairwise), so the loads overlap
+                    float a8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    int hh = 0;
+                    for (; hh + 8 <= A.Nm; hh += 8) {
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) a8[u] += E[(hh + u) * kEStride + h];
+                        for (int u = 0; u < 8; ++u) a8[u] += E[(hh + u) * kEStride + et];
+                    }
+#pragma unroll
+                    for (int u = 0; u < 7; ++u)               // the last Nm % 8 heads
+                        if (hh + u < A.Nm) a8[u] += E[(hh + u) * kEStride + et];
+                    const float acc = ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
+                    const int j = it.tile * 128 + et;
+                    if (j < K) A.p[(int64_t)it.t * K + j] = acc * inv_nm;
                 }
-#pragma unroll
-                for (int u = 0; u < 7; ++u)                   // the last Nm % 8 heads
-                    if (hh + u < A.Nm) a8[u] += E[(hh + u) * kEStride + h];
-                const float acc = ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
-                const int j = it.tile * 128 + h;
-                if (j < K) A.p[(int64_t)it.t * K + j] = acc * inv_nm;
                 if (!group_sync(&bars->sm_sync, ph, &abort_flag, P.status)) { ok = false; break; }
-                if (it.last) {
+                if (it.last && et < 128) {
                     // p = 0 on the row's empty tiles
                     const uint64_t all = P.tok_tiles[it.t];
                     for (int tl = 0; tl * 128 < K; ++tl) {
                         if ((all >> tl) & 1) continue;
-                        const int jz = tl * 128 + h;
+                        const int jz = tl * 128 + et;
                         if (jz < K) A.p[(int64_t)it.t * K + jz] = 0.f;
                     }
                 }
