@@ -21,7 +21,8 @@
 //                   records, dW, dq readback
 //
 // TMEM: S buffers [0, 4 N1P) (buffer b, half h at (2b + h) N1P), dq^T at 4 N1P, the per-slot
-// dW partials of half h at 5 N1P + h N1P. Shared memory: two K stages of 256 rows (two
+// dW partials of half h at 5 N1P + h N1P, and (rows of at most 4096 slots) the parked logits
+// of two tokens at 7 N1P + 32 (ordinal % 2) + 2 pair + h. Shared memory: two K stages of 256 rows (two
 // 128-row halves of two 64-column SW128 blocks), two q buffers, one dS tile [256 keys x 64
 // heads] (two halves), the producers' index rings.
 //
@@ -166,8 +167,10 @@ struct PSched {
 };
 
 // kMode: 1 = records with fp32 dI; 2 = deterministic (64-bit fixed-point dI, 16-byte records
-// at least)
-template <int N1P, int D, typename T, int kMode>
+// at least). kTP: the logits I of pass A are parked in TMEM (rows of at most 16 tile pairs,
+// two tokens in flight: 64 columns) instead of in softmax_out, saving a global store and load
+// per slot
+template <int N1P, int D, typename T, int kMode, bool kTP>
 __global__ void __launch_bounds__(kPThreads, 1)
     fused_pair_sm100(Params P, const __grid_constant__ CUtensorMap qmap) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -187,6 +190,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
     constexpr uint32_t kColDw = 5 * N1P;
     static_assert(N1P <= 64, "paired items take at most 64 heads");
     static_assert(kColDw + 2 * N1P <= kPTmemCols, "TMEM columns");
+    constexpr uint32_t kColPark = kColDw + 2 * N1P;   // parked I: [token ordinal % 2][32]
+    static_assert(!kTP || kColPark + 64 <= kPTmemCols, "TMEM columns (parked logits)");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t0 = P.meta[kMetaHeader + 2 * blockIdx.x];
@@ -449,7 +454,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 const int jn = nx.pair * 256 + h * 128 + lrow;
                 o.v[h] = jn < K ? P.idx[ro + jn] : -1;
                 o.p[h] = (nx.kind == 1 && jn < K) ? P.p[ro + jn] : 0.f;
-                o.I[h] = (o.haveI && jn < K) ? P.y[ro + jn] : 0.f;
+                o.I[h] = (!kTP && o.haveI && jn < K) ? P.y[ro + jn] : 0.f;
             }
         };
         PItem it = sc.next();
@@ -517,6 +522,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars->s_empty[sb]);
+                float park[2];
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const int32_t v = cur.v[h];
@@ -529,8 +535,15 @@ __global__ void __launch_bounds__(kPThreads, 1)
                         }
                         z_a += __expf(I - m_a);
                     }
+                    park[h] = valid ? I : -INFINITY;
                     const int j = it.pair * 256 + h * 128 + lrow;
-                    if (j < K) P.y[row_off + j] = valid ? I : -INFINITY;      // parked for pass B
+                    if (!kTP && j < K) P.y[row_off + j] = park[h];            // parked for pass B
+                }
+                if constexpr (kTP) {
+                    // parked for pass B in this thread's lane: columns 2 pair, 2 pair + 1 of
+                    // the token ordinal's half of the region
+                    tmem_st2(tmem + kColPark + (it.ord & 1) * 32 + 2 * it.pair + lane_addr, park[0], park[1]);
+                    tmem_wait_st();
                 }
                 if (it.last) {
                     float mw = m_a;
@@ -560,6 +573,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 }
                 float dI2[2], y2[2];
                 bool valid2[2];
+                float Ip[2] = {0.f, 0.f};
+                if constexpr (kTP) {
+                    tmem_ld2(tmem + kColPark + (it.ord & 1) * 32 + 2 * it.pair + lane_addr, Ip[0], Ip[1]);
+                    tmem_wait_ld();
+                }
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const int j = it.pair * 256 + h * 128 + lrow;
@@ -568,7 +586,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
                     dI2[h] = 0.f;
                     y2[h] = 0.f;
                     if (j < K) {
-                        const float I = cur.haveI ? cur.I[h] : P.y[row_off + j];
+                        const float I = kTP ? Ip[h] : (cur.haveI ? cur.I[h] : P.y[row_off + j]);
                         y2[h] = valid2[h] ? __expf(I - M_b) * iZ_b : 0.f;
                         dI2[h] = valid2[h] ? y2[h] - cur.p[h] : 0.f;
                     }
@@ -745,7 +763,10 @@ template <int N1P, int D, typename T>
 cudaError_t launch_pair_t(const Params &P, int workers, cudaStream_t s) {
     const PPlan sp = pair_plan<N1P>();
     if (sp.total > 226 * 1024) return cudaErrorInvalidConfiguration;
-    auto k = P.deterministic ? fused_pair_sm100<N1P, D, T, 2> : fused_pair_sm100<N1P, D, T, 1>;
+    // logits parked in TMEM for rows of at most 4096 slots (16 tile pairs)
+    auto k = P.K <= 4096
+                 ? (P.deterministic ? fused_pair_sm100<N1P, D, T, 2, true> : fused_pair_sm100<N1P, D, T, 1, true>)
+                 : (P.deterministic ? fused_pair_sm100<N1P, D, T, 2, false> : fused_pair_sm100<N1P, D, T, 1, false>);
     CUtensorMap qmap;
     cudaError_t e = encode_q_map<N1P, T>(P, &qmap);
     if (e != cudaSuccess) return e;

@@ -99,6 +99,20 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float *v) {
           "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15]))
         : "memory");
 }
+// 32 lanes x 32 bit, 2 consecutive columns per thread (taddr column even)
+__device__ __forceinline__ void tmem_ld2(uint32_t taddr, float &a, float &b) {
+    uint32_t r0, r1;
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];"
+                 : "=r"(r0), "=r"(r1)
+                 : "r"(taddr));
+    a = __uint_as_float(r0);
+    b = __uint_as_float(r1);
+}
+__device__ __forceinline__ void tmem_st2(uint32_t taddr, float a, float b) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1,%2};"
+                 ::"r"(taddr), "r"(__float_as_uint(a)), "r"(__float_as_uint(b))
+                 : "memory");
+}
 __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
