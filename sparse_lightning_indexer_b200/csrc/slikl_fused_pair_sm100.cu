@@ -21,8 +21,9 @@
 //                   records, dW, dq readback
 //
 // TMEM: S buffers [0, 4 N1P) (buffer b, half h at (2b + h) N1P), dq^T at 4 N1P, the per-slot
-// dW partials of half h at 5 N1P + h N1P, and (rows of at most 4096 slots) the parked logits
-// of two tokens at 7 N1P + 32 (ordinal % 2) + 2 pair + h. Shared memory: two K stages of 256 rows (two
+// dW partials at 5 N1P (both halves of a pair add into the same columns), and (rows of at
+// most 4096 slots) the parked logits of two tokens at 6 N1P + 32 (ordinal % 2) + 2 pair + h,
+// their slot indices 64 columns on. Shared memory: two K stages of 256 rows (two
 // 128-row halves of two 64-column SW128 blocks), two q buffers, one dS tile [256 keys x 64
 // heads] (two halves), the producers' index rings.
 //
@@ -189,9 +190,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
     constexpr uint32_t kColDq = 4 * N1P;
     constexpr uint32_t kColDw = 5 * N1P;
     static_assert(N1P <= 64, "paired items take at most 64 heads");
-    static_assert(kColDw + 2 * N1P <= kPTmemCols, "TMEM columns");
-    constexpr uint32_t kColPark = kColDw + 2 * N1P;   // parked I: [token ordinal % 2][32]
-    static_assert(!kTP || kColPark + 64 <= kPTmemCols, "TMEM columns (parked logits)");
+    static_assert(kColDw + N1P <= kPTmemCols, "TMEM columns");
+    // the dW partials of both halves of a pair share columns (one thread holds both slots);
+    // then the parked I [token ordinal % 2][32] and the parked slot indices, likewise
+    constexpr uint32_t kColPark = kColDw + N1P;
+    static_assert(!kTP || kColPark + 128 <= kPTmemCols, "TMEM columns (parked logits)");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t0 = P.meta[kMetaHeader + 2 * blockIdx.x];
@@ -452,7 +455,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int jn = nx.pair * 256 + h * 128 + lrow;
-                o.v[h] = jn < K ? P.idx[ro + jn] : -1;
+                // (pass-B slot indices come from the parked copy when parking)
+                o.v[h] = (!(kTP && nx.kind == 1) && jn < K) ? P.idx[ro + jn] : -1;
                 o.p[h] = (nx.kind == 1 && jn < K) ? P.p[ro + jn] : 0.f;
                 o.I[h] = (!kTP && o.haveI && jn < K) ? P.y[ro + jn] : 0.f;
             }
@@ -542,7 +546,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 if constexpr (kTP) {
                     // parked for pass B in this thread's lane: columns 2 pair, 2 pair + 1 of
                     // the token ordinal's half of the region
-                    tmem_st2(tmem + kColPark + (it.ord & 1) * 32 + 2 * it.pair + lane_addr, park[0], park[1]);
+                    const uint32_t pa = tmem + kColPark + (it.ord & 1) * 32 + 2 * it.pair + lane_addr;
+                    tmem_st2(pa, park[0], park[1]);
+                    tmem_st2(pa + 64, __int_as_float(cur.v[0]), __int_as_float(cur.v[1]));
                     tmem_wait_st();
                 }
                 if (it.last) {
@@ -574,14 +580,20 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 float dI2[2], y2[2];
                 bool valid2[2];
                 float Ip[2] = {0.f, 0.f};
+                int32_t vb[2] = {cur.v[0], cur.v[1]};
                 if constexpr (kTP) {
-                    tmem_ld2(tmem + kColPark + (it.ord & 1) * 32 + 2 * it.pair + lane_addr, Ip[0], Ip[1]);
+                    const uint32_t pa = tmem + kColPark + (it.ord & 1) * 32 + 2 * it.pair + lane_addr;
+                    float f0, f1;
+                    tmem_ld2(pa, Ip[0], Ip[1]);
+                    tmem_ld2(pa + 64, f0, f1);
                     tmem_wait_ld();
+                    vb[0] = __float_as_int(f0);
+                    vb[1] = __float_as_int(f1);
                 }
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const int j = it.pair * 256 + h * 128 + lrow;
-                    const int32_t v = cur.v[h];
+                    const int32_t v = vb[h];
                     valid2[h] = v >= 0 && v < kl;
                     dI2[h] = 0.f;
                     y2[h] = 0.f;
@@ -599,15 +611,16 @@ __global__ void __launch_bounds__(kPThreads, 1)
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const uint32_t sa = tm_s + (2 * sb + h) * N1P + lane_addr;
-                    const uint32_t dwa = tm_dw + h * N1P + lane_addr;
+                    const uint32_t dwa = tm_dw + lane_addr;
                     uint8_t *dsrow = ds_tile + h * 16384 + lrow * 128;
                     const float dI = dI2[h];
+                    const bool zacc = it.first && h == 0;      // the token's first partials
                     uint64_t smask = 0;
 #pragma unroll 1
                     for (int c = 0; c < N1P; c += 16) {
                         float sv[16], acc[16], wv[16];
                         tmem_ld16(sa + c, sv);
-                        if (!it.first) tmem_ld16(dwa + c, acc);
+                        if (!zacc) tmem_ld16(dwa + c, acc);
 #pragma unroll
                         for (int hh = 0; hh < 16; hh += 4) {
                             const float4 w4 = *reinterpret_cast<const float4 *>(ws + c + hh);
@@ -618,8 +631,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
 #pragma unroll
                         for (int hh = 0; hh < 16; hh += 2) {
                             const float s0 = sv[hh], s1 = sv[hh + 1];
-                            acc[hh] = fmaf(dI, fmaxf(s0, 0.f), it.first ? 0.f : acc[hh]);
-                            acc[hh + 1] = fmaf(dI, fmaxf(s1, 0.f), it.first ? 0.f : acc[hh + 1]);
+                            acc[hh] = fmaf(dI, fmaxf(s0, 0.f), zacc ? 0.f : acc[hh]);
+                            acc[hh + 1] = fmaf(dI, fmaxf(s1, 0.f), zacc ? 0.f : acc[hh + 1]);
                             pk[hh >> 1] = pack2<T>(s0 > 0.f ? dI * wv[hh] : 0.f, s1 > 0.f ? dI * wv[hh + 1] : 0.f);
                             m16 |= (s0 > 0.f ? 1u : 0u) << hh | (s1 > 0.f ? 2u : 0u) << hh;
                         }
@@ -632,6 +645,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
                         tmem_st16(dwa + c, acc);
                     }
                     smask2[h] = smask;
+                    if (h == 0) tmem_wait_st();                 // half 1 reads these columns
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -644,7 +658,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 for (int h = 0; h < 2; ++h) {
                     // record of this (token, key): the mask words are the same for every slot
                     // naming the key; dI is added, so repeated slots of a key sum their dI
-                    const int32_t v = cur.v[h];
+                    const int32_t v = vb[h];
                     if (valid2[h] && v < P.S2m) {
                         constexpr int rb = kRecBytes;
                         char *rp = static_cast<char *>(P.rec) + ((int64_t)it.t * P.S2m + v) * rb;
@@ -671,7 +685,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
                         const int jz = tl * 128 + et;
                         if (jz < K) P.y[row_off + jz] = 0.f;
                     }
-                    // dW: the two halves' per-slot partials, then a butterfly over the lanes
+                    // dW: the per-slot partials (both halves), then a butterfly over the lanes
                     // that leaves each lane kV / 32 heads, then the 4 warps in a fixed order
                     constexpr int kV = N1P < 32 ? 32 : N1P;
                     float vv[kV];
@@ -680,14 +694,6 @@ __global__ void __launch_bounds__(kPThreads, 1)
 #pragma unroll
                     for (int c = 0; c < N1P; c += 16) tmem_ld16(tm_dw + lane_addr + c, vv + c);
                     tmem_wait_ld();
-#pragma unroll
-                    for (int c = 0; c < N1P; c += 16) {
-                        float t16[16];
-                        tmem_ld16(tm_dw + N1P + lane_addr + c, t16);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int hh = 0; hh < 16; ++hh) vv[c + hh] += t16[hh];
-                    }
                     int len = kV;
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) {
