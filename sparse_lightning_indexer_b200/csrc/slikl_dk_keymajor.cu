@@ -15,6 +15,11 @@
 //
 // so a key row takes one fp32 add per run of work units instead of one per naming slot.
 //
+// Rows of fewer than 64 heads are packed into one stage: G = 64 / N1P query rows of a run
+// share the stage's 64-wide contraction (row g's heads are contraction indices g*N1P ..
+// g*N1P + N1P - 1), so a stage carries 64 contraction indices whatever N1. The MMAs of a
+// stage are issued row after row, as with one row per stage, so the sum order is unchanged.
+//
 // Work units are 32 query rows of one batch x one 256-key block pair (tables built by the
 // key-major metadata kernels). Each CTA takes a contiguous, cost-balanced range of units;
 // consecutive units on the same pair form a run that accumulates in one of two TMEM
@@ -25,13 +30,14 @@
 // to a per-CTA scratch that km_det_combine sums in CTA order.
 //
 // Warp roles (768 threads):
-//   warp 0      producer: per query row, TMA of q_t (128-byte swizzle, zero heads past N1)
-//               and a bulk copy of the pair's 256 records (lane 0); w_t through registers
+//   warp 0      producer: per stage, for each of its query rows a TMA of q_t (128-byte
+//               swizzle, zero heads past N1) and a bulk copy of the pair's 256 records
+//               (lane 0); w_t through registers
 //   warp 1      MMA issuer and TMEM owner
 //   warps 2-3   idle
 //   warps 4-7   flush: finished dK^T buffers from TMEM to the fp32 key rows
 //   warps 8-23  dS builders: two threads per key of the pair, each writing half of its
-//               128-byte K-major row (heads contiguous) with the 128-byte swizzle
+//               K-major row (contraction indices contiguous) with the 128-byte swizzle
 //
 // Every mbarrier wait is bounded; on expiry the CTA sets SLIKL_DEV_WAIT_TIMEOUT, the roles
 // stop, in-flight copies and MMAs are waited for (again bounded), TMEM is freed.
@@ -48,11 +54,16 @@ constexpr int kKmThreads = 768;
 constexpr int kKmStages = 4;             // most stages of any instance (barrier arrays)
 constexpr int kKmTmemCols = 512;         // two dK^T buffers of 256 columns
 
-// Per instance: the largest record (mask words of the heads, dI; 8-byte records of N1 <= 32
-// grow to 16 in deterministic mode), stages, and the dS tile of a stage ([256 keys x N1P
-// heads] as 64-head column blocks of 256 x 128 B)
+// Per instance: the query rows of a stage (G), its contraction width (G x N1P: 64, or 128
+// with 128 heads), the largest record (mask words of the heads, dI; 8-byte records of
+// N1 <= 32 grow to 16 in deterministic mode), stages, and the dS tile of a stage ([256 keys x
+// contraction] as 64-wide column blocks of 256 x 128 B)
+template <int N1P> __host__ __device__ constexpr int km_group() { return N1P < 64 ? 64 / N1P : 1; }
+template <int N1P> __host__ __device__ constexpr int km_kdim() { return km_group<N1P>() * N1P; }
 template <int N1P> __host__ __device__ constexpr int km_rec_bytes() { return N1P > 64 ? 32 : 16; }
-template <int N1P> __host__ __device__ constexpr int km_stages() { return N1P > 64 ? 2 : kKmStages; }
+template <int N1P> __host__ __device__ constexpr int km_stages() {
+    return N1P > 64 ? 2 : (N1P < 64 ? 3 : kKmStages);
+}
 template <int N1P> __host__ __device__ constexpr uint32_t km_ds_bytes() {
     return N1P > 64 ? 2u * 256u * 128u : 256u * 128u;
 }
@@ -74,16 +85,18 @@ __host__ __device__ constexpr uint32_t round_up(uint32_t x, uint32_t a) { return
 
 template <int N1P>
 __host__ __device__ constexpr KmPlan km_plan() {
-    // [stage][2 column blocks][N1P heads][128 B] | [stage][dS tile] |
-    // [stage][256 records] | [stage][N1P] | barriers
+    // [stage][2 column blocks][KD contraction rows][128 B] | [stage][dS tile] |
+    // [stage][G rows][256 records] | [stage][KD] | barriers
     constexpr uint32_t S = km_stages<N1P>(), RB = km_rec_bytes<N1P>(), DS = km_ds_bytes<N1P>();
+    constexpr uint32_t KD = km_kdim<N1P>(), G = km_group<N1P>();
+    constexpr uint32_t kQ = S * KD * 256u, kR = S * G * 256u * RB;
     return KmPlan{0u,
-                  S * N1P * 256u,
-                  S * N1P * 256u + S * DS,
-                  S * N1P * 256u + S * DS + S * 256u * RB,
-                  round_up(S * N1P * 256u + S * DS + S * 256u * RB + S * N1P * 4u, 8),
-                  round_up(S * N1P * 256u + S * DS + S * 256u * RB + S * N1P * 4u, 8) +
-                      (uint32_t)sizeof(KmBarriers) + 1024u};
+                  kQ,
+                  kQ + S * DS,
+                  kQ + S * DS + kR,
+                  round_up(kQ + S * DS + kR + S * KD * 4u, 8),
+                  round_up(kQ + S * DS + kR + S * KD * 4u, 8) + (uint32_t)sizeof(KmBarriers) +
+                      1024u};
 }
 
 struct KmItem {
@@ -148,6 +161,46 @@ struct KmIter {
     }
 };
 
+// The rows of one stage: up to G consecutive items of one run (a stage ends at its run's
+// last item), taken in the order of KmIter by every role alike.
+template <int G>
+struct KmGroup {
+    int t[G];        // query rows
+    int n;           // rows present, 1..G
+    int key0, kloc, nkeys;
+    bool first;      // starts a run
+    bool last;       // ends a run
+
+    __device__ bool next(KmIter &iter) {
+        n = 0;
+        bool open = true;
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+            KmItem it;
+            if (open && iter.next(it)) {
+                if (j == 0) {
+                    key0 = it.key0; kloc = it.kloc; nkeys = it.nkeys; first = it.first;
+                }
+                t[j] = it.t;
+                n = j + 1;
+                last = it.last;
+                open = !it.last;
+            } else {
+                open = false;
+            }
+        }
+        return n > 0;
+    }
+    // query row of contraction row block r (r < G)
+    __device__ int row(int r) const {
+        int v = t[0];
+#pragma unroll
+        for (int j = 1; j < G; ++j)
+            if (r == j) v = t[j];
+        return v;
+    }
+};
+
 template <int N1P, int D, typename T>
 __global__ void __launch_bounds__(kKmThreads, 1)
     dk_keymajor(Params P, const __grid_constant__ CUtensorMap qmap) {
@@ -155,13 +208,15 @@ __global__ void __launch_bounds__(kKmThreads, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     constexpr int RB = km_rec_bytes<N1P>();
+    constexpr int kG = km_group<N1P>();                          // query rows per stage
+    constexpr int KD = km_kdim<N1P>();                           // contraction width of a stage
     constexpr int kSt = km_stages<N1P>();
     constexpr uint32_t kDs = km_ds_bytes<N1P>();
     constexpr KmPlan SP = km_plan<N1P>();
     constexpr int kFmt = std::is_same<T, __nv_bfloat16>::value ? 1 : 0;
     constexpr uint32_t kIdesc = idesc_f16(kFmt, 128, 256, 1, 0);
     const int rb = P.rec_bytes;                                  // record bytes of this call
-    const uint32_t kTx = (D / 64) * N1P * 128 + 256 * rb;       // q boxes + records
+    const uint32_t kTxRow = (D / 64) * N1P * 128 + 256 * rb;    // q boxes + records of a row
     KmBarriers *bars = reinterpret_cast<KmBarriers *>(smem + SP.bar);
     __shared__ volatile int abort_flag;
     __shared__ uint32_t tmem_base;
@@ -185,9 +240,9 @@ __global__ void __launch_bounds__(kKmThreads, 1)
     }
     if (D == 64) {
         // the upper column block of every q stage stays zero (rows d >= 64 of q^T)
-        for (uint32_t i = threadIdx.x; i < kSt * N1P * 128 / 16; i += kKmThreads) {
-            const uint32_t st = i / (N1P * 8), r = i % (N1P * 8);
-            reinterpret_cast<uint4 *>(smem + SP.q + st * N1P * 256 + N1P * 128)[r] =
+        for (uint32_t i = threadIdx.x; i < kSt * KD * 128 / 16; i += kKmThreads) {
+            const uint32_t st = i / (KD * 8), r = i % (KD * 8);
+            reinterpret_cast<uint4 *>(smem + SP.q + st * KD * 256 + KD * 128)[r] =
                 make_uint4(0, 0, 0, 0);
         }
         fence_proxy_async();
@@ -204,49 +259,56 @@ __global__ void __launch_bounds__(kKmThreads, 1)
 
     KmIter iter;
     iter.init(P.units_c, u0, u1);
-    KmItem it;
+    KmGroup<kG> grp;
 
     if (warp == 0) {
         // =============================== producer ===============================
-        // w_t goes through registers (its rows need only 4-byte alignment), loaded one item
-        // ahead; q_t and the records by TMA / bulk copy, issued by lane 0
-        auto load_w = [&](int t, float *wv) {
+        // w of the stage's rows goes through registers (its rows need only 4-byte alignment),
+        // loaded one stage ahead; q_t and the records by TMA / bulk copy, issued by lane 0
+        auto load_w = [&](const KmGroup<kG> &g, float *wv) {
 #pragma unroll
-            for (int k = 0; k < (N1P + 31) / 32; ++k) {
-                const int h = lane + 32 * k;
-                wv[k] = h < P.N1 ? P.w[(int64_t)t * P.N1 + h] : 0.f;
+            for (int k = 0; k < KD / 32; ++k) {
+                const int c = lane + 32 * k;          // contraction index: row c / N1P, head c % N1P
+                const int r = c / N1P, h = c % N1P;
+                wv[k] = (r < g.n && h < P.N1) ? P.w[(int64_t)g.row(r) * P.N1 + h] : 0.f;
             }
         };
-        float wcur[(N1P + 31) / 32], wnxt[(N1P + 31) / 32];
+        float wcur[KD / 32], wnxt[KD / 32];
         uint32_t i = 0;
-        bool ok = true, have = iter.next(it);
-        if (have) load_w(it.t, wcur);
+        bool ok = true, have = grp.next(iter);
+        if (have) load_w(grp, wcur);
         while (have) {
-            KmItem nx;
-            const bool have_nx = iter.next(nx);
-            if (have_nx) load_w(nx.t, wnxt);
+            KmGroup<kG> nx;
+            const bool have_nx = nx.next(iter);
+            if (have_nx) load_w(nx, wnxt);
             const int s = i % kSt;
             if (!wait_bar(&bars->empty[s], ((i / kSt) & 1) ^ 1, &abort_flag, P.status)) { ok = false; break; }
-            float *wd = reinterpret_cast<float *>(smem + SP.w + s * N1P * 4);
+            float *wd = reinterpret_cast<float *>(smem + SP.w + s * KD * 4);
 #pragma unroll
-            for (int k = 0; k < (N1P + 31) / 32; ++k)
-                if (lane + 32 * k < N1P) wd[lane + 32 * k] = wcur[k];
+            for (int k = 0; k < KD / 32; ++k) wd[lane + 32 * k] = wcur[k];
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive_expect_tx(&bars->full[s], kTx);
-                const uint32_t qd = smem_u32(smem + SP.q + s * N1P * 256);
-                tma_load_3d(qd, &qmap, 0, 0, it.t, &bars->full[s]);
-                if (D == 128) tma_load_3d(qd + N1P * 128, &qmap, 64, 0, it.t, &bars->full[s]);
-                bulk_g2s(smem_u32(smem + SP.rec + s * 256 * RB),
-                         static_cast<const char *>(P.rec) + ((int64_t)it.t * P.S2m + it.kloc) * rb,
-                         256 * rb, &bars->full[s]);
+                mbar_arrive_expect_tx(&bars->full[s], kTxRow * (uint32_t)grp.n);
+                const uint32_t qd = smem_u32(smem + SP.q + s * KD * 256);
+#pragma unroll
+                for (int r = 0; r < kG; ++r) {
+                    if (r < grp.n) {
+                        const int t = grp.t[r];
+                        tma_load_3d(qd + r * N1P * 128, &qmap, 0, 0, t, &bars->full[s]);
+                        if (D == 128)
+                            tma_load_3d(qd + KD * 128 + r * N1P * 128, &qmap, 64, 0, t, &bars->full[s]);
+                        bulk_g2s(smem_u32(smem + SP.rec + (s * kG + r) * 256 * RB),
+                                 static_cast<const char *>(P.rec) + ((int64_t)t * P.S2m + grp.kloc) * rb,
+                                 256 * rb, &bars->full[s]);
+                    }
+                }
             }
             __syncwarp();
             ++i;
-            it = nx;
+            grp = nx;
             have = have_nx;
 #pragma unroll
-            for (int k = 0; k < (N1P + 31) / 32; ++k) wcur[k] = wnxt[k];
+            for (int k = 0; k < KD / 32; ++k) wcur[k] = wnxt[k];
         }
         if (!ok && lane == 0) {
             // wait (bounded) for the copies already issued before the CTA leaves
@@ -259,27 +321,31 @@ __global__ void __launch_bounds__(kKmThreads, 1)
     } else if (warp == 1) {
         // =============================== MMA issuer ===============================
         uint32_t i = 0, nrun = 0;
-        while (iter.next(it)) {
+        while (grp.next(iter)) {
             const int s = i % kSt;
             const int ab = nrun & 1;
             if (!wait_bar(&bars->dsr[s], (i / kSt) & 1, &abort_flag, P.status)) break;
-            if (it.first && !wait_bar(&bars->acce[ab], ((nrun >> 1) & 1) ^ 1, &abort_flag, P.status)) break;
+            if (grp.first && !wait_bar(&bars->acce[ab], ((nrun >> 1) & 1) ^ 1, &abort_flag, P.status)) break;
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t qa = smem_u32(smem + SP.q + s * N1P * 256);
+                const uint32_t qa = smem_u32(smem + SP.q + s * KD * 256);
                 const uint32_t da = smem_u32(smem + SP.ds + s * kDs);
+                const int nks = grp.n * (N1P / 16);   // 16-wide contraction steps of the rows present
 #pragma unroll
-                for (int ks = 0; ks < N1P / 16; ++ks) {
-                    const uint64_t a = sdesc(qa + ks * 2048, N1P * 128, 1024);   // q^T, MN-major
-                    // dS, K-major: 16 heads per step, 64-head column blocks of 256 rows
-                    const uint64_t b = sdesc(da + (ks >> 2) * (256 * 128) + (ks & 3) * 32, 16, 1024);
-                    umma_f16(tacc + ab * 256, a, b, kIdesc, (it.first && ks == 0) ? 0u : 1u);
+                for (int ks = 0; ks < KD / 16; ++ks) {
+                    if (ks < nks) {
+                        const uint64_t a = sdesc(qa + ks * 2048, KD * 128, 1024);   // q^T, MN-major
+                        // dS, K-major: 16 contraction indices per step, 64-wide column blocks
+                        // of 256 rows
+                        const uint64_t b = sdesc(da + (ks >> 2) * (256 * 128) + (ks & 3) * 32, 16, 1024);
+                        umma_f16(tacc + ab * 256, a, b, kIdesc, (grp.first && ks == 0) ? 0u : 1u);
+                    }
                 }
                 umma_commit(&bars->empty[s]);
-                if (it.last) umma_commit(&bars->accf[ab]);
+                if (grp.last) umma_commit(&bars->accf[ab]);
             }
             __syncwarp();
-            if (it.last) ++nrun;
+            if (grp.last) ++nrun;
             ++i;
         }
         if (lane == 0) umma_commit(&bars->drain);
@@ -301,32 +367,32 @@ __global__ void __launch_bounds__(kKmThreads, 1)
         const int head_key = u0 < u1 ? P.units_c[u0].y : -1;
         const int tail_key = u0 < u1 ? P.units_c[u1 - 1].y : -1;
         uint32_t nrun = 0;
-        while (iter.next(it)) {
-            if (!it.last) continue;
+        while (grp.next(iter)) {
+            if (!grp.last) continue;
             const int ab = nrun & 1;
             if (!wait_bar(&bars->accf[ab], (nrun >> 1) & 1, &abort_flag, P.status)) break;
             tc_fence_after();
             if (quad * 32 < D) {
-                float *dst = P.dk_acc + (int64_t)it.key0 * D;
-                if (cut_head && it.key0 == head_key)
+                float *dst = P.dk_acc + (int64_t)grp.key0 * D;
+                if (cut_head && grp.key0 == head_key)
                     dst = P.km_scratch + (int64_t)(2 * blockIdx.x) * 256 * D;
-                else if (cut_tail && it.key0 == tail_key)
+                else if (cut_tail && grp.key0 == tail_key)
                     dst = P.km_scratch + (int64_t)(2 * blockIdx.x + 1) * 256 * D;
                 dst += quad * 32 + lane;
 #pragma unroll 1
                 for (int c = 0; c < 256; c += 32) {
-                    if (c >= it.nkeys) break;
+                    if (c >= grp.nkeys) break;
                     float v[32];
                     tmem_ld32(tacc + ab * 256 + lane_addr + c, v);
                     tmem_wait_ld();
                     if (det) {
 #pragma unroll
                         for (int k = 0; k < 32; ++k)
-                            if (c + k < it.nkeys) dst[(int64_t)(c + k) * D] = v[k];
+                            if (c + k < grp.nkeys) dst[(int64_t)(c + k) * D] = v[k];
                     } else {
 #pragma unroll
                         for (int k = 0; k < 32; ++k)
-                            if (c + k < it.nkeys) red_add_f32(dst + (int64_t)(c + k) * D, v[k]);
+                            if (c + k < grp.nkeys) red_add_f32(dst + (int64_t)(c + k) * D, v[k]);
                     }
                 }
             }
@@ -337,48 +403,50 @@ __global__ void __launch_bounds__(kKmThreads, 1)
         }
     } else if (warp >= 8) {
         // =============================== dS builders ===============================
-        // two threads per key of the pair: half of its heads each (32, or 64 with 128 heads)
+        // two threads per key of the pair, each writing half of its K-major row: 32
+        // contraction indices (64 with 128 heads), i.e. two rows of 16 heads, one row of 32, or
+        // half the heads of one row of 64 or 128
         const int e = (threadIdx.x - 256) >> 1;   // key of the pair, 0..255
         const int half = threadIdx.x & 1;
-        constexpr int kChunks = N1P / 8;          // 16-byte chunks of 8 heads per row
-        constexpr int kPer = N1P > 64 ? 8 : (kChunks < 4 ? kChunks : 4);   // chunks per thread
-        const bool has_work = half * kPer < kChunks;
+        constexpr int kPer = KD / 16;             // 16-byte chunks (8 contraction indices) per thread
+        constexpr int kSpan = 8 * kPer;           // contraction indices per thread
+        constexpr int kRowsPer = kSpan >= N1P ? kSpan / N1P : 1;   // query rows per thread
+        constexpr int kChRow = kPer / kRowsPer;   // chunks per query row (at most 8: two mask words)
+        const int c0 = half * kPer;               // first chunk of this thread
+        const int g0 = (8 * c0) / N1P;            // its first query row of the stage
+        const int hb = (8 * c0) % N1P;            // and the first head within that row
         uint32_t i = 0;
-        while (iter.next(it)) {
+        while (grp.next(iter)) {
             const int s = i % kSt;
             if (!wait_bar(&bars->full[s], (i / kSt) & 1, &abort_flag, P.status)) break;
-            if (has_work) {
-                uint32_t m0, m1 = 0;              // mask bits of this thread's heads
-                float dI;
-                const uint8_t *rp = smem + SP.rec + s * 256 * RB + e * rb;
-                if (N1P > 64) {
-                    const uint4 r = *reinterpret_cast<const uint4 *>(rp);
-                    m0 = half ? r.z : r.x;
-                    m1 = half ? r.w : r.y;
-                } else if (N1P > 32) {
-                    const uint2 r = *reinterpret_cast<const uint2 *>(rp);
-                    m0 = half ? r.y : r.x;
-                } else {
-                    m0 = *reinterpret_cast<const uint32_t *>(rp);
-                }
-                const uint8_t *dp = rp + rec_di_offset(rb);
-                dI = P.deterministic ? di_from_fixed(*reinterpret_cast<const long long *>(dp))
-                                     : *reinterpret_cast<const float *>(dp);
-                const float *ws = reinterpret_cast<const float *>(smem + SP.w + s * N1P * 4) + 8 * kPer * half;
-                uint8_t *row = smem + SP.ds + s * kDs + e * 128;
+            const float *ws = reinterpret_cast<const float *>(smem + SP.w + s * KD * 4);
+            uint8_t *row = smem + SP.ds + s * kDs + e * 128;
 #pragma unroll
-                for (int cc = 0; cc < kPer; ++cc) {   // 8 heads = one 16-byte chunk
-                    const int c = half * kPer + cc;   // chunk of the row; column block c / 8
-                    const float4 wa = *reinterpret_cast<const float4 *>(ws + 8 * cc);
-                    const float4 wb = *reinterpret_cast<const float4 *>(ws + 8 * cc + 4);
-                    const uint32_t mb = ((cc < 4 ? m0 : m1) >> ((cc & 3) * 8)) & 0xFFu;
-                    const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-                    float d[8];
+            for (int rr = 0; rr < kRowsPer; ++rr) {
+                const int g = g0 + rr;
+                if (g < grp.n) {                  // the MMA reads the chunks of present rows only
+                    const uint8_t *rp = smem + SP.rec + (s * kG + g) * 256 * RB + e * rb;
+                    const uint32_t *mw = reinterpret_cast<const uint32_t *>(rp) + hb / 32;
+                    const uint32_t m0 = mw[0];    // mask bits of this thread's heads
+                    const uint32_t m1 = kChRow > 4 ? mw[1] : 0u;
+                    const uint8_t *dp = rp + rec_di_offset(rb);
+                    const float dI = P.deterministic
+                                         ? di_from_fixed(*reinterpret_cast<const long long *>(dp))
+                                         : *reinterpret_cast<const float *>(dp);
 #pragma unroll
-                    for (int h = 0; h < 8; ++h) d[h] = ((mb >> h) & 1u) ? dI * wv[h] : 0.f;
-                    const uint4 o = make_uint4(pack2<T>(d[0], d[1]), pack2<T>(d[2], d[3]),
-                                               pack2<T>(d[4], d[5]), pack2<T>(d[6], d[7]));
-                    *reinterpret_cast<uint4 *>(row + (c >> 3) * (256 * 128) + ((((c & 7) ^ e) & 7) << 4)) = o;
+                    for (int j = 0; j < kChRow; ++j) {   // 8 heads = one 16-byte chunk
+                        const int c = c0 + rr * kChRow + j;   // chunk of the K-major row; column block c / 8
+                        const float4 wa = *reinterpret_cast<const float4 *>(ws + 8 * c);
+                        const float4 wb = *reinterpret_cast<const float4 *>(ws + 8 * c + 4);
+                        const uint32_t mb = ((j < 4 ? m0 : m1) >> ((j & 3) * 8)) & 0xFFu;
+                        const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+                        float d[8];
+#pragma unroll
+                        for (int h = 0; h < 8; ++h) d[h] = ((mb >> h) & 1u) ? dI * wv[h] : 0.f;
+                        const uint4 o = make_uint4(pack2<T>(d[0], d[1]), pack2<T>(d[2], d[3]),
+                                                   pack2<T>(d[4], d[5]), pack2<T>(d[6], d[7]));
+                        *reinterpret_cast<uint4 *>(row + (c >> 3) * (256 * 128) + ((((c & 7) ^ e) & 7) << 4)) = o;
+                    }
                 }
             }
             fence_proxy_async();

@@ -393,14 +393,26 @@ def test_owner_only_producers_are_caught():
 # key-major dK kernel (sparse_lightning_indexer_b200/csrc/slikl_dk_keymajor.cu)
 # ---------------------------------------------------------------------------
 
-def km_items(runs):
-    """Items of one CTA: one per (query row, work unit); consecutive units on the same key
-    block pair form a run (first / last mark its ends). runs = list of run lengths."""
+def km_items(runs, group=1):
+    """Stages of one CTA. An item is one (query row, work unit); consecutive units on the same
+    key block pair form a run (first / last mark its ends). runs = list of run lengths. A stage
+    takes up to `group` consecutive items of one run (query rows of fewer than 64 heads share a
+    stage), ending at its run's last item, as KmGroup::next forms them."""
     items = []
     for r, n in enumerate(runs):
         for k in range(n):
             items.append(dict(run=r, first=k == 0, last=k == n - 1))
-    return items
+    stages, i = [], 0
+    while i < len(items):
+        rows = []
+        while len(rows) < group and i < len(items):
+            rows.append(items[i])
+            i += 1
+            if rows[-1]["last"]:
+                break
+        stages.append(dict(run=rows[0]["run"], first=rows[0]["first"], last=rows[-1]["last"],
+                           n=len(rows)))
+    return stages
 
 
 def km_build(items, stages=4, builders=16, flushers=4, wait_empty=True):
@@ -488,9 +500,9 @@ def km_build(items, stages=4, builders=16, flushers=4, wait_empty=True):
     return roles
 
 
-def km_run(runs, seed, **kw):
+def km_run(runs, seed, group=1, **kw):
     rnd = random.Random(seed)
-    roles = km_build(km_items(runs), **kw)
+    roles = km_build(km_items(runs, group), **kw)
     blocked = {}
     while roles:
         progressed = False
@@ -515,15 +527,32 @@ def km_run(runs, seed, **kw):
     return None
 
 
-@pytest.mark.parametrize("stages", [4, 2], ids=["4stages", "2stages_128heads"])
-def test_keymajor_protocol_finishes_and_is_safe(stages):
+@pytest.mark.parametrize("stages,group", [(4, 1), (2, 1), (3, 2), (3, 4)],
+                         ids=["64heads", "128heads", "32heads", "16heads"])
+def test_keymajor_protocol_finishes_and_is_safe(stages, group):
     rnd = random.Random(20261203)
-    cases = [[1], [1, 1, 1], [32], [1, 32, 1], [5, 5, 5, 5, 5]]
+    cases = [[1], [1, 1, 1], [32], [1, 32, 1], [5, 5, 5, 5, 5], [3, 4, 5, 6, 7]]
     cases += [[rnd.randint(1, 12) for _ in range(rnd.randint(1, 8))] for _ in range(150)]
     for i, runs in enumerate(cases):
         for seed in range(3):
-            assert km_run(runs, seed=1000 * i + seed, stages=stages) is None, \
+            assert km_run(runs, seed=1000 * i + seed, group=group, stages=stages) is None, \
                 f"deadlock with runs {runs}"
+
+
+@pytest.mark.parametrize("group", [1, 2, 4])
+def test_keymajor_stage_groups(group):
+    """Stages keep the item order, hold rows of one run only, at most `group` of them, and
+    are full except where a run ends."""
+    rnd = random.Random(group)
+    for _ in range(200):
+        runs = [rnd.randint(1, 13) for _ in range(rnd.randint(1, 9))]
+        st = km_items(runs, group)
+        assert sum(x["n"] for x in st) == sum(runs)
+        for r, n in enumerate(runs):
+            mine = [x for x in st if x["run"] == r]
+            assert [x["n"] for x in mine] == [group] * (n // group) + ([n % group] if n % group else [])
+            assert mine[0]["first"] and mine[-1]["last"]
+            assert not any(x["first"] for x in mine[1:]) and not any(x["last"] for x in mine[:-1])
 
 
 def test_keymajor_planted_mistake_is_caught():
