@@ -542,10 +542,11 @@ def main():
     t_roof = step_roofline_ms(stats, peaks, peak_tf) / 1e3
     t_roof_nom = step_roofline_ms(stats, peaks, NOMINAL_BF16_TFLOPS) / 1e3
     # our kernels per call: 3 work-split + fused + cast; the key-major path adds 2 metadata
-    # kernels and its dK kernel (and in deterministic mode the combine of cut runs); the sorted
+    # kernels, the w-scaled copy of q and its dK kernel (and in deterministic mode the combine
+    # of cut runs); the sorted
     # reduction replaces the cast by sort init, 3 per radix pass, row pointers and the
     # segmented reduce
-    launches_per_step = 5 + (3 if dk_path == "keymajor" else 0)
+    launches_per_step = 5 + (4 if dk_path == "keymajor" else 0)
     if args.deterministic and dk_path == "keymajor":
         launches_per_step += 1
     elif args.deterministic:

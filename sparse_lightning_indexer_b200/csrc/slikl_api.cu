@@ -91,6 +91,7 @@ slikl_status choose_dk_path(const slikl_problem *pr, Derived *dv, int32_t path) 
             k.rec_bytes = rb;
             k.nkpw = (int)((s2m / 256 + 31) / 32);
             k.units_max = (s2m / 256) * ((dv->T1 + 31) / 32 + pr->B);
+            k.qw_bytes = dv->T1 * pr->N1 * pr->D * 2;
             dv->km = k;
         }
     }
@@ -158,6 +159,7 @@ Params make_params(const slikl_problem *pr, const Derived &dv, const slikl_tenso
         P.unit_prefix = reinterpret_cast<int64_t *>(base + L.unit_prefix);
         P.km_range = reinterpret_cast<int32_t *>(base + L.km_range);
         P.km_scratch = reinterpret_cast<float *>(base + L.km_scratch);
+        P.km_qw = base + L.km_qw;
     }
     return P;
 }

@@ -66,6 +66,8 @@ struct Params {
     // next) are stored here instead of added, [kKmDetWorkers][2][256][D], and summed in CTA
     // order afterwards
     float *km_scratch;
+    // key-major path: q scaled by the head weights, w_th q_th, [T1][N1][D] in the input type
+    void *km_qw;
 };
 
 // Shape of the key-major dK path of one call (km = 0: scatter path).
@@ -73,13 +75,14 @@ struct KmShape {
     int km;
     int S2m, nkpw, rec_bytes;
     int64_t units_max, kbound;
+    int64_t qw_bytes;     // the w-scaled copy of q
 };
 
 // Byte offsets of the workspace regions; every region starts 256-byte aligned.
 struct WsLayout {
     size_t status, meta, tok_kbase, tok_klen, tok_cost, tok_tiles, cost_prefix;
     size_t dk_acc, partials, keys0, vals0, keys1, vals1, hist, row_ptr;
-    size_t tok_pairs, rec, units, units_c, unit_off, unit_prefix, km_range, km_scratch;
+    size_t tok_pairs, rec, units, units_c, unit_off, unit_prefix, km_range, km_scratch, km_qw;
     size_t total;
 };
 
@@ -119,6 +122,7 @@ inline WsLayout make_layout(int64_t T1, int64_t T2, int64_t K, int64_t D, int de
     L.unit_prefix = take(k ? sizeof(int64_t) * (size_t)(km.units_max + 1) : 0);
     L.km_range = take(k ? sizeof(int32_t) * (kMaxWorkers + 1) : 0);
     L.km_scratch = take(k && det ? sizeof(float) * (size_t)kKmDetWorkers * 2 * 256 * (size_t)D : 0);
+    L.km_qw = take(k ? (size_t)km.qw_bytes : 0);
     L.total = off;
     return L;
 }

@@ -7,11 +7,16 @@
 //   dK_j = sum over the rows t that name key j of  sum_h dS_t[h, j] q_t[h, :]
 //
 // The fused kernel leaves one record per named (t, j): dI_tj and the set of heads with
-// S_tjh > 0. dS_tjh = dI_tj * w_th * [S_tjh > 0] is rebuilt from it here (the same fp32
-// product and rounding as the fused kernel's dS), and for one 256-key block pair the
-// products of all rows that name a key of the pair accumulate in TMEM:
+// S_tjh > 0. With dS_tjh = dI_tj * w_th * [S_tjh > 0], the head weight moves to q:
 //
-//   dK^T [D x 256 keys] += q_t^T [D x heads] . dS_t [heads x 256 keys]   (M = 128, N = 256)
+//   dK_j = sum_t sum_h (w_th q_th) (dI_tj [S_tjh > 0])
+//
+// km_scale_q forms qw_th = w_th q_th once per call (fp32 product rounded to the input type),
+// the dS builders here form dI_tj [S_tjh > 0] (dI rounded to the input type) from the
+// records alone, and for one 256-key block pair the products of all rows that name a key of
+// the pair accumulate in TMEM:
+//
+//   dK^T [D x 256 keys] += qw_t^T [D x heads] . dS'_t [heads x 256 keys]   (M = 128, N = 256)
 //
 // so a key row takes one fp32 add per run of work units instead of one per naming slot.
 //
@@ -29,12 +34,18 @@
 // contribution to its key rows is stored, and the pieces of a run cut by the CTA ranges go
 // to a per-CTA scratch that km_det_combine sums in CTA order.
 //
+// A stage's data sit in three rings, each freed by its own consumer, so that the loads run
+// ahead of the tensor cores by as many stages as their ring holds:
+//   q ring      qw of the stage's rows (TMA), freed by the MMA (tcgen05.commit)
+//   record ring the rows' records (bulk copy), freed by the dS builders once read
+//   dS ring     the dS tile, written by the builders, freed by the MMA
+//
 // Warp roles (768 threads):
-//   warp 0      producer: per stage, for each of its query rows a TMA of q_t (128-byte
-//               swizzle, zero heads past N1) and a bulk copy of the pair's 256 records
-//               (lane 0); w_t through registers
+//   warp 0      q producer: for each row of a stage a TMA of qw_t (128-byte swizzle, zero
+//               heads past N1), issued by lane 0
 //   warp 1      MMA issuer and TMEM owner
-//   warps 2-3   idle
+//   warp 2      record producer: a bulk copy of each row's 256 records of the pair (lane 0)
+//   warp 3      idle
 //   warps 4-7   flush: finished dK^T buffers from TMEM to the fp32 key rows
 //   warps 8-23  dS builders: two threads per key of the pair, each writing half of its
 //               K-major row (contraction indices contiguous) with the 128-byte swizzle
@@ -51,52 +62,57 @@ namespace {
 using namespace sm100;
 
 constexpr int kKmThreads = 768;
-constexpr int kKmStages = 4;             // most stages of any instance (barrier arrays)
+constexpr int kKmMaxQ = 4, kKmMaxR = 8, kKmDs = 2;   // ring slots (barrier arrays)
 constexpr int kKmTmemCols = 512;         // two dK^T buffers of 256 columns
 
 // Per instance: the query rows of a stage (G), its contraction width (G x N1P: 64, or 128
 // with 128 heads), the largest record (mask words of the heads, dI; 8-byte records of
-// N1 <= 32 grow to 16 in deterministic mode), stages, and the dS tile of a stage ([256 keys x
-// contraction] as 64-wide column blocks of 256 x 128 B)
+// N1 <= 32 grow to 16 in deterministic mode), the slots of the q and record rings, and the
+// dS tile of a stage ([256 keys x contraction] as 64-wide column blocks of 256 x 128 B)
 template <int N1P> __host__ __device__ constexpr int km_group() { return N1P < 64 ? 64 / N1P : 1; }
 template <int N1P> __host__ __device__ constexpr int km_kdim() { return km_group<N1P>() * N1P; }
 template <int N1P> __host__ __device__ constexpr int km_rec_bytes() { return N1P > 64 ? 32 : 16; }
-template <int N1P> __host__ __device__ constexpr int km_stages() {
-    return N1P > 64 ? 2 : (N1P < 64 ? 3 : kKmStages);
+template <int N1P> __host__ __device__ constexpr int km_q_slots() { return N1P > 64 ? 2 : 4; }
+template <int N1P> __host__ __device__ constexpr int km_rec_slots() {
+    return N1P > 64 ? 3 : (N1P < 32 ? 5 : 8);
 }
 template <int N1P> __host__ __device__ constexpr uint32_t km_ds_bytes() {
     return N1P > 64 ? 2u * 256u * 128u : 256u * 128u;
 }
 
 struct KmBarriers {
-    uint64_t full[kKmStages];            // q, w, records landed (producer, TMA bytes)
-    uint64_t dsr[kKmStages];             // dS tile written (16 builder warps)
-    uint64_t empty[kKmStages];           // stage consumed by the MMA (tcgen05.commit)
+    uint64_t qfull[kKmMaxQ];             // q landed (TMA bytes)
+    uint64_t qempty[kKmMaxQ];            // q read by the MMA (tcgen05.commit)
+    uint64_t rfull[kKmMaxR];             // records landed (bulk-copy bytes)
+    uint64_t rempty[kKmMaxR];            // records read (16 builder warps)
+    uint64_t dsr[kKmDs];                 // dS tile written (16 builder warps)
+    uint64_t dsempty[kKmDs];             // dS tile read by the MMA (tcgen05.commit)
     uint64_t accf[2];                    // dK^T buffer complete (tcgen05.commit)
     uint64_t acce[2];                    // dK^T buffer flushed (4 flush warps)
     uint64_t drain;
 };
 
 struct KmPlan {
-    uint32_t q, ds, rec, w, bar, total;
+    uint32_t q, ds, rec, rec_slot, bar, total;
 };
 
 __host__ __device__ constexpr uint32_t round_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
 template <int N1P>
 __host__ __device__ constexpr KmPlan km_plan() {
-    // [stage][2 column blocks][KD contraction rows][128 B] | [stage][dS tile] |
-    // [stage][G rows][256 records] | [stage][KD] | barriers
-    constexpr uint32_t S = km_stages<N1P>(), RB = km_rec_bytes<N1P>(), DS = km_ds_bytes<N1P>();
+    // [q slot][2 column blocks][KD contraction rows][128 B] | [dS slot][dS tile] |
+    // [record slot][G rows][256 records] | barriers
+    constexpr uint32_t RB = km_rec_bytes<N1P>(), DS = km_ds_bytes<N1P>();
     constexpr uint32_t KD = km_kdim<N1P>(), G = km_group<N1P>();
-    constexpr uint32_t kQ = S * KD * 256u, kR = S * G * 256u * RB;
+    constexpr uint32_t kQ = km_q_slots<N1P>() * KD * 256u, kD = kKmDs * DS;
+    constexpr uint32_t kSlot = G * 256u * RB;
+    constexpr uint32_t kR = km_rec_slots<N1P>() * kSlot;
     return KmPlan{0u,
                   kQ,
-                  kQ + S * DS,
-                  kQ + S * DS + kR,
-                  round_up(kQ + S * DS + kR + S * KD * 4u, 8),
-                  round_up(kQ + S * DS + kR + S * KD * 4u, 8) + (uint32_t)sizeof(KmBarriers) +
-                      1024u};
+                  kQ + kD,
+                  kSlot,
+                  round_up(kQ + kD + kR, 8),
+                  round_up(kQ + kD + kR, 8) + (uint32_t)sizeof(KmBarriers) + 1024u};
 }
 
 struct KmItem {
@@ -210,13 +226,14 @@ __global__ void __launch_bounds__(kKmThreads, 1)
     constexpr int RB = km_rec_bytes<N1P>();
     constexpr int kG = km_group<N1P>();                          // query rows per stage
     constexpr int KD = km_kdim<N1P>();                           // contraction width of a stage
-    constexpr int kSt = km_stages<N1P>();
+    constexpr int kSQ = km_q_slots<N1P>();                      // q ring slots
+    constexpr int kSR = km_rec_slots<N1P>();                    // record ring slots
     constexpr uint32_t kDs = km_ds_bytes<N1P>();
     constexpr KmPlan SP = km_plan<N1P>();
     constexpr int kFmt = std::is_same<T, __nv_bfloat16>::value ? 1 : 0;
     constexpr uint32_t kIdesc = idesc_f16(kFmt, 128, 256, 1, 0);
     const int rb = P.rec_bytes;                                  // record bytes of this call
-    const uint32_t kTxRow = (D / 64) * N1P * 128 + 256 * rb;    // q boxes + records of a row
+    constexpr uint32_t kQRow = (D / 64) * N1P * 128;            // q boxes of a row
     KmBarriers *bars = reinterpret_cast<KmBarriers *>(smem + SP.bar);
     __shared__ volatile int abort_flag;
     __shared__ uint32_t tmem_base;
@@ -226,10 +243,17 @@ __global__ void __launch_bounds__(kKmThreads, 1)
 
     if (threadIdx.x == 0) {
         abort_flag = 0;
-        for (int s = 0; s < kSt; ++s) {
-            mbar_init(&bars->full[s], 1);
+        for (int s = 0; s < kSQ; ++s) {
+            mbar_init(&bars->qfull[s], 1);
+            mbar_init(&bars->qempty[s], 1);
+        }
+        for (int s = 0; s < kSR; ++s) {
+            mbar_init(&bars->rfull[s], 1);
+            mbar_init(&bars->rempty[s], 16);
+        }
+        for (int s = 0; s < kKmDs; ++s) {
             mbar_init(&bars->dsr[s], 16);
-            mbar_init(&bars->empty[s], 1);
+            mbar_init(&bars->dsempty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&bars->accf[b], 1);
@@ -239,8 +263,8 @@ __global__ void __launch_bounds__(kKmThreads, 1)
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (D == 64) {
-        // the upper column block of every q stage stays zero (rows d >= 64 of q^T)
-        for (uint32_t i = threadIdx.x; i < kSt * KD * 128 / 16; i += kKmThreads) {
+        // the upper column block of every q slot stays zero (rows d >= 64 of q^T)
+        for (uint32_t i = threadIdx.x; i < kSQ * KD * 128 / 16; i += kKmThreads) {
             const uint32_t st = i / (KD * 8), r = i % (KD * 8);
             reinterpret_cast<uint4 *>(smem + SP.q + st * KD * 256 + KD * 128)[r] =
                 make_uint4(0, 0, 0, 0);
@@ -262,59 +286,63 @@ __global__ void __launch_bounds__(kKmThreads, 1)
     KmGroup<kG> grp;
 
     if (warp == 0) {
-        // =============================== producer ===============================
-        // w of the stage's rows goes through registers (its rows need only 4-byte alignment),
-        // loaded one stage ahead; q_t and the records by TMA / bulk copy, issued by lane 0
-        auto load_w = [&](const KmGroup<kG> &g, float *wv) {
-#pragma unroll
-            for (int k = 0; k < KD / 32; ++k) {
-                const int c = lane + 32 * k;          // contraction index: row c / N1P, head c % N1P
-                const int r = c / N1P, h = c % N1P;
-                wv[k] = (r < g.n && h < P.N1) ? P.w[(int64_t)g.row(r) * P.N1 + h] : 0.f;
-            }
-        };
-        float wcur[KD / 32], wnxt[KD / 32];
+        // =============================== q producer ===============================
         uint32_t i = 0;
-        bool ok = true, have = grp.next(iter);
-        if (have) load_w(grp, wcur);
-        while (have) {
-            KmGroup<kG> nx;
-            const bool have_nx = nx.next(iter);
-            if (have_nx) load_w(nx, wnxt);
-            const int s = i % kSt;
-            if (!wait_bar(&bars->empty[s], ((i / kSt) & 1) ^ 1, &abort_flag, P.status)) { ok = false; break; }
-            float *wd = reinterpret_cast<float *>(smem + SP.w + s * KD * 4);
-#pragma unroll
-            for (int k = 0; k < KD / 32; ++k) wd[lane + 32 * k] = wcur[k];
-            __syncwarp();
+        bool ok = true;
+        while (grp.next(iter)) {
+            const int s = i % kSQ;
+            if (!wait_bar(&bars->qempty[s], ((i / kSQ) & 1) ^ 1, &abort_flag, P.status)) { ok = false; break; }
             if (lane == 0) {
-                mbar_arrive_expect_tx(&bars->full[s], kTxRow * (uint32_t)grp.n);
+                mbar_arrive_expect_tx(&bars->qfull[s], kQRow * (uint32_t)grp.n);
                 const uint32_t qd = smem_u32(smem + SP.q + s * KD * 256);
 #pragma unroll
                 for (int r = 0; r < kG; ++r) {
                     if (r < grp.n) {
-                        const int t = grp.t[r];
-                        tma_load_3d(qd + r * N1P * 128, &qmap, 0, 0, t, &bars->full[s]);
+                        tma_load_3d(qd + r * N1P * 128, &qmap, 0, 0, grp.t[r], &bars->qfull[s]);
                         if (D == 128)
-                            tma_load_3d(qd + KD * 128 + r * N1P * 128, &qmap, 64, 0, t, &bars->full[s]);
-                        bulk_g2s(smem_u32(smem + SP.rec + (s * kG + r) * 256 * RB),
-                                 static_cast<const char *>(P.rec) + ((int64_t)t * P.S2m + grp.kloc) * rb,
-                                 256 * rb, &bars->full[s]);
+                            tma_load_3d(qd + KD * 128 + r * N1P * 128, &qmap, 64, 0, grp.t[r],
+                                        &bars->qfull[s]);
                     }
                 }
             }
             __syncwarp();
             ++i;
-            grp = nx;
-            have = have_nx;
-#pragma unroll
-            for (int k = 0; k < KD / 32; ++k) wcur[k] = wnxt[k];
         }
         if (!ok && lane == 0) {
             // wait (bounded) for the copies already issued before the CTA leaves
-            for (uint32_t j = i > kSt ? i - kSt : 0; j < i; ++j) {
+            for (uint32_t j = i > kSQ ? i - kSQ : 0; j < i; ++j) {
                 const long long st = clock64();
-                while (!mbar_try_wait(&bars->full[j % kSt], (j / kSt) & 1) &&
+                while (!mbar_try_wait(&bars->qfull[j % kSQ], (j / kSQ) & 1) &&
+                       clock64() - st < kWaitCycles) {}
+            }
+        }
+    } else if (warp == 2) {
+        // ============================= record producer =============================
+        // the rows' records by bulk copy, issued by lane 0
+        uint32_t i = 0;
+        bool ok = true;
+        while (grp.next(iter)) {
+            const int s = i % kSR;
+            if (!wait_bar(&bars->rempty[s], ((i / kSR) & 1) ^ 1, &abort_flag, P.status)) { ok = false; break; }
+            if (lane == 0) {
+                uint8_t *slot = smem + SP.rec + s * SP.rec_slot;
+                mbar_arrive_expect_tx(&bars->rfull[s], 256u * (uint32_t)rb * (uint32_t)grp.n);
+#pragma unroll
+                for (int r = 0; r < kG; ++r) {
+                    if (r < grp.n)
+                        bulk_g2s(smem_u32(slot + r * 256 * RB),
+                                 static_cast<const char *>(P.rec) +
+                                     ((int64_t)grp.t[r] * P.S2m + grp.kloc) * rb,
+                                 256 * rb, &bars->rfull[s]);
+                }
+            }
+            __syncwarp();
+            ++i;
+        }
+        if (!ok && lane == 0) {
+            for (uint32_t j = i > kSR ? i - kSR : 0; j < i; ++j) {
+                const long long st = clock64();
+                while (!mbar_try_wait(&bars->rfull[j % kSR], (j / kSR) & 1) &&
                        clock64() - st < kWaitCycles) {}
             }
         }
@@ -322,14 +350,15 @@ __global__ void __launch_bounds__(kKmThreads, 1)
         // =============================== MMA issuer ===============================
         uint32_t i = 0, nrun = 0;
         while (grp.next(iter)) {
-            const int s = i % kSt;
+            const int sq = i % kSQ, sd = i % kKmDs;
             const int ab = nrun & 1;
-            if (!wait_bar(&bars->dsr[s], (i / kSt) & 1, &abort_flag, P.status)) break;
+            if (!wait_bar(&bars->qfull[sq], (i / kSQ) & 1, &abort_flag, P.status)) break;
+            if (!wait_bar(&bars->dsr[sd], (i / kKmDs) & 1, &abort_flag, P.status)) break;
             if (grp.first && !wait_bar(&bars->acce[ab], ((nrun >> 1) & 1) ^ 1, &abort_flag, P.status)) break;
             tc_fence_after();
             if (lane == 0) {
-                const uint32_t qa = smem_u32(smem + SP.q + s * KD * 256);
-                const uint32_t da = smem_u32(smem + SP.ds + s * kDs);
+                const uint32_t qa = smem_u32(smem + SP.q + sq * KD * 256);
+                const uint32_t da = smem_u32(smem + SP.ds + sd * kDs);
                 const int nks = grp.n * (N1P / 16);   // 16-wide contraction steps of the rows present
 #pragma unroll
                 for (int ks = 0; ks < KD / 16; ++ks) {
@@ -341,7 +370,8 @@ __global__ void __launch_bounds__(kKmThreads, 1)
                         umma_f16(tacc + ab * 256, a, b, kIdesc, (grp.first && ks == 0) ? 0u : 1u);
                     }
                 }
-                umma_commit(&bars->empty[s]);
+                umma_commit(&bars->qempty[sq]);
+                umma_commit(&bars->dsempty[sd]);
                 if (grp.last) umma_commit(&bars->accf[ab]);
             }
             __syncwarp();
@@ -415,17 +445,23 @@ __global__ void __launch_bounds__(kKmThreads, 1)
         const int c0 = half * kPer;               // first chunk of this thread
         const int g0 = (8 * c0) / N1P;            // its first query row of the stage
         const int hb = (8 * c0) % N1P;            // and the first head within that row
+        // chunks held in registers until the dS slot is free, so that the record slot is
+        // released early; with 128 heads (8 chunks a thread) the dS slot is awaited first and
+        // the chunks are stored as they are formed
+        constexpr bool kHold = kPer <= 4;
         uint32_t i = 0;
         while (grp.next(iter)) {
-            const int s = i % kSt;
-            if (!wait_bar(&bars->full[s], (i / kSt) & 1, &abort_flag, P.status)) break;
-            const float *ws = reinterpret_cast<const float *>(smem + SP.w + s * KD * 4);
-            uint8_t *row = smem + SP.ds + s * kDs + e * 128;
+            const int sr = i % kSR, sd = i % kKmDs;
+            if (!wait_bar(&bars->rfull[sr], (i / kSR) & 1, &abort_flag, P.status)) break;
+            if (!kHold && !wait_bar(&bars->dsempty[sd], ((i / kKmDs) & 1) ^ 1, &abort_flag, P.status)) break;
+            const uint8_t *slot = smem + SP.rec + sr * SP.rec_slot;
+            uint8_t *row = smem + SP.ds + sd * kDs + e * 128;
+            uint4 o[kRowsPer][kChRow];            // this thread's chunks, packed
 #pragma unroll
             for (int rr = 0; rr < kRowsPer; ++rr) {
                 const int g = g0 + rr;
                 if (g < grp.n) {                  // the MMA reads the chunks of present rows only
-                    const uint8_t *rp = smem + SP.rec + (s * kG + g) * 256 * RB + e * rb;
+                    const uint8_t *rp = slot + g * 256 * RB + e * rb;
                     const uint32_t *mw = reinterpret_cast<const uint32_t *>(rp) + hb / 32;
                     const uint32_t m0 = mw[0];    // mask bits of this thread's heads
                     const uint32_t m1 = kChRow > 4 ? mw[1] : 0u;
@@ -433,25 +469,43 @@ __global__ void __launch_bounds__(kKmThreads, 1)
                     const float dI = P.deterministic
                                          ? di_from_fixed(*reinterpret_cast<const long long *>(dp))
                                          : *reinterpret_cast<const float *>(dp);
+                    const uint32_t hh = pack2<T>(dI, dI);   // dI rounded to T, in both halves
 #pragma unroll
                     for (int j = 0; j < kChRow; ++j) {   // 8 heads = one 16-byte chunk
-                        const int c = c0 + rr * kChRow + j;   // chunk of the K-major row; column block c / 8
-                        const float4 wa = *reinterpret_cast<const float4 *>(ws + 8 * c);
-                        const float4 wb = *reinterpret_cast<const float4 *>(ws + 8 * c + 4);
+                        const int c = c0 + rr * kChRow + j;
                         const uint32_t mb = ((j < 4 ? m0 : m1) >> ((j & 3) * 8)) & 0xFFu;
-                        const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-                        float d[8];
+                        uint32_t wd[4];                  // heads 2k, 2k + 1: dI where S > 0, else +0
 #pragma unroll
-                        for (int h = 0; h < 8; ++h) d[h] = ((mb >> h) & 1u) ? dI * wv[h] : 0.f;
-                        const uint4 o = make_uint4(pack2<T>(d[0], d[1]), pack2<T>(d[2], d[3]),
-                                                   pack2<T>(d[4], d[5]), pack2<T>(d[6], d[7]));
-                        *reinterpret_cast<uint4 *>(row + (c >> 3) * (256 * 128) + ((((c & 7) ^ e) & 7) << 4)) = o;
+                        for (int k = 0; k < 4; ++k) {
+                            const uint32_t lo = 0u - ((mb >> (2 * k)) & 1u);
+                            const uint32_t hi = 0u - ((mb >> (2 * k + 1)) & 1u);
+                            wd[k] = hh & ((lo & 0xFFFFu) | (hi & 0xFFFF0000u));
+                        }
+                        const uint4 v = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+                        if (kHold)
+                            o[rr][j] = v;
+                        else   // chunk of the K-major row; column block c / 8
+                            *reinterpret_cast<uint4 *>(row + (c >> 3) * (256 * 128) + ((((c & 7) ^ e) & 7) << 4)) = v;
+                    }
+                }
+            }
+            // the records of this slot are read (their values are in registers)
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->rempty[sr]);
+            if (kHold && !wait_bar(&bars->dsempty[sd], ((i / kKmDs) & 1) ^ 1, &abort_flag, P.status)) break;
+#pragma unroll
+            for (int rr = 0; rr < kRowsPer; ++rr) {
+                if (kHold && g0 + rr < grp.n) {
+#pragma unroll
+                    for (int j = 0; j < kChRow; ++j) {
+                        const int c = c0 + rr * kChRow + j;   // chunk of the K-major row; column block c / 8
+                        *reinterpret_cast<uint4 *>(row + (c >> 3) * (256 * 128) + ((((c & 7) ^ e) & 7) << 4)) = o[rr][j];
                     }
                 }
             }
             fence_proxy_async();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->dsr[s]);
+            if (lane == 0) mbar_arrive(&bars->dsr[sd]);
             ++i;
         }
     }
@@ -502,12 +556,42 @@ __global__ void km_det_combine(Params P, int workers) {
     }
 }
 
+// qw = w . q per (row, head), the fp32 product rounded to T (round to nearest even); 8
+// elements per thread (q rows are 16-byte aligned, D a multiple of 8).
+template <typename T>
+__global__ void km_scale_q(Params P) {
+    const int64_t per_row = P.D / 8;
+    const int64_t n = (int64_t)P.T1 * P.N1 * per_row;
+    const uint4 *src = static_cast<const uint4 *>(P.q);
+    uint4 *dst = static_cast<uint4 *>(P.km_qw);
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const float wv = P.w[i / per_row];               // row index t * N1 + h
+        const uint4 v = src[i];
+        const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+        uint32_t out[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 f = unpack2<T>(in[k]);
+            out[k] = pack2<T>(wv * f.x, wv * f.y);
+        }
+        dst[i] = make_uint4(out[0], out[1], out[2], out[3]);
+    }
+}
+
 template <int N1P, int D, typename T>
 cudaError_t launch_km_t(const Params &P, int workers, cudaStream_t s) {
     constexpr KmPlan sp = km_plan<N1P>();
     static_assert(sp.total <= 227 * 1024, "key-major kernel shared memory");
+    static_assert(km_q_slots<N1P>() <= kKmMaxQ && km_rec_slots<N1P>() <= kKmMaxR, "ring slots");
+    km_scale_q<T><<<8 * 148, 256, 0, s>>>(P);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    // the MMA's A operand is qw, laid out as q
+    Params Pw = P;
+    Pw.q = P.km_qw;
     CUtensorMap qmap;
-    cudaError_t e = encode_q_map<N1P, T>(P, &qmap);
+    e = encode_q_map<N1P, T>(Pw, &qmap);
     if (e != cudaSuccess) return e;
     auto k = dk_keymajor<N1P, D, T>;
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp.total);

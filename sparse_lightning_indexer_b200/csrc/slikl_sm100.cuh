@@ -207,6 +207,20 @@ __device__ __forceinline__ uint32_t pack2<__half>(float a, float b) {
     return *reinterpret_cast<const uint32_t *>(&v);
 }
 
+// The inverse: two packed 16-bit values (low, high) as floats (exact).
+template <typename T>
+__device__ __forceinline__ float2 unpack2(uint32_t u);
+template <>
+__device__ __forceinline__ float2 unpack2<__nv_bfloat16>(uint32_t u) {
+    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+}
+template <>
+__device__ __forceinline__ float2 unpack2<__half>(uint32_t u) {
+    __half2 v;
+    *reinterpret_cast<uint32_t *>(&v) = u;
+    return __half22float2(v);
+}
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point.
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                    const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,

@@ -17,9 +17,10 @@ A negative test keeps the model honest: the producer variant in which each warp 
 stage only at the items it owns is caught.
 
 The key-major dK kernel (sparse_lightning_indexer_b200/csrc/slikl_dk_keymajor.cu) is modelled
-the same way: its producer, 16 dS-builder warps, MMA issuer and 4 flush warps over runs of work
-units, with checks on stage reuse (q, w, records and the dS tile) and on the two TMEM dK
-buffers (a run accumulates only into its own buffer, which is not reused before its flush).
+the same way: its two producers (w-scaled q; records), 16 dS-builder warps, MMA issuer and 4
+flush warps over runs of work units, with checks on the reuse of each ring's slots (q, records,
+dS tiles) and on the two TMEM dK buffers (a run accumulates only into its own buffer, which
+is not reused before its flush).
 """
 
 import itertools
@@ -415,19 +416,33 @@ def km_items(runs, group=1):
     return stages
 
 
-def km_build(items, stages=4, builders=16, flushers=4, wait_empty=True):
-    """Roles of the key-major kernel. wait_empty=False is a planted mistake (the producer
-    fills a stage without waiting for the MMA to release it)."""
+def km_build(items, sq=4, sr=5, sd=2, hold=True, builders=16, flushers=4, skip=None):
+    """Roles of the key-major kernel over its three rings: w-scaled q (sq slots, loaded by the
+    q producer, released by the MMA), records (sr slots, loaded by the record producer,
+    released by the builders once read) and dS tiles (sd slots, written by the builders,
+    released by the MMA). hold: the builders release the record slot before they wait for the
+    dS slot (else, with 128 heads, they wait for the dS slot first). skip names a planted
+    mistake: the wait that role leaves out ("qempty": q producer, "rempty": record producer,
+    "dsempty": builders)."""
     bars = {}
-    for s in range(stages):
-        bars[f"full{s}"] = Bar(1)
+    for s in range(sq):
+        bars[f"qfull{s}"] = Bar(1)
+        bars[f"qempty{s}"] = Bar(1)
+    for s in range(sr):
+        bars[f"rfull{s}"] = Bar(1)
+        bars[f"rempty{s}"] = Bar(builders)
+    for s in range(sd):
         bars[f"dsr{s}"] = Bar(builders)
-        bars[f"empty{s}"] = Bar(1)
+        bars[f"dsempty{s}"] = Bar(1)
     for b in range(2):
         bars[f"accf{b}"] = Bar(1)
         bars[f"acce{b}"] = Bar(flushers)
     serial = itertools.count()
-    st = dict(stage_free=[0] * stages, ds_fill=[[0] * stages for _ in range(builders)],
+    # q_in[s] / rec_in[s] / ds_in[w][s]: the group whose data a slot holds; q_done[s],
+    # rec_read[w][s], ds_done[s]: uses of a slot finished by its consumer(s)
+    st = dict(q_in=[None] * sq, q_done=[0] * sq, rec_in=[None] * sr,
+              rec_read=[[0] * sr for _ in range(builders)],
+              ds_in=[[None] * sd for _ in range(builders)], ds_done=[0] * sd,
               acc_run=[None, None], acc_flushed=[[0, 0] for _ in range(flushers)])
 
     def wait(name, parity):
@@ -435,35 +450,58 @@ def km_build(items, stages=4, builders=16, flushers=4, wait_empty=True):
         while not bars[name].ready(parity):
             yield ("wait", name, token)
 
-    def producer():
+    def q_producer():
         for i, _ in enumerate(items):
-            s = i % stages
-            if wait_empty:
-                yield from wait(f"empty{s}", ((i // stages) & 1) ^ 1)
-            # q, w and records of item i land in stage s
-            if st["stage_free"][s] < i // stages:
-                raise Violation(f"producer overwrote stage {s} (item {i}) still in use")
-            bars[f"full{s}"].arrive()
+            s = i % sq
+            if skip != "qempty":
+                yield from wait(f"qempty{s}", ((i // sq) & 1) ^ 1)
+            if st["q_done"][s] < i // sq:
+                raise Violation(f"q producer overwrote q slot {s} (group {i}) still in use")
+            st["q_in"][s] = i
+            bars[f"qfull{s}"].arrive()
+            yield ("step",)
+
+    def rec_producer():
+        for i, _ in enumerate(items):
+            s = i % sr
+            if skip != "rempty":
+                yield from wait(f"rempty{s}", ((i // sr) & 1) ^ 1)
+            if min(w[s] for w in st["rec_read"]) < i // sr:
+                raise Violation(f"record producer overwrote records slot {s} (group {i}) "
+                                "not yet read")
+            st["rec_in"][s] = i
+            bars[f"rfull{s}"].arrive()
             yield ("step",)
 
     def builder(wb):
         for i, _ in enumerate(items):
-            s = i % stages
-            yield from wait(f"full{s}", (i // stages) & 1)
-            # the dS tile of stage s is rewritten: the MMA must be done with item i - stages
-            if st["stage_free"][s] < i // stages:
-                raise Violation(f"builder {wb} overwrote dS of stage {s} (item {i}) still in use")
-            st["ds_fill"][wb][s] += 1
-            bars[f"dsr{s}"].arrive()
+            r, d = i % sr, i % sd
+            yield from wait(f"rfull{r}", (i // sr) & 1)
+            if not hold and skip != "dsempty":
+                yield from wait(f"dsempty{d}", ((i // sd) & 1) ^ 1)
+            if st["rec_in"][r] != i:
+                raise Violation(f"builder {wb} read records slot {r} not holding group {i}")
+            st["rec_read"][wb][r] += 1
+            bars[f"rempty{r}"].arrive()
+            yield ("step",)
+            if hold and skip != "dsempty":
+                yield from wait(f"dsempty{d}", ((i // sd) & 1) ^ 1)
+            if st["ds_done"][d] < i // sd:
+                raise Violation(f"builder {wb} overwrote dS slot {d} (group {i}) still in use")
+            st["ds_in"][wb][d] = i
+            bars[f"dsr{d}"].arrive()
             yield ("step",)
 
     def mma():
         nrun = 0
         for i, it in enumerate(items):
-            s, ab = i % stages, nrun & 1
-            yield from wait(f"dsr{s}", (i // stages) & 1)
-            if min(w[s] for w in st["ds_fill"]) != i // stages + 1:
-                raise Violation(f"MMA read dS of stage {s} not holding item {i}")
+            q, d, ab = i % sq, i % sd, nrun & 1
+            yield from wait(f"qfull{q}", (i // sq) & 1)
+            yield from wait(f"dsr{d}", (i // sd) & 1)
+            if st["q_in"][q] != i:
+                raise Violation(f"MMA read q slot {q} not holding group {i}")
+            if any(w[d] != i for w in st["ds_in"]):
+                raise Violation(f"MMA read dS slot {d} not holding group {i}")
             if it["first"]:
                 yield from wait(f"acce{ab}", ((nrun >> 1) & 1) ^ 1)
                 if min(w[ab] for w in st["acc_flushed"]) < nrun >> 1:
@@ -471,8 +509,10 @@ def km_build(items, stages=4, builders=16, flushers=4, wait_empty=True):
                 st["acc_run"][ab] = it["run"]
             elif st["acc_run"][ab] != it["run"]:
                 raise Violation(f"run {it['run']} accumulates into buffer {ab} of another run")
-            st["stage_free"][s] += 1
-            bars[f"empty{s}"].arrive()
+            st["q_done"][q] += 1
+            st["ds_done"][d] += 1
+            bars[f"qempty{q}"].arrive()
+            bars[f"dsempty{d}"].arrive()
             if it["last"]:
                 bars[f"accf{ab}"].arrive()
                 nrun += 1
@@ -492,7 +532,7 @@ def km_build(items, stages=4, builders=16, flushers=4, wait_empty=True):
             nrun += 1
             yield ("step",)
 
-    roles = {"producer": producer(), "mma": mma()}
+    roles = {"q_producer": q_producer(), "rec_producer": rec_producer(), "mma": mma()}
     for w in range(builders):
         roles[f"builder{w}"] = builder(w)
     for w in range(flushers):
@@ -527,16 +567,22 @@ def km_run(runs, seed, group=1, **kw):
     return None
 
 
-@pytest.mark.parametrize("stages,group", [(4, 1), (2, 1), (3, 2), (3, 4)],
-                         ids=["64heads", "128heads", "32heads", "16heads"])
-def test_keymajor_protocol_finishes_and_is_safe(stages, group):
+# (q slots, record slots, dS slots, query rows per stage, chunks held across the dS wait) of
+# the kernel's instances
+KM_SHAPES = {"16heads": (4, 5, 2, 4, True), "32heads": (4, 8, 2, 2, True),
+             "64heads": (4, 8, 2, 1, True), "128heads": (2, 3, 2, 1, False)}
+
+
+@pytest.mark.parametrize("shape", list(KM_SHAPES))
+def test_keymajor_protocol_finishes_and_is_safe(shape):
+    sq, sr, sd, group, hold = KM_SHAPES[shape]
     rnd = random.Random(20261203)
     cases = [[1], [1, 1, 1], [32], [1, 32, 1], [5, 5, 5, 5, 5], [3, 4, 5, 6, 7]]
     cases += [[rnd.randint(1, 12) for _ in range(rnd.randint(1, 8))] for _ in range(150)]
     for i, runs in enumerate(cases):
         for seed in range(3):
-            assert km_run(runs, seed=1000 * i + seed, group=group, stages=stages) is None, \
-                f"deadlock with runs {runs}"
+            assert km_run(runs, seed=1000 * i + seed, group=group, sq=sq, sr=sr, sd=sd,
+                          hold=hold) is None, f"deadlock with runs {runs}"
 
 
 @pytest.mark.parametrize("group", [1, 2, 4])
@@ -555,13 +601,15 @@ def test_keymajor_stage_groups(group):
             assert not any(x["first"] for x in mine[1:]) and not any(x["last"] for x in mine[:-1])
 
 
-def test_keymajor_planted_mistake_is_caught():
+@pytest.mark.parametrize("hold", [True, False])
+@pytest.mark.parametrize("skip", ["qempty", "rempty", "dsempty"])
+def test_keymajor_planted_mistake_is_caught(skip, hold):
     rnd = random.Random(11)
     caught = 0
     for i in range(40):
         runs = [rnd.randint(1, 12) for _ in range(rnd.randint(2, 8))]
         try:
-            if km_run(runs, seed=i, wait_empty=False) is not None:
+            if km_run(runs, seed=i, skip=skip, sq=2, sr=2, sd=2, hold=hold) is not None:
                 caught += 1
         except Violation:
             caught += 1
