@@ -143,7 +143,10 @@ SLIKL_API slikl_status slikl_grad(const slikl_problem *problem, const slikl_tens
                         void *workspace, size_t workspace_bytes, void *stream);
 
 /*
- * dK paths (slikl_options.dk_path). Both give the same dK up to the order of fp32 additions.
+ * dK paths (slikl_options.dk_path). Both give dK to within the input type's rounding: the
+ * scatter path multiplies q by dS = dI w [S > 0] rounded to the input type, the key-major path
+ * multiplies w q rounded to the input type by dI [S > 0] rounded to it; the fp32 additions run
+ * in different orders.
  *   SLIKL_DK_SCATTER   every named slot adds its dK row into an fp32 accumulator with
  *                      atomic adds (the page's default), or, deterministic = 1, stores it for
  *                      a sort by key and a fixed-order reduction;
@@ -153,7 +156,7 @@ SLIKL_API slikl_status slikl_grad(const slikl_problem *problem, const slikl_tens
  *                      Needs a key-range bound (BSND: S2; TND: problem->S2 > 0) of at most
  *                      16384 keys; its workspace holds T1 x roundup(S2, 256) records of 8
  *                      (N1 <= 32), 16 (N1 <= 64; also N1 <= 32 with deterministic = 1) or 32
- *                      bytes. With deterministic = 1 repeated slots of a key sum their dI as
+ *                      bytes, and the w-scaled copy of q (T1 x N1 x D of the input type). With deterministic = 1 repeated slots of a key sum their dI as
  *                      64-bit fixed-point integers and every key row is summed in a fixed
  *                      order, so the result is bitwise repeatable.
  *   SLIKL_DK_AUTO      the key-major path when it is possible, the key range is at most 16x
@@ -169,8 +172,8 @@ typedef struct {
     void *fused_begin;   /* optional cudaEvent_t recorded just before the fused kernel, or NULL */
     void *fused_end;     /* optional cudaEvent_t recorded just after it, or NULL */
     void *dk_begin;      /* optional cudaEvent_t recorded before the dK stage that follows the
-                            fused kernel (key-major kernel and cast, the cast alone, or the
-                            deterministic reduction), or NULL */
+                            fused kernel (w-scaled q, key-major kernel and cast, the cast alone,
+                            or the deterministic reduction), or NULL */
     void *dk_end;        /* optional cudaEvent_t recorded after that stage, or NULL */
     float *loss;         /* optional DEVICE output, fp32 [T1] (4-byte aligned), or NULL: the KL
                             loss per query row, L_t = sum over valid slots with p > 0 of
