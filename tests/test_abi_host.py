@@ -196,6 +196,13 @@ def test_keymajor_workspace_holds_the_records(lib):
     rc_k, n_k = ws_ex(lib, pr, "keymajor")
     assert rc_s == rc_k == sli.SLIKL_OK
     assert n_k - n_s >= 4096 * 4096 * 16
+    # plus the w-scaled copy of q (T1 x N1 x D elements of the input type): the key-major
+    # workspace grows with N1 beyond the records' own growth
+    rc_k16, n_k16 = ws_ex(lib, base_problem(N1=16), "keymajor")
+    rc_k48, n_k48 = ws_ex(lib, base_problem(N1=48), "keymajor")
+    assert rc_k16 == rc_k48 == sli.SLIKL_OK
+    assert n_k48 - n_k16 >= 4096 * 32 * 128 * 2 + 4096 * 4096 * (16 - 8)
+    assert n_k - n_s >= 4096 * 4096 * 16 + 4096 * 64 * 128 * 2
     pr32 = base_problem(N1=32, S2=1000)        # 8-byte records, rows rounded up to 1024 keys
     rc, n32 = ws_ex(lib, pr32, "keymajor")
     assert rc == sli.SLIKL_OK and n32 - ws_ex(lib, pr32, "scatter")[1] >= 4096 * 1024 * 8
